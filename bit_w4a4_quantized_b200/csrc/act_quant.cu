@@ -1,0 +1,424 @@
+// act_quant.cu -- kernel 1: smoothing, NVFP4 quantization and low-rank down projection of X
+// in one pass over X.
+//
+// SVDQuant summary page, section 4.3 "Nunchaku" (Figure 6(b)): the down
+// projection of the low-rank branch shares the activation read of the
+// quantization kernel, so X leaves HBM once.  Per 16 elements along K:
+//   x_hat = bf16(x * (1/lambda))                           (section 4.2 smoothing)
+//   s_b   = E4M3(amax|x_hat| * c_a),  c_a = 1 / (6 g_a)     (section 3 quantizer,
+//   d     = value(s_b) * g_a,  code = E2M1(x_hat * rcp(d))   q_max = 6, per block)
+// and lr' = bf16((x_hat L1) / (g_a g_w)) on the tensor cores.
+//
+// Design (sm_100a):
+//   * CTA = 128 rows of X x a slice of K.  Warp 4 streams X chunks of 128 rows
+//     x 64 columns with a 2D TMA load (128-byte swizzle), the matching
+//     1/lambda slice and L1^T chunk with bulk copies, through a 4-stage
+//     mbarrier ring.
+//   * Warps 0-3: one thread per row converts its 64 elements in shared
+//     memory, writes x_hat back in place (it is the A operand of the MMA),
+//     and stores codes and block scales straight into the GEMM's tiled layout.
+//   * Warp 5: one thread issues tcgen05.mma kind::f16 (M = 128, N = rank)
+//     accumulating X_hat L1 in tensor memory.
+//   * K is split across the CTAs of a cluster so that enough CTAs stream HBM;
+//     their partial X_hat L1 tiles are summed in a fixed order through
+//     distributed shared memory (no global scratch, deterministic).
+//   * Every wait is bounded; a timeout sets the layer's status word and the
+//     CTA drains its copies and MMAs, frees tensor memory and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace svdq {
+
+namespace {
+
+using namespace ptx;
+
+constexpr int kStages1 = 4;
+constexpr int kThreads1 = 192;
+constexpr uint32_t kXBytes = kBM * 128;  // 16 KB: 128 rows x 64 bf16
+constexpr uint32_t kInvSlot = 1024;      // 64 floats of 1/lambda (256 B), padded for alignment
+constexpr uint32_t kCtrlBytes = 128;
+
+struct ActQuantParams {
+  const float* inv_lam;  // [KC * 64]
+  const uint8_t* l1t;    // L1^T chunks, rc16 rows of 128 B each
+  uint8_t* codes;        // act + off_codes
+  uint8_t* sf;           // act + off_sf
+  uint8_t* lr;           // act + off_lr
+  uint32_t* status;      // layer status word
+  int32_t MT, KT, KC, RJ, r_tot, rc16, splits;
+  uint32_t stage_bytes, tmem_cols;
+  float g_a, c_a, inv_alpha;
+  uint64_t timeout_ns;
+};
+
+// One 16-element block of one row: read x from the swizzled stage, write
+// x_hat back, return 8 bytes of E2M1 codes and the E4M3 block scale.
+__device__ __forceinline__ void quant_block(uint8_t* xrow, uint32_t t7, int g, const float* inv, float g_a,
+                                            float c_a, uint32_t& w0, uint32_t& w1, uint32_t& scale) {
+  uint4* p0 = reinterpret_cast<uint4*>(xrow + (((2u * g) ^ t7) << 4));
+  uint4* p1 = reinterpret_cast<uint4*>(xrow + (((2u * g + 1u) ^ t7) << 4));
+  const uint4 a = *p0, b = *p1;
+  const float4* iv = reinterpret_cast<const float4*>(inv);
+  const float4 i0 = iv[0], i1 = iv[1], i2 = iv[2], i3 = iv[3];
+  const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  const float il[16] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w,
+                        i2.x, i2.y, i2.z, i2.w, i3.x, i3.y, i3.z, i3.w};
+  uint32_t h[8];
+  float xh[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float lo = __fmul_rn(bf16lo(in[j]), il[2 * j]);
+    const float hi = __fmul_rn(bf16hi(in[j]), il[2 * j + 1]);
+    h[j] = f32x2_to_bf16x2(lo, hi);
+    xh[2 * j] = bf16lo(h[j]);
+    xh[2 * j + 1] = bf16hi(h[j]);
+    amax = fmaxf(amax, fmaxf(fabsf(xh[2 * j]), fabsf(xh[2 * j + 1])));
+  }
+  *p0 = make_uint4(h[0], h[1], h[2], h[3]);
+  *p1 = make_uint4(h[4], h[5], h[6], h[7]);
+  const uint32_t sc = f32_to_e4m3(__fmul_rn(amax, c_a));
+  const float d = __fmul_rn(e4m3_value(sc), g_a);
+  const float rcp = d == 0.0f ? 0.0f : __frcp_rn(d);
+  w0 = f32x8_to_e2m1(__fmul_rn(xh[0], rcp), __fmul_rn(xh[1], rcp), __fmul_rn(xh[2], rcp), __fmul_rn(xh[3], rcp),
+                     __fmul_rn(xh[4], rcp), __fmul_rn(xh[5], rcp), __fmul_rn(xh[6], rcp), __fmul_rn(xh[7], rcp));
+  w1 = f32x8_to_e2m1(__fmul_rn(xh[8], rcp), __fmul_rn(xh[9], rcp), __fmul_rn(xh[10], rcp),
+                     __fmul_rn(xh[11], rcp), __fmul_rn(xh[12], rcp), __fmul_rn(xh[13], rcp),
+                     __fmul_rn(xh[14], rcp), __fmul_rn(xh[15], rcp));
+  scale = sc;
+}
+
+// Scale 8 fp32 ranks by 1/alpha, round to bf16, store 16 bytes of lr'.
+__device__ __forceinline__ void store_lr8(const ActQuantParams& p, int mt, uint32_t row, int c, const float* v) {
+  uint4 w;
+  w.x = f32x2_to_bf16x2(__fmul_rn(v[0], p.inv_alpha), __fmul_rn(v[1], p.inv_alpha));
+  w.y = f32x2_to_bf16x2(__fmul_rn(v[2], p.inv_alpha), __fmul_rn(v[3], p.inv_alpha));
+  w.z = f32x2_to_bf16x2(__fmul_rn(v[4], p.inv_alpha), __fmul_rn(v[5], p.inv_alpha));
+  w.w = f32x2_to_bf16x2(__fmul_rn(v[6], p.inv_alpha), __fmul_rn(v[7], p.inv_alpha));
+  uint8_t* tile = p.lr + (size_t(mt) * p.RJ + size_t(c / kRChunk)) * kATileBytes;
+  *reinterpret_cast<uint4*>(tile + sw128(row, uint32_t(c % kRChunk) * 2u)) = w;
+}
+
+__global__ void __launch_bounds__(kThreads1, 1)
+    act_quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const ActQuantParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_s + pad;
+
+  const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
+  const int split = int(blockIdx.x), mt = int(blockIdx.y);
+  const int kc0 = int(int64_t(split) * p.KC / p.splits);
+  const int kc1 = int(int64_t(split + 1) * p.KC / p.splits);
+  const int nchunks = kc1 - kc0;
+  const bool lowrank = p.r_tot > 0;
+
+  uint8_t* ctrl = smem + kStages1 * p.stage_bytes;
+  const uint32_t ctrl_s = sbase + kStages1 * p.stage_bytes;
+  const uint32_t FULL = ctrl_s, CONV = ctrl_s + 32u, EMPTY = ctrl_s + 64u;
+  const uint32_t ACCF = ctrl_s + 96u, DRAIN = ctrl_s + 104u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 112);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 116);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages1; ++s) {
+      mbar_init(FULL + 8u * s, 1);
+      mbar_init(CONV + 8u * s, 128);
+      mbar_init(EMPTY + 8u * s, 1);
+    }
+    mbar_init(ACCF, 1);
+    mbar_init(DRAIN, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 5 && lowrank) {
+    tmem_alloc(ctrl_s + 112u, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = lowrank ? *tmem_slot : 0u;
+
+  auto fail = [&](uint32_t code) {
+    *abort_flag = 1u;
+    atomicOr(p.status, code);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_x);
+      const uint32_t tx = kXBytes + 256u + (lowrank ? uint32_t(p.r_tot) * 128u : 0u);
+      int issued = 0;
+      for (int i = 0; i < nchunks; ++i) {
+        const int s = i % kStages1;
+        const uint32_t ph = uint32_t(i / kStages1) & 1u;
+        if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
+          fail(0x1u);
+          break;
+        }
+        const uint32_t st = sbase + uint32_t(s) * p.stage_bytes;
+        const int kc = kc0 + i;
+        mbar_expect_tx(FULL + 8u * s, tx);
+        tma_load_2d(st, &tmap_x, kc * kKChunk, mt * kBM, FULL + 8u * s);
+        bulk_g2s(st + kXBytes, p.inv_lam + size_t(kc) * kKChunk, 256u, FULL + 8u * s);
+        if (lowrank)
+          bulk_g2s(st + kXBytes + kInvSlot, p.l1t + size_t(kc) * size_t(p.rc16) * 128u, uint32_t(p.r_tot) * 128u,
+                   FULL + 8u * s);
+        issued = i + 1;
+      }
+      // every issued copy must land before this CTA may exit
+      for (int i = issued > kStages1 ? issued - kStages1 : 0; i < issued; ++i)
+        mbar_wait(FULL + 8u * (i % kStages1), uint32_t(i / kStages1) & 1u, nullptr, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ----------------------------------------------------------- converters
+    const uint32_t t = threadIdx.x;  // row inside the 128-row tile
+    const uint32_t t7 = t & 7u;
+    for (int i = 0; i < nchunks; ++i) {
+      const int s = i % kStages1;
+      const uint32_t ph = uint32_t(i / kStages1) & 1u;
+      if (!mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
+        fail(0x2u);
+        break;
+      }
+      uint8_t* stage = smem + size_t(s) * p.stage_bytes;
+      uint8_t* xrow = stage + t * 128u;
+      const float* inv = reinterpret_cast<const float*>(stage + kXBytes);
+      uint32_t cw[8], sc[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) quant_block(xrow, t7, g, inv + 16 * g, p.g_a, p.c_a, cw[2 * g], cw[2 * g + 1], sc[g]);
+      const int kc = kc0 + i, kt = kc >> 2, sub = kc & 3;
+      uint8_t* ctile = p.codes + (size_t(mt) * p.KT + kt) * kATileBytes;
+      *reinterpret_cast<uint4*>(ctile + sw128(t, uint32_t(sub) * 32u)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      *reinterpret_cast<uint4*>(ctile + sw128(t, uint32_t(sub) * 32u + 16u)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      uint8_t* stile = p.sf + (size_t(mt) * p.KT + kt) * kSFATileBytes + size_t(sub) * kSFAtomBytes;
+      *reinterpret_cast<uint32_t*>(stile + sf_atom(t, 0)) = sc[0] | (sc[1] << 8) | (sc[2] << 16) | (sc[3] << 24);
+      fence_proxy_async_smem();  // x_hat (generic writes) -> tensor-core reads
+      mbar_arrive(CONV + 8u * s);
+    }
+  } else {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      bool any = false;
+      const uint32_t idesc = idesc_bf16(p.r_tot);
+      for (int i = 0; i < nchunks; ++i) {
+        const int s = i % kStages1;
+        const uint32_t ph = uint32_t(i / kStages1) & 1u;
+        if (!mbar_wait(CONV + 8u * s, ph, abort_flag, p.timeout_ns)) {
+          fail(0x4u);
+          break;
+        }
+        if (lowrank) {
+          if (!mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
+            fail(0x4u);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xa = sbase + uint32_t(s) * p.stage_bytes;
+          const uint32_t la = xa + kXBytes + kInvSlot;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            umma_bf16(tmem, sdesc_sw128(xa + 32u * ks), sdesc_sw128(la + 32u * ks), idesc, (i | ks) ? 1u : 0u);
+          tc_commit(EMPTY + 8u * s);
+          any = true;
+        } else {
+          mbar_arrive(EMPTY + 8u * s);
+        }
+      }
+      if (any) {
+        tc_commit(ACCF);
+        tc_commit(DRAIN);
+        mbar_wait(DRAIN, 0u, nullptr, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  }
+
+  // ------------------------------------------------- low-rank output lr'
+  if (lowrank) {
+    const bool multi = p.splits > 1;
+    float* part = reinterpret_cast<float*>(smem);  // stages are idle now: [128][r_tot + 4]
+    const int pstride = p.r_tot + 4;
+    if (warp < 4) {
+      bool ok = (*abort_flag == 0u) && mbar_wait(ACCF, 0u, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t t = threadIdx.x;
+        const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+        for (int c = 0; c < p.r_tot; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + uint32_t(c), v);
+          tmem_wait_ld();
+          float f[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) f[j] = __uint_as_float(v[j]);
+          if (multi) {
+            float4* dst = reinterpret_cast<float4*>(part + size_t(t) * pstride + c);
+            dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+            dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+            dst[2] = make_float4(f[8], f[9], f[10], f[11]);
+            dst[3] = make_float4(f[12], f[13], f[14], f[15]);
+          } else {
+            store_lr8(p, mt, t, c, f);
+            store_lr8(p, mt, t, c + 8, f + 8);
+          }
+        }
+      } else if (*abort_flag == 0u) {
+        fail(0x8u);
+      }
+    }
+    if (multi) {
+      cluster_sync();  // every partial tile of the cluster is in shared memory
+      if (warp < 4 && *abort_flag == 0u) {
+        const int rows = (kBM + p.splits - 1) / p.splits;
+        const int rank = int(cluster_ctarank());
+        const int row0 = rank * rows;
+        const int row1 = row0 + rows < kBM ? row0 + rows : kBM;
+        const int groups = p.r_tot / 8;
+        for (int item = int(threadIdx.x); item < (row1 - row0) * groups; item += 128) {
+          const int row = row0 + item / groups, c = (item % groups) * 8;
+          const uint32_t off = uint32_t((row * pstride + c) * 4);
+          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          for (int q = 0; q < p.splits; ++q) {  // fixed order: deterministic sums
+            const uint32_t a = mapa(sbase + off, uint32_t(q));
+            const float4 v0 = ld_dsmem_f4(a), v1 = ld_dsmem_f4(a + 16u);
+            acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+            acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+          }
+          store_lr8(p, mt, uint32_t(row), c, acc);
+        }
+      }
+      cluster_sync();  // peers keep their shared memory until every read is done
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5 && lowrank) {
+    tc_fence_after();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+uint32_t next_pow2_at_least32(int v) {
+  uint32_t c = 32;
+  while (c < uint32_t(v)) c <<= 1;
+  return c;
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char** why) {
+  const LayerGeom& lg = a.lg;
+  const ActGeom ag = make_act_geom(lg, a.M);
+  if (ag.MT > 65535) {
+    *why = "M too large for one launch (more than 65535 tiles of 128 rows)";
+    return cudaErrorInvalidValue;
+  }
+  auto encode = tensor_map_encoder();
+  if (!encode) {
+    *why = "cuTensorMapEncodeTiled is not available from the driver";
+    return cudaErrorNotSupported;
+  }
+  alignas(64) CUtensorMap map;
+  const cuuint64_t dims[2] = {cuuint64_t(lg.K), cuuint64_t(a.M)};
+  const cuuint64_t strides[1] = {cuuint64_t(lg.K) * 2u};
+  const cuuint32_t box[2] = {uint32_t(kKChunk), uint32_t(kBM)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult cr = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.X), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    *why = "cuTensorMapEncodeTiled rejected the X operand";
+    return cudaErrorInvalidValue;
+  }
+
+  ActQuantParams p{};
+  p.inv_lam = reinterpret_cast<const float*>(a.layer + lg.off_inv_lam);
+  p.l1t = a.layer + lg.off_l1t;
+  p.codes = a.act + ag.off_codes;
+  p.sf = a.act + ag.off_sf;
+  p.lr = a.act + ag.off_lr;
+  p.status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.layer) + lg.off_status);
+  p.MT = int32_t(ag.MT);
+  p.KT = int32_t(lg.KT);
+  p.KC = int32_t(lg.KC);
+  p.RJ = int32_t(lg.RJ);
+  p.r_tot = a.r_tot;
+  p.rc16 = int32_t(lg.RC16);
+  p.stage_bytes = uint32_t(round_up(kXBytes + kInvSlot + uint32_t(a.r_tot) * 128u, 1024));
+  p.tmem_cols = a.r_tot > 0 ? next_pow2_at_least32(a.r_tot) : 0u;
+  p.g_a = a.g_a;
+  p.c_a = a.c_a;
+  p.inv_alpha = a.inv_alpha;
+  p.timeout_ns = a.timeout_ns;
+
+  const size_t smem = size_t(kStages1) * p.stage_bytes + kCtrlBytes + 1024;
+  const int per_sm = smem <= 113 * 1024 ? 2 : 1;
+  int splits = int((int64_t(per_sm) * a.num_sms) / ag.MT);
+  const int max_splits = a.r_tot > 0 ? 8 : 64;  // the cluster reduction needs a portable cluster
+  if (splits > max_splits) splits = max_splits;
+  if (splits > p.KC) splits = p.KC;
+  if (splits < 1) splits = 1;
+  p.splits = splits;
+
+  {
+    // the attribute is per device: remember the largest value set on each
+    static std::atomic<size_t> smem_set[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::atomic<size_t>& done = smem_set[dev & 63];
+    if (smem > done.load()) {
+      cudaError_t e = cudaFuncSetAttribute(act_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (e != cudaSuccess) {
+        *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
+        return e;
+      }
+      done.store(smem);
+    }
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(splits), unsigned(ag.MT), 1);
+  cfg.blockDim = dim3(kThreads1, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (a.r_tot > 0 && splits > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, map, p);
+  if (e != cudaSuccess) *why = "launch of the activation kernel failed";
+  return e;
+}
+
+}  // namespace svdq

@@ -1,0 +1,297 @@
+// api.cpp -- the extern "C" entry points declared in include/svdq.h.
+//
+// Argument checking, device checks and marshalling only: the preparation
+// lives in prepare.cpp / svd.cpp, the hot path in act_quant.cu and gemm.cu.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <string>
+
+#include "kernels.h"
+#include "layer.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<int> g_arch_override{0};
+
+svdq_status fail(svdq_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+svdq_status cuda_fail(cudaError_t e, const char* what) {
+  std::string m = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return fail(SVDQ_ERR_CUDA, m);
+}
+
+// The kernels use tcgen05 / TMA forms that exist on sm_100 only.  Like the
+// Nunchaku-Lite loader (Diffusers page, "kernel variants per GPU generation"),
+// refuse other devices with a clear error instead of producing wrong output.
+svdq_status check_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0, sms = 0;
+  if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute(major)");
+  if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute(minor)");
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+  int sm = major * 10 + minor;
+  const int ov = g_arch_override.load();
+  if (ov > 0) sm = ov;
+  if (sm != 100)
+    return fail(SVDQ_ERR_UNSUPPORTED_DEVICE, "device " + std::to_string(dev) + " is sm_" + std::to_string(sm) +
+                                                 "; these kernels need sm_100 (B200/GB200)");
+  if (dev_out) *dev_out = dev;
+  if (sms_out) *sms_out = sms;
+  return SVDQ_OK;
+}
+
+svdq_status check_uploaded(const svdq_layer* L) {
+  if (!L) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is NULL");
+  if (!L->dev_buf) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer has not been uploaded (svdq_layer_upload)");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != L->device)
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "current device " + std::to_string(dev) + " differs from the layer's device " +
+                                               std::to_string(L->device));
+  return SVDQ_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int svdq_abi_version(void) { return SVDQ_ABI_VERSION; }
+
+const char* svdq_last_error(void) { return g_last_error.c_str(); }
+
+svdq_status svdq_calibrate_amax(const uint16_t* X, int64_t M, int64_t K, float* amax) {
+  if (!X || !amax) return fail(SVDQ_ERR_INVALID_ARGUMENT, "X and amax are required");
+  if (M < 0 || K < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "bad shape");
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k) {
+      const uint32_t u = uint32_t(X[m * K + k] & 0x7FFFu) << 16;
+      float f;
+      std::memcpy(&f, &u, 4);
+      amax[k] = std::max(amax[k], f);
+    }
+  return SVDQ_OK;
+}
+
+size_t svdq_layer_device_bytes(const svdq_prepare_desc* d) {
+  std::string err;
+  if (svdq::validate_desc(d, &err) != SVDQ_OK) {
+    g_last_error = err;
+    return 0;
+  }
+  return svdq::make_layer_geom(d->K, d->N, d->rank, d->rank_capacity).total;
+}
+
+svdq_status svdq_prepare_host(const svdq_prepare_desc* d, svdq_layer** out) {
+  std::string err;
+  svdq_status st = svdq::prepare_host(d, out, &err);
+  if (st != SVDQ_OK) return fail(st, err);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_layer_upload(svdq_layer* L, void* dev_buf, size_t dev_buf_bytes, void* stream) {
+  if (!L || !dev_buf) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and dev_buf are required");
+  if (!aligned(dev_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "dev_buf must be 256-byte aligned");
+  if (dev_buf_bytes < L->g.total)
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "dev_buf needs " + std::to_string(L->g.total) + " bytes");
+  int dev = 0, sms = 0;
+  svdq_status st = check_device(&dev, &sms);
+  if (st != SVDQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(dev_buf, L->image.data(), L->g.total, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(layer image)");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  L->dev_buf = dev_buf;
+  L->dev_bytes = dev_buf_bytes;
+  L->device = dev;
+  L->num_sms = sms;
+  L->r_tot = L->g.rank;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_prepare_weights(const svdq_prepare_desc* d, void* dev_buf, size_t dev_buf_bytes,
+                                 svdq_layer** out, void* stream) {
+  if (!out) return fail(SVDQ_ERR_INVALID_ARGUMENT, "out is NULL");
+  svdq_layer* L = nullptr;
+  svdq_status st = svdq_prepare_host(d, &L);
+  if (st != SVDQ_OK) return st;
+  st = svdq_layer_upload(L, dev_buf, dev_buf_bytes, stream);
+  if (st != SVDQ_OK) {
+    delete L;
+    return st;
+  }
+  *out = L;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_act_buffer_bytes(const svdq_layer* L, int64_t M, size_t* bytes) {
+  if (!L || !bytes) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and bytes are required");
+  if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
+  *bytes = svdq::make_act_geom(L->g, M).total;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, void* act_buf, size_t act_buf_bytes,
+                              void* stream) {
+  svdq_status st = check_uploaded(L);
+  if (st != SVDQ_OK) return st;
+  if (!X || !act_buf) return fail(SVDQ_ERR_INVALID_ARGUMENT, "X and act_buf are required");
+  if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
+  if (!aligned(X, 16)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "X must be 16-byte aligned");
+  if (!aligned(act_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf must be 256-byte aligned");
+  const size_t need = svdq::make_act_geom(L->g, M).total;
+  if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");
+  if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
+  svdq::ActQuantLaunch a{};
+  a.X = X;
+  a.layer = static_cast<const uint8_t*>(L->dev_buf);
+  a.act = static_cast<uint8_t*>(act_buf);
+  a.lg = L->g;
+  a.M = M;
+  a.r_tot = L->r_tot;
+  a.g_a = L->g_a;
+  a.c_a = L->c_a;
+  a.inv_alpha = L->inv_alpha;
+  a.num_sms = L->num_sms;
+  a.timeout_ns = svdq::kDefaultTimeoutNs;
+  const char* why = "";
+  cudaError_t e = svdq::launch_act_quant(a, static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_w4a4_linear(const svdq_layer* L, const void* act_buf, size_t act_buf_bytes, int64_t M, void* Y,
+                             int epilogue, void* stream) {
+  svdq_status st = check_uploaded(L);
+  if (st != SVDQ_OK) return st;
+  if (!act_buf || !Y) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf and Y are required");
+  if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
+  if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU_TANH)
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "unknown epilogue");
+  if (!aligned(Y, 16)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "Y must be 16-byte aligned");
+  if (!aligned(act_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf must be 256-byte aligned");
+  const size_t need = svdq::make_act_geom(L->g, M).total;
+  if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");
+  if (M * L->g.N > (int64_t(1) << 31) * 2 || M > (int64_t(1) << 31) - 1)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M too large");
+  if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
+  svdq::GemmLaunch a{};
+  a.act = static_cast<const uint8_t*>(act_buf);
+  a.layer = static_cast<const uint8_t*>(L->dev_buf);
+  a.Y = Y;
+  a.lg = L->g;
+  a.M = M;
+  a.r_tot = L->r_tot;
+  a.has_bias = L->has_bias ? 1 : 0;
+  a.epilogue = epilogue;
+  a.alpha = L->alpha;
+  a.num_sms = L->num_sms;
+  a.timeout_ns = svdq::kDefaultTimeoutNs;
+  const char* why = "";
+  cudaError_t e = svdq::launch_gemm(a, static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_lora_swap(svdq_layer* L, const void* A, const void* B, int32_t r_e, float scale, void* stream) {
+  svdq_status st = check_uploaded(L);
+  if (st != SVDQ_OK) return st;
+  if (r_e < 0 || r_e % 16) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "LoRA rank must be a multiple of 16");
+  if (L->g.rank + r_e > L->g.rcap)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank + LoRA rank exceeds rank_capacity (" + std::to_string(L->g.rcap) + ")");
+  if (r_e > 0 && (!A || !B)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "A and B are required");
+  if (!std::isfinite(scale)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "scale must be finite");
+  svdq::LoraLaunch a{};
+  a.layer = static_cast<uint8_t*>(L->dev_buf);
+  a.lg = L->g;
+  a.A = static_cast<const uint16_t*>(A);
+  a.B = static_cast<const uint16_t*>(B);
+  a.r_e = r_e;
+  a.scale = scale;
+  cudaError_t e = svdq::launch_lora_swap(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the LoRA swap kernel");
+  L->r_tot = L->g.rank + r_e;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_layer_export(const svdq_layer* L, int what, void* host_dst, size_t bytes) {
+  if (!L || !host_dst) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and host_dst are required");
+  std::string err;
+  svdq_status st = svdq::export_array(L, what, host_dst, bytes, &err);
+  if (st != SVDQ_OK) return fail(st, err);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_act_unpack(const svdq_layer* L, int64_t M, const void* act_host, size_t bytes, uint8_t* codes,
+                            uint8_t* scales, uint16_t* lr) {
+  if (!L || !act_host) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and act_host are required");
+  if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
+  std::string err;
+  svdq_status st = svdq::act_unpack(L, M, static_cast<const uint8_t*>(act_host), bytes, codes, scales, lr, &err);
+  if (st != SVDQ_OK) return fail(st, err);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_get_layer_info(const svdq_layer* L, svdq_layer_info* info) {
+  if (!L || !info) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and info are required");
+  info->K = L->g.K;
+  info->N = L->g.N;
+  info->rank = L->g.rank;
+  info->rank_total = L->r_tot;
+  info->rank_capacity = L->g.rcap;
+  info->format = L->format;
+  info->g_a = L->g_a;
+  info->g_w = L->g_w;
+  info->alpha = L->alpha;
+  info->device_bytes = L->g.total;
+  info->dev_buf = L->dev_buf;
+  info->device = L->device;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_poll_status(const svdq_layer* L, void* stream) {
+  svdq_status st = check_uploaded(L);
+  if (st != SVDQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  uint8_t* status = static_cast<uint8_t*>(L->dev_buf) + L->g.off_status;
+  cudaError_t e = cudaMemcpyAsync(&word, status, 4, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(status)");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  if (word == 0) return SVDQ_OK;
+  if ((e = cudaMemsetAsync(status, 0, 4, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  char buf[96];
+  std::snprintf(buf, sizeof buf, "a kernel gave up a bounded wait (status word 0x%x)", word);
+  return fail(SVDQ_ERR_TIMEOUT, buf);
+}
+
+void svdq_layer_destroy(svdq_layer* L) { delete L; }
+
+void svdq_test_override_device_arch(int sm) { g_arch_override.store(sm); }
+
+svdq_status svdq_test_bounded_wait(uint64_t timeout_ns, uint32_t* status_out, void* stream) {
+  if (!status_out) return fail(SVDQ_ERR_INVALID_ARGUMENT, "status_out is NULL");
+  svdq_status st = check_device(nullptr, nullptr);
+  if (st != SVDQ_OK) return st;
+  cudaError_t e = svdq::run_bounded_wait_test(timeout_ns, status_out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bounded-wait test kernel");
+  return SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// kernels.h -- host-side launch interface of the CUDA kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/svdq.h"
+#include "layout.h"
+
+namespace svdq {
+
+// Kernel 1: smoothing + NVFP4 quantization of X + down projection.
+struct ActQuantLaunch {
+  const void* X;         // device bf16 [M, K]
+  const uint8_t* layer;  // device layer image
+  uint8_t* act;          // device activation buffer
+  LayerGeom lg;
+  int64_t M;
+  int32_t r_tot;         // ranks in use (0: no low-rank branch)
+  float g_a, c_a, inv_alpha;
+  int num_sms;
+  uint64_t timeout_ns;
+};
+cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char** why);
+
+// Kernel 2: block-scaled NVFP4 GEMM + low-rank up projection + epilogue.
+struct GemmLaunch {
+  const uint8_t* act;    // device activation buffer (filled by kernel 1)
+  const uint8_t* layer;  // device layer image
+  void* Y;               // device bf16 [M, N]
+  LayerGeom lg;
+  int64_t M;
+  int32_t r_tot;
+  int32_t has_bias;
+  int32_t epilogue;
+  float alpha;
+  int num_sms;
+  uint64_t timeout_ns;
+};
+cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why);
+
+// LoRA attach/detach: rewrite ranks [rank, rank_capacity) of L1^T and L2^T.
+struct LoraLaunch {
+  uint8_t* layer;
+  LayerGeom lg;
+  const uint16_t* A;  // device bf16 [K, r_e] or NULL when r_e == 0
+  const uint16_t* B;  // device bf16 [r_e, N]
+  int32_t r_e;
+  float scale;
+};
+cudaError_t launch_lora_swap(const LoraLaunch& a, cudaStream_t s);
+
+// Test hook: bounded wait on an mbarrier nothing arrives on.
+cudaError_t run_bounded_wait_test(uint64_t timeout_ns, uint32_t* status_out, cudaStream_t s);
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+
+}  // namespace svdq

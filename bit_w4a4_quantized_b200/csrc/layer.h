@@ -1,0 +1,42 @@
+// layer.h -- the host-side handle of one prepared layer (internal to the library).
+#pragma once
+
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/svdq.h"
+#include "layout.h"
+
+struct svdq_layer {
+  svdq::LayerGeom g{};
+  int32_t format = SVDQ_FMT_NVFP4;
+  std::vector<uint8_t> image;  // device image in its base state (rank r, no adapter)
+  std::vector<float> lam, inv_lam;
+  std::vector<uint16_t> l1, l2;  // base factors, bf16 [K, r] and [r, N]
+  std::vector<float> r32;        // R as float [K, N] (kept only when asked)
+  std::vector<double> sigma;     // singular values (library SVD only)
+  double resid_f64 = -1.0, resid_bf16 = -1.0;
+  float g_a = 1.f, g_w = 1.f, alpha = 1.f, inv_alpha = 1.f, c_a = 1.f;
+  int32_t r_tot = 0;  // ranks in use: base rank + attached adapter rank
+  bool has_bias = false;
+  // device state (after upload)
+  void* dev_buf = nullptr;
+  size_t dev_bytes = 0;
+  int device = -1;
+  int num_sms = 0;
+};
+
+namespace svdq {
+
+// Host preparation (prepare.cpp).  Returns SVDQ_OK or an error with message.
+svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::string* err);
+svdq_status validate_desc(const svdq_prepare_desc* d, std::string* err);
+
+// Logical views of the image / of an activation buffer (prepare.cpp).
+svdq_status export_array(const svdq_layer* L, int what, void* dst, size_t bytes, std::string* err);
+svdq_status act_unpack(const svdq_layer* L, int64_t M, const uint8_t* act, size_t bytes, uint8_t* codes,
+                       uint8_t* scales, uint16_t* lr, std::string* err);
+
+}  // namespace svdq

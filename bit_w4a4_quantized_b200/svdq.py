@@ -1,0 +1,316 @@
+"""ctypes binding of libsvdq.so (the C ABI in include/svdq.h).
+
+Argument marshalling only: every step of the layer runs in the library (host
+preparation in C++, the forward pass in the CUDA kernels).  PyTorch supplies
+device memory and streams.  There is no fallback: if the library is missing
+or a call fails, an exception is raised.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libsvdq.so")
+
+OK = 0
+ERR_INVALID_ARGUMENT = 1
+ERR_UNSUPPORTED_SHAPE = 2
+ERR_UNSUPPORTED_DEVICE = 3
+ERR_BUFFER_TOO_SMALL = 4
+ERR_CUDA = 5
+ERR_TIMEOUT = 6
+ERR_INTERNAL = 7
+ERR_HOST_ALLOC = 8
+
+FMT_NVFP4 = 1
+PREPARE_KEEP_R = 1
+EPI_NONE = 0
+EPI_GELU_TANH = 1
+
+EXPORT_LAMBDA = 1
+EXPORT_INV_LAMBDA = 2
+EXPORT_L1 = 3
+EXPORT_L2 = 4
+EXPORT_R = 5
+EXPORT_W_CODES = 6
+EXPORT_W_SCALES = 7
+EXPORT_SIGMA = 8
+EXPORT_SCALARS = 9
+EXPORT_RESID_NORM = 10
+
+# every symbol include/svdq.h declares
+EXPORTED_SYMBOLS = (
+    "svdq_abi_version", "svdq_last_error", "svdq_calibrate_amax", "svdq_layer_device_bytes",
+    "svdq_prepare_host", "svdq_layer_upload", "svdq_prepare_weights", "svdq_act_buffer_bytes",
+    "svdq_quantize_act", "svdq_w4a4_linear", "svdq_lora_swap", "svdq_layer_export", "svdq_act_unpack",
+    "svdq_get_layer_info", "svdq_poll_status", "svdq_layer_destroy", "svdq_test_override_device_arch",
+    "svdq_test_bounded_wait",
+)
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"svdq status {status}: {message}")
+        self.status = status
+
+
+class PrepareDesc(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int64), ("N", ctypes.c_int64),
+        ("rank", ctypes.c_int32), ("rank_capacity", ctypes.c_int32),
+        ("format", ctypes.c_int32), ("num_threads", ctypes.c_int32), ("flags", ctypes.c_int32),
+        ("W", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("act_amax", ctypes.c_void_p),
+        ("L1", ctypes.c_void_p), ("L2", ctypes.c_void_p),
+        ("svd_seed", ctypes.c_uint64), ("svd_power_iters", ctypes.c_int32), ("svd_oversample", ctypes.c_int32),
+    ]
+
+
+class LayerInfo(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int64), ("N", ctypes.c_int64),
+        ("rank", ctypes.c_int32), ("rank_total", ctypes.c_int32), ("rank_capacity", ctypes.c_int32),
+        ("format", ctypes.c_int32),
+        ("g_a", ctypes.c_float), ("g_w", ctypes.c_float), ("alpha", ctypes.c_float),
+        ("device_bytes", ctypes.c_size_t), ("dev_buf", ctypes.c_void_p), ("device", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """Load libsvdq.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m bit_w4a4_quantized_b200.build` "
+                           "(or __graft_entry__.build()); there is no fallback implementation")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    st = ctypes.c_int
+    sig = {
+        "svdq_abi_version": ([], ctypes.c_int),
+        "svdq_last_error": ([], ctypes.c_char_p),
+        "svdq_calibrate_amax": ([vp, i64, i64, vp], st),
+        "svdq_layer_device_bytes": ([ctypes.POINTER(PrepareDesc)], sz),
+        "svdq_prepare_host": ([ctypes.POINTER(PrepareDesc), ctypes.POINTER(vp)], st),
+        "svdq_layer_upload": ([vp, vp, sz, vp], st),
+        "svdq_prepare_weights": ([ctypes.POINTER(PrepareDesc), vp, sz, ctypes.POINTER(vp), vp], st),
+        "svdq_act_buffer_bytes": ([vp, i64, ctypes.POINTER(sz)], st),
+        "svdq_quantize_act": ([vp, vp, i64, vp, sz, vp], st),
+        "svdq_w4a4_linear": ([vp, vp, sz, i64, vp, ctypes.c_int, vp], st),
+        "svdq_lora_swap": ([vp, vp, vp, i32, ctypes.c_float, vp], st),
+        "svdq_layer_export": ([vp, ctypes.c_int, vp, sz], st),
+        "svdq_act_unpack": ([vp, i64, vp, sz, vp, vp, vp], st),
+        "svdq_get_layer_info": ([vp, ctypes.POINTER(LayerInfo)], st),
+        "svdq_poll_status": ([vp, vp], st),
+        "svdq_layer_destroy": ([vp], None),
+        "svdq_test_override_device_arch": ([ctypes.c_int], None),
+        "svdq_test_bounded_wait": ([ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32), vp], st),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def last_error():
+    return lib().svdq_last_error().decode()
+
+
+def check(status):
+    if status != OK:
+        raise SvdqError(status, last_error())
+
+
+def _ptr(a):
+    """Data pointer of a numpy array or torch tensor (None -> NULL)."""
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        return a.ctypes.data
+    return a.data_ptr()  # torch.Tensor
+
+
+def _bf16_bits(a):
+    """Host bf16 data as a contiguous uint16 numpy array."""
+    if a is None:
+        return None
+    if not isinstance(a, np.ndarray):  # torch tensor
+        import torch
+
+        a = a.detach().to("cpu").contiguous()
+        if a.dtype == torch.bfloat16:
+            return a.view(torch.int16).numpy().view(np.uint16).copy()
+        a = a.numpy()
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray(a)
+    if a.dtype.name == "bfloat16":
+        return np.ascontiguousarray(a).view(np.uint16)
+    raise TypeError(f"expected bfloat16 data, got {a.dtype}")
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def calibrate_amax(X, amax=None):
+    """Running max_i |X_ij| over a host bf16 [M, K] batch (the library's calibration)."""
+    x = _bf16_bits(X)
+    M, K = x.shape
+    if amax is None:
+        amax = np.zeros(K, np.float32)
+    check(lib().svdq_calibrate_amax(_ptr(x), M, K, _ptr(amax)))
+    return amax
+
+
+class Layer:
+    """One prepared SVDQuant W4A4 + low-rank layer (host handle + device image)."""
+
+    def __init__(self, W, act_amax, rank, *, rank_capacity=None, bias=None, factors=None, seed=0, threads=0,
+                 keep_r=False, power_iters=0, oversample=0, device=None, stream=None):
+        self._h = None
+        w = _bf16_bits(W)
+        self.N, self.K = w.shape
+        amax = np.ascontiguousarray(np.asarray(act_amax, dtype=np.float32))
+        b = _bf16_bits(bias)
+        l1 = l2 = None
+        if factors is not None:
+            l1, l2 = _bf16_bits(factors[0]), _bf16_bits(factors[1])
+        self._keep = (w, amax, b, l1, l2)  # alive during the call
+        d = PrepareDesc()
+        d.K, d.N, d.rank = self.K, self.N, rank
+        d.rank_capacity = rank if rank_capacity is None else rank_capacity
+        d.format = FMT_NVFP4
+        d.num_threads = threads
+        d.flags = PREPARE_KEEP_R if keep_r else 0
+        d.W, d.bias, d.act_amax = _ptr(w), _ptr(b), _ptr(amax)
+        d.L1, d.L2 = _ptr(l1), _ptr(l2)
+        d.svd_seed, d.svd_power_iters, d.svd_oversample = seed, power_iters, oversample
+        self.desc = d
+        self.device_bytes = lib().svdq_layer_device_bytes(ctypes.byref(d))
+        if self.device_bytes == 0:
+            raise SvdqError(ERR_INVALID_ARGUMENT, last_error())
+        h = ctypes.c_void_p()
+        check(lib().svdq_prepare_host(ctypes.byref(d), ctypes.byref(h)))
+        self._h = h
+        self._keep = None
+        self.rank = rank
+        self.dev_buf = None
+        if device is not None:
+            self.upload(device, stream)
+
+    # ------------------------------------------------------------- device side
+    def upload(self, device="cuda", stream=None):
+        import torch
+
+        self.dev_buf = torch.empty(self.device_bytes, dtype=torch.uint8, device=device)
+        with torch.cuda.device(self.dev_buf.device):
+            check(lib().svdq_layer_upload(self._h, self.dev_buf.data_ptr(), self.device_bytes, _stream(stream)))
+        return self
+
+    def act_buffer_bytes(self, M):
+        n = ctypes.c_size_t()
+        check(lib().svdq_act_buffer_bytes(self._h, M, ctypes.byref(n)))
+        return n.value
+
+    def new_act_buffer(self, M):
+        import torch
+
+        return torch.empty(self.act_buffer_bytes(M), dtype=torch.uint8, device=self.dev_buf.device)
+
+    def quantize_act(self, X, act=None, stream=None):
+        """Kernel 1 on a device bf16 [M, K] tensor; returns the activation buffer."""
+        M = X.shape[0]
+        if act is None:
+            act = self.new_act_buffer(M)
+        if not X.is_contiguous():
+            raise ValueError("X must be contiguous")
+        check(lib().svdq_quantize_act(self._h, X.data_ptr(), M, act.data_ptr(), act.numel(), _stream(stream)))
+        return act
+
+    def linear(self, act, M, out=None, epilogue=EPI_NONE, stream=None):
+        """Kernel 2; returns Y bf16 [M, N]."""
+        import torch
+
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=act.device)
+        check(lib().svdq_w4a4_linear(self._h, act.data_ptr(), act.numel(), M, out.data_ptr(), epilogue,
+                                     _stream(stream)))
+        return out
+
+    def forward(self, X, out=None, epilogue=EPI_NONE, act=None, stream=None):
+        act = self.quantize_act(X, act, stream)
+        return self.linear(act, X.shape[0], out, epilogue, stream)
+
+    def lora_swap(self, A=None, B=None, scale=1.0, stream=None):
+        """Attach a LoRA (device bf16 A [K, r_e], B [r_e, N]); A=None detaches."""
+        r_e = 0 if A is None else A.shape[1]
+        check(lib().svdq_lora_swap(self._h, _ptr(A), _ptr(B), r_e, float(scale), _stream(stream)))
+
+    def poll_status(self, stream=None):
+        check(lib().svdq_poll_status(self._h, _stream(stream)))
+
+    # --------------------------------------------------------------- host side
+    def info(self):
+        i = LayerInfo()
+        check(lib().svdq_get_layer_info(self._h, ctypes.byref(i)))
+        return i
+
+    def export(self, what):
+        K, N, r = self.K, self.N, self.rank
+        shapes = {
+            EXPORT_LAMBDA: ((K,), np.float32), EXPORT_INV_LAMBDA: ((K,), np.float32),
+            EXPORT_L1: ((K, r), np.uint16), EXPORT_L2: ((r, N), np.uint16),
+            EXPORT_R: ((K, N), np.float32), EXPORT_W_CODES: ((N, K // 2), np.uint8),
+            EXPORT_W_SCALES: ((N, K // 16), np.uint8), EXPORT_SIGMA: ((r,), np.float64),
+            EXPORT_SCALARS: ((4,), np.float32), EXPORT_RESID_NORM: ((2,), np.float64),
+        }
+        shape, dt = shapes[what]
+        out = np.empty(shape, dtype=dt)
+        check(lib().svdq_layer_export(self._h, what, out.ctypes.data, out.nbytes))
+        return out
+
+    def act_unpack(self, act_host, M):
+        """Logical codes [M, K/2], scales [M, K/16], lr bf16 bits [M, r_tot] of a host copy."""
+        a = np.ascontiguousarray(np.asarray(act_host, dtype=np.uint8))
+        rt = self.info().rank_total
+        codes = np.empty((M, self.K // 2), np.uint8)
+        scales = np.empty((M, self.K // 16), np.uint8)
+        lr = np.empty((M, rt), np.uint16)
+        check(lib().svdq_act_unpack(self._h, M, a.ctypes.data, a.nbytes, codes.ctypes.data, scales.ctypes.data,
+                                    lr.ctypes.data if rt else None))
+        return codes, scales, lr
+
+    def close(self):
+        if self._h is not None and _lib is not None:
+            _lib.svdq_layer_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def test_bounded_wait(timeout_ns, stream=None):
+    """Run the library's bounded-wait test kernel; returns its status word."""
+    out = ctypes.c_uint32(0)
+    check(lib().svdq_test_bounded_wait(timeout_ns, ctypes.byref(out), _stream(stream)))
+    return out.value
+
+
+def override_device_arch(sm):
+    lib().svdq_test_override_device_arch(int(sm))

@@ -1,0 +1,251 @@
+/*
+ * svdq.h -- C ABI of the SVDQuant W4A4 + low-rank linear layer for B200 (sm_100a).
+ *
+ * The layer (SVDQuant summary page, hoonably.github.io/blog/svdquant,
+ * section 4.2 "SVDQuant: absorbing outliers via low-rank branch", eq. for XW):
+ *
+ *     Y = act( Q(X diag(lambda)^-1) Q(R) + (X diag(lambda)^-1 L1) L2 + b ),
+ *     R = diag(lambda) W^T - L1 L2,
+ *
+ * with W in nn.Linear layout [N, K], L1 [K, r] and L2 [r, N] the top-r SVD
+ * factors of the smoothed weight (L1 = U_r Sigma_r, L2 = V_r^T, same section),
+ * Q the NVFP4 quantizer (E2M1 elements, one E4M3 scale per 16 consecutive
+ * elements along K, one float32 scale per tensor; the page's quantizer of
+ * section 3 "Quantization preliminary" with q_max = 6, applied per block),
+ * and act either the identity or tanh-GELU.
+ *
+ * Conventions for every entry point:
+ *   - Return value: svdq_status.  No entry point aborts, exits or traps; on
+ *     failure a message is left in svdq_last_error() (thread local).
+ *   - Device memory is owned by the caller (allocate it with PyTorch, cudaMalloc,
+ *     a pool...).  The library never allocates device memory.  The layer handle
+ *     owns host memory only.
+ *   - Streams are cudaStream_t values passed as void*; NULL is the legacy
+ *     default stream.  Launching entry points are asynchronous and stream
+ *     ordered unless stated otherwise.
+ *   - bf16 arrays are passed as raw 16-bit patterns (uint16_t / void*).
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified (but memory-safe)
+ *     results.
+ *   - Shapes: K and N multiples of 64, rank and LoRA rank multiples of 16,
+ *     rank capacity <= 256, any M >= 1 (partial tiles are masked).
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SVDQ_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARGUMENT = 1,  /* null pointer, M < 1, bad enum value        */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2, /* K or N % 64, rank % 16, rank > capacity ... */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 3,/* not an sm_100 device (the pages: a capability
+                                     check must fail loudly rather than return
+                                     wrong output -- Diffusers/Nunchaku page,
+                                     "kernel variants per GPU generation")       */
+  SVDQ_ERR_BUFFER_TOO_SMALL = 4,  /* a caller buffer is smaller than required    */
+  SVDQ_ERR_CUDA = 5,              /* a CUDA runtime call failed                  */
+  SVDQ_ERR_TIMEOUT = 6,           /* a kernel's bounded wait ran out (see poll)  */
+  SVDQ_ERR_INTERNAL = 7,          /* a library invariant was violated            */
+  SVDQ_ERR_HOST_ALLOC = 8         /* host memory allocation failed               */
+} svdq_status;
+
+typedef struct svdq_layer svdq_layer; /* opaque host handle of one prepared layer */
+
+enum { SVDQ_FMT_NVFP4 = 1 };
+enum { SVDQ_PREPARE_KEEP_R = 1 /* keep float32 R in the handle for SVDQ_EXPORT_R */ };
+enum { SVDQ_EPI_NONE = 0, SVDQ_EPI_GELU_TANH = 1 };
+
+/*
+ * Offline preparation parameters (the quantize step of the Diffusers page's
+ * calibrate / quantize / package workflow; its "--precision nvfp4" and
+ * "--rank" flags are `format` and `rank`).
+ */
+typedef struct svdq_prepare_desc {
+  int64_t K;               /* in features, multiple of 64                          */
+  int64_t N;               /* out features, multiple of 64 (a fused QKV layer is
+                              W_q, W_k, W_v concatenated along N in that order)    */
+  int32_t rank;            /* r of the low-rank branch, multiple of 16, may be 0   */
+  int32_t rank_capacity;   /* >= rank, multiple of 16, <= 256: room for LoRA ranks */
+  int32_t format;          /* SVDQ_FMT_NVFP4                                       */
+  int32_t num_threads;     /* host threads for preparation; 0 = all cores          */
+  int32_t flags;           /* SVDQ_PREPARE_* bits                                  */
+  const uint16_t* W;       /* host bf16 [N, K] row-major (nn.Linear weight)        */
+  const uint16_t* bias;    /* host bf16 [N], or NULL                               */
+  const float* act_amax;   /* host float [K]: max_i |X_ij| over calibration rows
+                              (see svdq_calibrate_amax); sets lambda and the static
+                              activation tensor scale                               */
+  const uint16_t* L1;      /* optional host bf16 [K, rank]: use these low-rank
+                              factors (e.g. from a checkpoint) instead of the
+                              library's SVD; NULL = compute them                   */
+  const uint16_t* L2;      /* optional host bf16 [rank, N]; both or neither        */
+  uint64_t svd_seed;       /* seed of the randomized SVD's test matrix             */
+  int32_t svd_power_iters; /* subspace iterations, 0 = default (8)                 */
+  int32_t svd_oversample;  /* extra columns of the sketch, 0 = default (16)        */
+} svdq_prepare_desc;
+
+/* Library version of this header (SVDQ_ABI_VERSION). */
+SVDQ_API int svdq_abi_version(void);
+
+/* Thread-local message of the last failure in this thread ("" if none). */
+SVDQ_API const char* svdq_last_error(void);
+
+/*
+ * Calibration statistic: amax[j] = max(amax[j], max_i |X_ij|) over the M rows
+ * of a host bf16 [M, K] batch.  Initialise amax to zeros before the first
+ * batch.  Host only; no CUDA call.
+ */
+SVDQ_API svdq_status svdq_calibrate_amax(const uint16_t* X, int64_t M, int64_t K, float* amax);
+
+/*
+ * Bytes of device memory a layer with this descriptor needs (weights, scales,
+ * smoothing factors, low-rank factors at rank_capacity, bias, status word).
+ * Returns 0 if the descriptor is invalid (svdq_last_error says why).
+ */
+SVDQ_API size_t svdq_layer_device_bytes(const svdq_prepare_desc* d);
+
+/*
+ * Host half of the preparation, no CUDA call (usable without a GPU):
+ *   lambda_j = sqrt(act_amax_j / max_n |W_nj|) (1 where either is 0), float32;
+ *   W_hat^T = diag(lambda) W^T; top-r factors by randomized subspace iteration
+ *   (Halko, Martinsson & Tropp 2011) + one-sided Jacobi SVD, rounded to bf16
+ *   (or the caller's L1/L2); R = W_hat^T - L1 L2 in float64; NVFP4 of R^T with
+ *   g_w = max|R| / 2688; static activation scale g_a from act_amax.
+ * (SVDQuant summary page, section 4.2.)  The result is packed into the
+ * device image (tiled, swizzled layouts of the kernels) held by the handle.
+ * *out must be released with svdq_layer_destroy.
+ */
+SVDQ_API svdq_status svdq_prepare_host(const svdq_prepare_desc* d, svdq_layer** out);
+
+/*
+ * Device half: checks the current device is sm_100 (SVDQ_ERR_UNSUPPORTED_DEVICE
+ * otherwise), copies the image into dev_buf (>= svdq_layer_device_bytes,
+ * 256-byte aligned) on stream s and synchronizes s.  The handle remembers
+ * dev_buf and the current device; dev_buf must outlive the handle's use.
+ */
+SVDQ_API svdq_status svdq_layer_upload(svdq_layer* layer, void* dev_buf, size_t dev_buf_bytes, void* stream);
+
+/* svdq_prepare_host followed by svdq_layer_upload. */
+SVDQ_API svdq_status svdq_prepare_weights(const svdq_prepare_desc* d, void* dev_buf, size_t dev_buf_bytes,
+                                 svdq_layer** out, void* stream);
+
+/*
+ * Bytes of the per-call activation buffer for M tokens: NVFP4 codes and block
+ * scales of X_hat in the GEMM's tiled layout, and the bf16 down-projection
+ * lr' = (X_hat L1) / (g_a g_w) for rank_capacity ranks.  Host only.
+ */
+SVDQ_API svdq_status svdq_act_buffer_bytes(const svdq_layer* layer, int64_t M, size_t* bytes);
+
+/*
+ * Kernel 1 (Nunchaku fusion of the down projection into the quantizer,
+ * SVDQuant summary page section 4.3 / Figure 6(b)).  One pass over X:
+ *   x_hat = bf16(x / lambda); per 16 elements along K: E4M3 block scale,
+ *   E2M1 codes; lr' = bf16((x_hat L1) / (g_a g_w)) on the tensor cores.
+ * X: device bf16 [M, K] row-major, 16-byte aligned, row stride K.
+ * act_buf: device, >= svdq_act_buffer_bytes(M) bytes, 256-byte aligned.
+ */
+SVDQ_API svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, int64_t M, void* act_buf,
+                              size_t act_buf_bytes, void* stream);
+
+/*
+ * Kernel 2 (Nunchaku fusion of the up projection into the 4-bit GEMM, same
+ * section): Y = act(g_a g_w (Q(X_hat) Q(R) + lr' L2) + b) with the FP4
+ * block-scaled MMA and the bf16 up projection accumulating into the same
+ * tensor-memory tile.
+ * act_buf: the buffer svdq_quantize_act filled for the same M.
+ * Y: device bf16 [M, N] row-major, 16-byte aligned.
+ * epilogue: SVDQ_EPI_NONE or SVDQ_EPI_GELU_TANH (bias is added first).
+ */
+SVDQ_API svdq_status svdq_w4a4_linear(const svdq_layer* layer, const void* act_buf, size_t act_buf_bytes,
+                             int64_t M, void* Y, int epilogue, void* stream);
+
+/*
+ * Attach a LoRA adapter to the low-rank branch without touching R (abstract of
+ * arXiv 2411.05007: off-the-shelf LoRAs without re-quantization).  Device
+ * bf16 A [K, r_e] and B [r_e, N] (row-major); the layer computes
+ * Y += scale X A B by storing L1' = [L1 | bf16(lambda A scale)], L2' = [L2 ; B].
+ * r_e = 0 detaches the current adapter.  rank + r_e <= rank_capacity.
+ * Stream ordered, no host synchronization; calls on `layer` issued after this
+ * one (on any stream ordered after s) see the new rank.  Not thread safe
+ * against concurrent calls on the same handle.
+ */
+SVDQ_API svdq_status svdq_lora_swap(svdq_layer* layer, const void* A, const void* B, int32_t r_e, float scale,
+                           void* stream);
+
+/* What svdq_layer_export can copy out (logical, unswizzled layouts). */
+enum {
+  SVDQ_EXPORT_LAMBDA = 1,     /* float [K]                                        */
+  SVDQ_EXPORT_INV_LAMBDA = 2, /* float [K]                                        */
+  SVDQ_EXPORT_L1 = 3,         /* bf16 [K, rank] (base factors)                    */
+  SVDQ_EXPORT_L2 = 4,         /* bf16 [rank, N]                                   */
+  SVDQ_EXPORT_R = 5,          /* float [K, N] = float32(R)                        */
+  SVDQ_EXPORT_W_CODES = 6,    /* uint8 [N, K/2] E2M1 codes of R^T, element 2i in
+                                 the low nibble                                   */
+  SVDQ_EXPORT_W_SCALES = 7,   /* uint8 [N, K/16] E4M3 block scales                */
+  SVDQ_EXPORT_SIGMA = 8,      /* double [rank] singular values (library SVD only) */
+  SVDQ_EXPORT_SCALARS = 9,    /* float [4]: g_a, g_w, alpha = g_a g_w, 1/alpha    */
+  SVDQ_EXPORT_RESID_NORM = 10 /* double [2]: ||W_hat^T - L1 L2||_F with float64
+                                 factors, and with the bf16 factors               */
+};
+
+/* Copy one prepared array from the handle's host image into host_dst. */
+SVDQ_API svdq_status svdq_layer_export(const svdq_layer* layer, int what, void* host_dst, size_t bytes);
+
+/*
+ * Unpack a host copy of an activation buffer (M rows) into logical layouts:
+ * codes uint8 [M, K/2], scales uint8 [M, K/16], lr bf16 [M, rank_total]
+ * (rank_total = rank + attached LoRA rank).  Any output may be NULL.
+ */
+SVDQ_API svdq_status svdq_act_unpack(const svdq_layer* layer, int64_t M, const void* act_host, size_t bytes,
+                            uint8_t* codes, uint8_t* scales, uint16_t* lr);
+
+typedef struct svdq_layer_info {
+  int64_t K, N;
+  int32_t rank, rank_total, rank_capacity, format;
+  float g_a, g_w, alpha;
+  size_t device_bytes;
+  void* dev_buf;  /* NULL before upload */
+  int32_t device; /* CUDA ordinal, -1 before upload */
+} svdq_layer_info;
+
+SVDQ_API svdq_status svdq_get_layer_info(const svdq_layer* layer, svdq_layer_info* info);
+
+/*
+ * Read and clear the layer's device status word (synchronizes `stream`).
+ * SVDQ_ERR_TIMEOUT if any kernel of this layer gave up a bounded wait since the
+ * last poll (its outputs are then invalid), SVDQ_OK otherwise.
+ */
+SVDQ_API svdq_status svdq_poll_status(const svdq_layer* layer, void* stream);
+
+/* Free the handle's host memory (the caller frees dev_buf). NULL is a no-op. */
+SVDQ_API void svdq_layer_destroy(svdq_layer* layer);
+
+/*
+ * Test hooks.
+ * svdq_test_override_device_arch: pretend the device reports this sm version
+ * (e.g. 90) in the capability checks; 0 restores the real query.
+ * svdq_test_bounded_wait: launch a one-CTA kernel that waits, with the same
+ * bounded-wait routine the kernels use, on an mbarrier nothing arrives on, for
+ * at most timeout_ns; writes the kernel's status word (nonzero = gave up) to
+ * *status_out and synchronizes the stream.  Faults, traps or hangs nothing.
+ */
+SVDQ_API void svdq_test_override_device_arch(int sm);
+SVDQ_API svdq_status svdq_test_bounded_wait(uint64_t timeout_ns, uint32_t* status_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H */

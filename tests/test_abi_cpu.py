@@ -1,0 +1,116 @@
+"""The C ABI without a GPU: the library loads, exports exactly what
+include/svdq.h declares, validates arguments, and its host-only entry points
+work (no CUDA call is made by these tests)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from bit_w4a4_quantized_b200 import svdq
+from bit_w4a4_quantized_b200 import workloads as WL
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    return sorted(set(re.findall(r"^SVDQ_API\s+[\w\s\*]+?\b(svdq_\w+)\(", text, flags=re.M)))
+
+
+def test_library_loads_and_reports_version():
+    assert svdq.lib().svdq_abi_version() == 1
+
+
+def test_exports_match_header():
+    decl = declared_symbols()
+    assert len(decl) >= 18
+    assert sorted(svdq.EXPORTED_SYMBOLS) == decl
+    L = svdq.lib()
+    for name in decl:
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", svdq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted(l.split()[-1] for l in out.splitlines() if " T " in l and "svdq_" in l)
+    assert exported == decl
+
+
+def _desc(K=256, N=256, rank=16, cap=16):
+    W = WL.make_w(N, K, seed=0).view(np.uint16)
+    amax = np.ones(K, np.float32)
+    d = svdq.PrepareDesc()
+    d.K, d.N, d.rank, d.rank_capacity, d.format = K, N, rank, cap, svdq.FMT_NVFP4
+    d.W, d.act_amax = W.ctypes.data, amax.ctypes.data
+    return d, (W, amax)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("K", 100, svdq.ERR_UNSUPPORTED_SHAPE),
+    ("N", 0, svdq.ERR_UNSUPPORTED_SHAPE),
+    ("rank", 8, svdq.ERR_UNSUPPORTED_SHAPE),
+    ("rank_capacity", 8, svdq.ERR_UNSUPPORTED_SHAPE),
+    ("rank_capacity", 512, svdq.ERR_UNSUPPORTED_SHAPE),
+    ("format", 7, svdq.ERR_INVALID_ARGUMENT),
+    ("W", None, svdq.ERR_INVALID_ARGUMENT),
+])
+def test_prepare_rejects_bad_descriptors(field, value, status):
+    d, keep = _desc()
+    setattr(d, field, value)
+    h = ctypes.c_void_p()
+    st = svdq.lib().svdq_prepare_host(ctypes.byref(d), ctypes.byref(h))
+    assert st == status
+    assert svdq.last_error()
+    assert svdq.lib().svdq_layer_device_bytes(ctypes.byref(d)) == 0
+    del keep
+
+
+def test_null_arguments_are_errors_not_crashes():
+    L = svdq.lib()
+    assert L.svdq_prepare_host(None, None) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_act_buffer_bytes(None, 4, None) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_layer_export(None, 1, None, 0) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_act_unpack(None, 1, None, 0, None, None, None) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_quantize_act(None, None, 1, None, 0, None) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_w4a4_linear(None, None, 0, 1, None, 0, None) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_lora_swap(None, None, None, 0, 1.0, None) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_poll_status(None, None) == svdq.ERR_INVALID_ARGUMENT
+    L.svdq_layer_destroy(None)
+
+
+def test_host_only_layer_cannot_launch():
+    spec = WL.CFG1
+    X = spec.x()
+    layer = svdq.Layer(spec.w(), np.max(np.abs(X.astype(np.float32)), 0), spec.rank)
+    st = svdq.lib().svdq_quantize_act(layer._h, 16, 64, 256, 1 << 20, None)
+    assert st == svdq.ERR_INVALID_ARGUMENT
+    assert "uploaded" in svdq.last_error()
+    buf = np.zeros(16, np.uint8)
+    assert svdq.lib().svdq_layer_export(layer._h, 99, buf.ctypes.data, 16) == svdq.ERR_INVALID_ARGUMENT
+    assert svdq.lib().svdq_layer_export(layer._h, svdq.EXPORT_LAMBDA, buf.ctypes.data, 16) == \
+        svdq.ERR_BUFFER_TOO_SMALL
+    with pytest.raises(svdq.SvdqError):
+        layer.export(svdq.EXPORT_R)  # not kept
+
+
+def test_calibrate_amax_is_running_max():
+    x1 = WL.make_x(17, 64, seed=1)
+    x2 = WL.make_x(9, 64, seed=2)
+    amax = svdq.calibrate_amax(x1)
+    amax = svdq.calibrate_amax(x2, amax)
+    ref = np.maximum(np.abs(x1.astype(np.float32)).max(0), np.abs(x2.astype(np.float32)).max(0))
+    np.testing.assert_array_equal(amax, ref)
+
+
+def test_buffer_sizes_follow_tiling():
+    spec = WL.CFG1
+    X = spec.x()
+    layer = svdq.Layer(spec.w(), np.max(np.abs(X.astype(np.float32)), 0), 16, rank_capacity=48)
+    # activation tiles: 128 rows x (256 K -> 16 KB codes + 2 KB scales) + 1 chunk of 64 ranks (16 KB)
+    assert layer.act_buffer_bytes(1) == 16384 + 2048 + 16384
+    assert layer.act_buffer_bytes(129) == 2 * (16384 + 2048 + 16384)
+    info = layer.info()
+    assert (info.K, info.N, info.rank, info.rank_total, info.rank_capacity) == (256, 256, 16, 16, 48)
+    assert info.dev_buf is None and info.device == -1
+    assert info.device_bytes == layer.device_bytes > 0

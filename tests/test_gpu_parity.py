@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA path (through the C ABI) against the oracle.
+
+Codes and block scales are compared bit for bit, lr' = X_hat L1 within bf16
+rounding, Y with max|Y - Y_ref| / max|Y_ref| <= 1e-2.  Shapes cover several
+tiles, ragged tails, the smallest legal K and N, rank 0 (plain W4A4), GELU,
+bias, LoRA attach/detach, determinism and the full-size workloads (large ones
+on sampled rows: rows of the layer are independent because the activation
+scale is static)."""
+
+import numpy as np
+import pytest
+import torch
+
+from bit_w4a4_quantized_b200 import svdq
+from bit_w4a4_quantized_b200 import workloads as WL
+from gpu_cases import Case, check_act, check_y
+from oracle import svdquant as S
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    status = svdq.test_bounded_wait(50_000_000)  # 50 ms
+    t1.record()
+    torch.cuda.synchronize()
+    assert status == 1
+    assert t0.elapsed_time(t1) < 5000
+    # the context is still usable
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0
+
+
+def test_wrong_architecture_is_refused():
+    spec = WL.CFG1
+    X = spec.x()
+    layer = svdq.Layer(spec.w(), np.max(np.abs(X.astype(np.float32)), 0), spec.rank)
+    svdq.override_device_arch(90)
+    try:
+        with pytest.raises(svdq.SvdqError) as e:
+            layer.upload("cuda")
+        assert e.value.status == svdq.ERR_UNSUPPORTED_DEVICE
+    finally:
+        svdq.override_device_arch(0)
+    layer.upload("cuda")
+
+
+def _spec_case(spec, M=None, **kw):
+    return Case(spec.x(M), spec.w(), spec.rank, bias=spec.b(), **kw)
+
+
+def test_cfg1_bit_exact_codes_and_output():
+    case = _spec_case(WL.CFG1)
+    act, Y = case.run()
+    ref = check_act(case, act)
+    check_y(case, Y, ref)
+    case.layer.poll_status()
+
+
+@pytest.mark.parametrize("M", [1, 63, 127, 129, 200, 385])
+def test_ragged_rows(M):
+    case = _spec_case(WL.CFG1, M=M)
+    act, Y = case.run()
+    check_y(case, Y, check_act(case, act))
+
+
+@pytest.mark.parametrize("K,N,r", [(64, 64, 16), (128, 320, 0), (320, 192, 32), (768, 512, 48)])
+def test_small_and_ragged_k_n(K, N, r):
+    X = WL.make_x(130, K, seed=K + N)
+    W = WL.make_w(N, K, seed=K + N)
+    case = Case(X, W, r, bias=WL.make_bias(N, 5))
+    act, Y = case.run()
+    check_y(case, Y, check_act(case, act))
+
+
+@pytest.mark.parametrize("r", [0, 16, 32, 64])
+def test_ranks_including_plain_w4a4(r):
+    X = WL.make_x(256, 1024, seed=r + 1)
+    W = WL.make_w(768, 1024, seed=r + 1)
+    case = Case(X, W, r)
+    act, Y = case.run()
+    check_y(case, Y, check_act(case, act))
+
+
+def test_gelu_epilogue_with_bias():
+    X = WL.make_x(300, 512, seed=7)
+    W = WL.make_w(512, 512, seed=7)
+    case = Case(X, W, 32, bias=WL.make_bias(512, 7))
+    act, Y = case.run(epilogue=svdq.EPI_GELU_TANH)
+    check_y(case, Y, check_act(case, act), epilogue=S.EPI_GELU_TANH)
+
+
+def test_deterministic_across_runs():
+    case = _spec_case(WL.CFG2, M=512)
+    act1, Y1 = case.run()
+    act2, Y2 = case.run()
+    assert torch.equal(act1, act2)
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_lora_attach_and_detach():
+    spec = WL.CFG1
+    case = _spec_case(spec, rank_capacity=spec.rank + 32)
+    _, Y0 = case.run()
+    A, B = WL.make_lora(spec.K, spec.N, 32, seed=0)
+    Ad = torch.from_numpy(A.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    Bd = torch.from_numpy(B.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    case.layer.lora_swap(Ad, Bd, scale=0.75)
+    assert case.layer.info().rank_total == spec.rank + 32
+    S.attach_lora(case.ref, A.astype(np.float32), B.astype(np.float32), scale=0.75)
+    act, Y = case.run()
+    check_y(case, Y, check_act(case, act))
+    case.layer.lora_swap(None)
+    S.detach_lora(case.ref)
+    assert case.layer.info().rank_total == spec.rank
+    _, Y2 = case.run()
+    assert torch.equal(Y0.view(torch.int16), Y2.view(torch.int16))
+
+
+def test_lora_over_capacity_is_refused():
+    spec = WL.CFG1
+    case = _spec_case(spec)
+    A = torch.zeros((spec.K, 16), dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros((16, spec.N), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(svdq.SvdqError) as e:
+        case.layer.lora_swap(A, B)
+    assert e.value.status == svdq.ERR_UNSUPPORTED_SHAPE
+
+
+# ---------------------------------------------------------- full workloads
+
+
+def _rows(M, n=256, seed=0):
+    g = np.random.default_rng([seed, WL.STREAM_SAMPLE])
+    return np.sort(np.concatenate([[0, M - 1], g.choice(M, size=min(n, M), replace=False)]))
+
+
+def test_cfg2_attention_projection_full():
+    case = _spec_case(WL.CFG2)
+    act, Y = case.run()
+    ref = check_act(case, act)
+    err = check_y(case, Y, ref)
+    print(f"cfg2 max rel err {err:.3e}")
+    case.layer.poll_status()
+
+
+def test_cfg3_mlp_pair_sampled_rows():
+    fc1 = _spec_case(WL.CFG3_FC1)
+    act1, H = fc1.run(epilogue=svdq.EPI_GELU_TANH)
+    rows = _rows(WL.CFG3_FC1.M, seed=3)
+    ref1 = check_act(fc1, act1, rows)
+    check_y(fc1, H, ref1, epilogue=S.EPI_GELU_TANH, rows=rows)
+    # fc2 runs on the oracle's fc1 output (bf16), so nothing expected comes from the GPU
+    h_ref = S.forward(fc1.ref, fc1.X32[rows], S.EPI_GELU_TANH)
+    X2 = WL.to_bf16(h_ref)
+    fc2 = Case(X2, WL.CFG3_FC2.w(), WL.CFG3_FC2.rank)
+    act2, Y2 = fc2.run()
+    check_y(fc2, Y2, check_act(fc2, act2))
+
+
+def test_cfg4_qkv_with_lora_sampled_rows():
+    spec = WL.CFG4
+    case = _spec_case(spec, rank_capacity=spec.rank + spec.lora_rank)
+    A, B = spec.lora()
+    Ad = torch.from_numpy(A.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    Bd = torch.from_numpy(B.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    case.layer.lora_swap(Ad, Bd)
+    S.attach_lora(case.ref, A.astype(np.float32), B.astype(np.float32))
+    act, Y = case.run()
+    rows = _rows(spec.M, seed=4)
+    check_y(case, Y, check_act(case, act, rows), rows=rows)
+
+
+@pytest.mark.parametrize("M,KN,r", [(256, 3072, 0), (256, 3072, 64), (4096, 3072, 16), (1024, 3072, 32)])
+def test_sweep_points(M, KN, r):
+    spec = WL.sweep_spec(M, KN, r)
+    case = _spec_case(spec)
+    act, Y = case.run()
+    rows = _rows(M, seed=5)
+    check_y(case, Y, check_act(case, act, rows), rows=rows)
+
+
+def test_two_calls_share_nothing_between_layers():
+    a = _spec_case(WL.CFG1)
+    b = Case(WL.make_x(64, 256, seed=9), WL.make_w(256, 256, seed=9), 16)
+    act_a, Ya = a.run()
+    act_b, Yb = b.run()
+    act_a2, Ya2 = a.run()
+    assert torch.equal(Ya.view(torch.int16), Ya2.view(torch.int16))
+    check_y(b, Yb, check_act(b, act_b))
+    assert torch.equal(act_a, act_a2)

@@ -1,0 +1,119 @@
+"""Host preparation (C++) against the oracle, without a GPU.
+
+With the same low-rank factors (computed by the oracle's LAPACK SVD and given
+to the library as a checkpoint would), every prepared quantity is a function
+of the inputs with exactly defined float32 / float64 arithmetic, so the
+library must match the oracle bit for bit: lambda, R, the weight codes and
+block scales, g_w and g_a.  The library's own randomized SVD is checked for
+quality against LAPACK (singular values, Eckart-Young residual)."""
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+from bit_w4a4_quantized_b200 import svdq
+from bit_w4a4_quantized_b200 import workloads as WL
+from oracle import formats as F
+from oracle import svdquant as S
+
+
+def _oracle_factors(W, amax, r):
+    lam, _ = S.smoothing_factors(amax, np.max(np.abs(W), 0))
+    l1, l2, s = S.low_rank_factors(lam.astype(np.float64)[:, None] * W.T.astype(np.float64), r)
+    return S.bf16_from_f64(l1), S.bf16_from_f64(l2), s
+
+
+def _case(spec, M=None, N=None):
+    X = spec.x(M).astype(np.float32)
+    W = spec.w()
+    if N is not None:
+        W = W[:N]
+    return X, W, np.max(np.abs(X), axis=0)
+
+
+CASES = [
+    ("cfg1", WL.CFG1, None, None),
+    ("cfg2_rows", WL.CFG2, 256, 512),
+    ("sweep_r0", WL.sweep_spec(256, 3072, 0), 64, 256),
+    ("cfg4_rank32", WL.CFG4, 64, 320),
+]
+
+
+@pytest.mark.parametrize("name,spec,M,N", CASES, ids=[c[0] for c in CASES])
+def test_prepare_with_given_factors_is_bit_exact(name, spec, M, N):
+    X, W, amax = _case(spec, M, N)
+    Wf = W.astype(np.float32)
+    r = spec.rank
+    if r:
+        l1b, l2b, _ = _oracle_factors(Wf, amax, r)
+        factors = (l1b, l2b)
+        lib_factors = (F.bf16_bits(l1b.astype(np.float32)), F.bf16_bits(l2b.astype(np.float32)))
+    else:
+        factors, lib_factors = None, None
+    ref = S.prepare(Wf, amax, r, bias=None, factors=factors)
+    layer = svdq.Layer(W, amax, r, factors=lib_factors, keep_r=True, threads=4)
+
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_LAMBDA), ref.lam)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_INV_LAMBDA), ref.inv_lam)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_R), ref.R.astype(np.float32))
+    g_a, g_w, alpha, inv_alpha = layer.export(svdq.EXPORT_SCALARS)
+    assert g_w == ref.g_w and g_a == ref.g_a
+    assert alpha == np.float32(ref.g_a * ref.g_w)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_CODES), F.pack_e2m1(ref.w_codes))
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_SCALES), ref.w_scales)
+    if r:
+        np.testing.assert_array_equal(F.bf16_from_bits(layer.export(svdq.EXPORT_L1)), l1b.astype(np.float32))
+        np.testing.assert_array_equal(F.bf16_from_bits(layer.export(svdq.EXPORT_L2)), l2b.astype(np.float32))
+
+
+def test_prepare_is_independent_of_thread_count():
+    X, W, amax = _case(WL.CFG1)
+    a = svdq.Layer(W, amax, 16, threads=1, keep_r=True)
+    b = svdq.Layer(W, amax, 16, threads=7, keep_r=True)
+    for what in (svdq.EXPORT_L1, svdq.EXPORT_L2, svdq.EXPORT_W_CODES, svdq.EXPORT_W_SCALES, svdq.EXPORT_SIGMA):
+        np.testing.assert_array_equal(a.export(what), b.export(what))
+
+
+@pytest.mark.parametrize("name,spec,M,N", [
+    ("cfg1", WL.CFG1, None, None),
+    ("cfg2_cols", WL.CFG2, 128, 1024),
+    ("sweep_r64", WL.sweep_spec(256, 3072, 64), 64, 512),
+], ids=lambda c: c if isinstance(c, str) else "")
+def test_library_svd_quality_against_lapack(name, spec, M, N):
+    X, W, amax = _case(spec, M, N)
+    Wf = W.astype(np.float32)
+    r = spec.rank
+    layer = svdq.Layer(W, amax, r, threads=8)
+    lam = layer.export(svdq.EXPORT_LAMBDA).astype(np.float64)
+    A = lam[:, None] * Wf.T.astype(np.float64)
+    s = scipy.linalg.svd(A, compute_uv=False, lapack_driver="gesvd")
+    sig = layer.export(svdq.EXPORT_SIGMA)
+    # Ritz values from a subspace never exceed the true singular values
+    # (interlacing); the well-separated leading ones are found to high accuracy
+    assert np.all(sig <= s[:r] * (1 + 1e-12))
+    lead = s[:r] > 1.5 * s[r]
+    np.testing.assert_allclose(sig[lead], s[:r][lead], rtol=1e-6)
+    tail = np.sqrt(np.sum(s[r:] ** 2))
+    r_f64, r_bf16 = layer.export(svdq.EXPORT_RESID_NORM)
+    # Eckart-Young: no rank-r factorization beats the tail; ours is within 1 %
+    assert tail * (1 - 1e-12) <= r_f64 <= 1.01 * tail
+    # bf16 rounding of the factors adds at most ~2^-8 relative of ||L1 L2||
+    assert r_bf16 <= r_f64 + 2 * 2.0**-8 * np.sqrt(np.sum(s[:r] ** 2))
+    # L2 rows orthonormal up to bf16 rounding
+    l2 = F.bf16_from_bits(layer.export(svdq.EXPORT_L2)).astype(np.float64)
+    np.testing.assert_allclose(l2 @ l2.T, np.eye(r), atol=2e-2)
+
+
+def test_library_svd_exact_rank():
+    g = np.random.default_rng(3)
+    K, N, r = 256, 192, 16
+    W = (g.standard_normal((N, r)) @ g.standard_normal((r, K)) * 0.05).astype(np.float32)
+    Wb = WL.to_bf16(W)
+    amax = np.ones(K, np.float32)
+    layer = svdq.Layer(Wb, amax, r, threads=4)
+    r_f64, _ = layer.export(svdq.EXPORT_RESID_NORM)
+    A = layer.export(svdq.EXPORT_LAMBDA).astype(np.float64)[:, None] * Wb.astype(np.float64).T
+    # bf16 rounding of W makes it full rank, but only barely: the tail is tiny
+    s = scipy.linalg.svd(A, compute_uv=False)
+    assert r_f64 <= 1.01 * np.sqrt(np.sum(s[r:] ** 2))
+    assert r_f64 < 1e-2 * np.linalg.norm(A)
