@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Throughput of the fused SVDQuant W4A4 + low-rank linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    (N > 1: launch with torch.distributed.run, one rank per GPU)
+
+One step = one pass of the whole hot path over one batch: kernel 1
+(smoothing, NVFP4 quantization of X, down projection X_hat L1) and kernel 2
+(block-scaled NVFP4 GEMM with the up projection folded into the same
+accumulator, bias epilogue).  The weights are prepared once, outside the
+timed region, as a model load would.
+
+Workload: the attention-projection layer M = 4096 tokens, K = N = 3072,
+rank 32, bf16 bias, Student-t(4) activations with 1 % outlier channels x 50,
+N(0, 0.02) weights with 0.5 % outlier columns x 20 (synthetic, seeded).
+
+Timing: each step is a CUDA graph (so host launch cost cannot bound the
+GPU); steps rotate over buffer sets (X, activation buffer, Y and a copy of
+the prepared layer) whose total exceeds the 126 MB L2, so every step reads
+its operands from HBM.  CUDA events on the launching stream, max over ranks.
+value = 2 M N K / step time, summed over ranks (weak scaling: every rank
+runs its own batch; the layer has no cross-GPU exchange, so ranks are
+replicas).  See the design doc for the roofline accounting.
+"""
+
+import argparse
+import datetime
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "fused W4A4+low-rank linear TFLOPS"
+UNIT = "TFLOP/s"
+
+
+# ----------------------------------------------------------------- workload
+def workload_spec(name):
+    from bit_w4a4_quantized_b200 import workloads as WL
+
+    table = {"cfg1": WL.CFG1, "cfg2": WL.CFG2, "cfg3_fc1": WL.CFG3_FC1, "cfg3_fc2": WL.CFG3_FC2, "cfg4": WL.CFG4}
+    if name in table:
+        return table[name]
+    if name.startswith("sweep:"):
+        _, m, kn, r = name.split(":")
+        return WL.sweep_spec(int(m), int(kn), int(r))
+    raise SystemExit(f"unknown workload {name}")
+
+
+def layer_flops(spec, r_tot):
+    """(FP4 GEMM flops, bf16 low-rank flops) of one forward of the layer."""
+    fp4 = 2 * spec.M * spec.N * spec.K
+    lowrank = 2 * spec.M * spec.K * r_tot + 2 * spec.M * spec.N * r_tot
+    return fp4, lowrank
+
+
+# ------------------------------------------------------------ multi-rank
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def rank_seed(base_seed, rank):
+    """Each rank draws its own batch (weak scaling); rank 0 keeps the workload's seed."""
+    return base_seed if rank == 0 else base_seed * 1000 + rank
+
+
+def reduce_max(value, device=None):
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units, world, seconds_max):
+    """Whole-job throughput: units of every rank over the slowest rank's time."""
+    return per_rank_units * world / seconds_max
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region.
+
+    All GPUs are sampled; rows are kept for the one whose UUID matches the
+    benchmarked device (the first GPU if the UUID is unknown)."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = None if uuid is None else str(uuid).lower().replace("gpu-", "")
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self, load_mhz_floor=500):
+        rows = [[x.strip() for x in l.split(",")] for l in self.lines]
+        rows = [r for r in rows if len(r) >= 9]
+        if self.uuid is not None and any(self.uuid in r[0].lower() for r in rows):
+            rows = [r for r in rows if self.uuid in r[0].lower()]
+        elif rows:
+            first = rows[0][0]
+            rows = [r for r in rows if r[0] == first]
+        sm, mx, reasons = [], None, set()
+        for r in rows:
+            try:
+                mhz, mx = float(r[1]), float(r[2])
+            except ValueError:
+                continue
+            if mhz >= load_mhz_floor:
+                sm.append(mhz)
+                for n, v in zip(self.REASONS, r[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows), "samples_under_load": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("bf16_tflops"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+# -------------------------------------------------------------- CPU oracle
+def oracle_throughput(spec, budget_s, min_steps=1, max_rows=None, steps=None, warmup=0):
+    """Time the CPU oracle (quantize_act + linear) on a bounded sample of the workload.
+
+    Returns (value TFLOP/s, seconds, steps, rows per step, threads)."""
+    import threadpoolctl
+
+    from oracle import svdquant as S
+
+    X = spec.x(min(spec.M, 256)).astype(np.float32)
+    W = spec.w().astype(np.float32)
+    amax = np.max(np.abs(X), axis=0)
+    b = spec.b()
+    layer = S.prepare(W, amax, spec.rank, bias=None if b is None else b.astype(np.float64))
+    _ = layer.deq_w  # weights are dequantized once per layer
+    epi = S.EPI_GELU_TANH if spec.gelu else S.EPI_NONE
+    # size the per-step sample from one calibration step
+    t0 = time.perf_counter()
+    S.linear(layer, S.quantize_act(layer, X[:1]), epi)
+    t_row = max(time.perf_counter() - t0, 1e-4)
+    n_steps = steps if steps is not None else max(min_steps, 1)
+    rows = int(max(1, min(X.shape[0], max_rows or X.shape[0], budget_s / (n_steps + warmup) / t_row)))
+    xs = X[:rows]
+    for _ in range(warmup):
+        S.linear(layer, S.quantize_act(layer, xs), epi)
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        S.linear(layer, S.quantize_act(layer, xs), epi)
+        done += 1
+        el = time.perf_counter() - t0
+        if steps is not None:
+            if done >= steps:
+                break
+        elif el >= budget_s and done >= min_steps:
+            break
+    el = time.perf_counter() - t0
+    info = threadpoolctl.threadpool_info()
+    threads = max([i.get("num_threads", 1) for i in info] or [1])
+    flops = 2 * rows * spec.N * spec.K * done
+    return flops / el / 1e12, el, done, rows, threads
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_w4a4_quantized_b200 import svdq
+    from bit_w4a4_quantized_b200 import workloads as WL
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    spec = workload_spec(args.workload)
+    seed = rank_seed(spec.seed, rank)
+    X = WL.make_x(spec.M, spec.K, seed, spec.x_dist, spec.x_outliers, spec.x_outlier_scale)
+    W = spec.w()
+    bias = spec.b()
+    amax = svdq.calibrate_amax(X)  # calibrated on the batch it runs, like the parity tests
+    t_prep = time.perf_counter()
+    layer0 = svdq.Layer(W, amax, spec.rank, bias=bias, device=device)
+    t_prep = time.perf_counter() - t_prep
+    r_tot = layer0.info().rank_total
+    lora_note = None
+    if spec.lora_rank:
+        layer0 = svdq.Layer(W, amax, spec.rank, rank_capacity=spec.rank + spec.lora_rank, bias=bias,
+                            factors=(layer0.export(svdq.EXPORT_L1), layer0.export(svdq.EXPORT_L2)), device=device)
+        A, B = spec.lora()
+        to_dev = lambda a: torch.from_numpy(a.view(np.uint16).astype(np.int16)).view(torch.bfloat16).to(device)
+        lora_dev = (to_dev(A), to_dev(B))
+        layer0.lora_swap(*lora_dev)
+        r_tot = layer0.info().rank_total
+        lora_note = f"LoRA rank {spec.lora_rank} attached"
+    epi = svdq.EPI_GELU_TANH if spec.gelu else svdq.EPI_NONE
+    M, N, K = spec.M, spec.N, spec.K
+
+    # buffer sets: (layer copy, X, act, Y); total > 3x L2 so each step misses L2
+    Xd = torch.from_numpy(X.view(np.uint16).astype(np.int16)).view(torch.bfloat16).to(device)
+    act_bytes = layer0.act_buffer_bytes(M)
+    per_set = layer0.device_bytes + act_bytes + 2 * M * K + 2 * M * N
+    nsets = int(min(16, max(2, math.ceil(3 * L2_BYTES / per_set))))
+    factors = (layer0.export(svdq.EXPORT_L1), layer0.export(svdq.EXPORT_L2)) if spec.rank else None
+    layers = [layer0]
+    for _ in range(nsets - 1):
+        L = svdq.Layer(W, amax, spec.rank, rank_capacity=layer0.info().rank_capacity, bias=bias, factors=factors,
+                       device=device)
+        if spec.lora_rank:
+            L.lora_swap(*lora_dev)
+        layers.append(L)
+    Xs = [Xd] + [Xd.clone() for _ in range(nsets - 1)]
+    acts = [L.new_act_buffer(M) for L in layers]
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize(device)
+
+    def q(i):
+        layers[i].quantize_act(Xs[i], acts[i])
+
+    def g(i):
+        layers[i].linear(acts[i], M, out=Ys[i], epilogue=epi)
+
+    with torch.cuda.stream(stream):
+        for i in range(nsets):  # eager warm-up: sets function attributes, loads modules
+            q(i)
+            g(i)
+        stream.synchronize()
+        for L in layers:
+            L.poll_status()
+
+    def capture(fn):
+        graphs = []
+        for i in range(nsets):
+            cg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(cg, stream=stream, capture_error_mode="thread_local"):
+                fn(i)
+            graphs.append(cg)
+        return graphs
+
+    step_graphs = capture(lambda i: (q(i), g(i)))
+    k1_graphs = capture(q)
+    k2_graphs = capture(g)
+
+    def timed(graphs, steps, sampler=None):
+        with torch.cuda.stream(stream):
+            barrier(device)
+            torch.cuda.synchronize(device)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(steps):
+                graphs[i % nsets].replay()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            barrier(device)
+        return e0.elapsed_time(e1) / 1e3
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step_graphs[i % nsets].replay()
+    props = torch.cuda.get_device_properties(device)
+    with ClockSampler(getattr(props, "uuid", None)) as clk:
+        t_step = timed(step_graphs, args.steps)
+    t_step_max = reduce_max(t_step, device)
+    t_k1 = reduce_max(timed(k1_graphs, args.steps), device)
+    t_k2 = reduce_max(timed(k2_graphs, args.steps), device)
+    for L in layers:
+        L.poll_status()
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    e2e_steps = max(3, min(args.steps, 30))
+    Xh = Xd.cpu().pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xe = torch.empty_like(Xd)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            Xe.copy_(Xh, non_blocking=True)
+            layers[0].forward(Xe, out=Ys[0], epilogue=epi, act=acts[0])
+            Yh.copy_(Ys[0], non_blocking=True)
+        barrier(device)
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            Xe.copy_(Xh, non_blocking=True)
+            layers[0].forward(Xe, out=Ys[0], epilogue=epi, act=acts[0])
+            Yh.copy_(Ys[0], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+    t_e2e = reduce_max(e0.elapsed_time(e1) / 1e3, device)
+
+    fp4, lowrank = layer_flops(spec, r_tot)
+    value = aggregate(2 * M * N * K * args.steps, world, t_step_max) / 1e12
+    e2e_value = aggregate(2 * M * N * K * e2e_steps, world, t_e2e) / 1e12
+
+    # roofline of the dominant kernel
+    bf16_peak, hbm_peak, peak_src = measured_peaks()
+    fp4_peak = bf16_peak * 4.0  # dense FP4 / BF16 nominal ratio (9 / 2.25 PFLOP/s)
+    per_k2 = t_k2 / args.steps
+    per_k1 = t_k1 / args.steps
+    k2_flops = fp4 + 2 * M * N * r_tot
+    k2_roof_s = fp4 / (fp4_peak * 1e12) + 2 * M * N * r_tot / (bf16_peak * 1e12)
+    k1_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * M * r_tot + 2 * K * r_tot + 4 * K
+    if per_k2 >= per_k1:
+        roof = {"kernel": "svdq_gemm (kernel 2)", "bound": "tensor", "achieved": k2_flops / per_k2 / 1e12,
+                "peak": k2_flops / k2_roof_s / 1e12, "unit": "TFLOP/s", "traffic": None}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["peak_basis"] = (f"{peak_src} bf16 {bf16_peak} TF/s x 4 (nominal FP4:BF16) for the FP4 flops, "
+                              f"bf16 {bf16_peak} TF/s for the fold")
+    else:
+        roof = {"kernel": "act_quant (kernel 1)", "bound": "hbm", "achieved": k1_bytes / per_k1 / 1e9,
+                "peak": hbm_peak, "unit": "GB/s", "traffic": None, "peak_basis": f"{peak_src} HBM copy"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+
+    clocks = clk.summary()
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_step_max / args.steps * 1e3, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4(e2m1,e4m3 scales)+bf16 low-rank, fp32 acc",
+        "data": "synthetic (seeded; stands in for FLUX.1 projection inputs)",
+        "config": {"workload": spec.name, "M": M, "K": K, "N": N, "rank": spec.rank, "rank_total": r_tot,
+                   "bias": bias is not None, "epilogue": "gelu_tanh" if spec.gelu else "none",
+                   "lora": lora_note, "parallelism": f"replicas x{world} (no collective on the data path)",
+                   "l2": f"rotating {nsets} buffer sets of {per_set / 2**20:.1f} MiB (X, act, Y, layer copy): "
+                         f"{nsets * per_set / 2**20:.0f} MiB > L2", "timing": "CUDA graph per step, CUDA events"},
+        "kernels": {"act_quant_us": round(per_k1 * 1e6, 3), "gemm_us": round(per_k2 * 1e6, 3),
+                    "act_quant_GBps": round(k1_bytes / per_k1 / 1e9, 1),
+                    "gemm_TFLOPs": round(k2_flops / per_k2 / 1e12, 1), "flops_fp4": fp4,
+                    "flops_lowrank": lowrank, "prepare_s": round(t_prep, 3)},
+        "roofline": {k: (round(v, 4) if isinstance(v, float) else v) for k, v in roof.items()},
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": 2 * M * K,
+                "d2h_bytes_per_step": 2 * M * N},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, el, done, rows, threads = oracle_throughput(spec, args.cpu_budget)
+        out["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                               "sample": f"{rows} rows x {done} calls of the CPU oracle (quantize_act + linear, "
+                                         f"float64 NumPy/BLAS) on the same layer, {el:.1f} s; "
+                                         f"host has {os.cpu_count()} logical cores"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    for cg in step_graphs + k1_graphs + k2_graphs:
+        del cg
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+# --------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0  # the oracle runs on the host of rank 0 only
+    spec = workload_spec(args.workload)
+    budget = args.cpu_budget
+    v, el, done, rows, threads = oracle_throughput(spec, budget, steps=args.steps, warmup=args.warmup)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / done * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 (oracle: float32 quantization decisions, float64 accumulation)",
+        "data": "synthetic (seeded; stands in for FLUX.1 projection inputs)",
+        "config": {"workload": spec.name, "M": spec.M, "K": spec.K, "N": spec.N, "rank": spec.rank,
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of {spec.M} rows per step, {done} steps, {el:.1f} s"},
+        "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    _, world, _ = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

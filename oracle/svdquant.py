@@ -202,6 +202,13 @@ class Layer:
     def alpha(self):
         return np.float64(self.g_a) * np.float64(self.g_w)
 
+    @property
+    def deq_w(self):
+        """Dequantized Q(R)^T block values [N, K] (computed once per layer)."""
+        if getattr(self, "_deq_w", None) is None:
+            self._deq_w = nvfp4_dequantize(self.w_codes, self.w_scales)
+        return self._deq_w
+
 
 def act_global_scale(act_amax, inv_lam):
     """Static g_a: max over j of bf16(f32(a_j / lambda_j)) over 2688.
@@ -299,8 +306,7 @@ def linear(layer, act, epilogue=EPI_NONE, rows=None):
     if rows is not None:
         codes, scales, lr = codes[rows], scales[rows], lr[rows]
     deq_a = nvfp4_dequantize(codes, scales)
-    deq_w = nvfp4_dequantize(layer.w_codes, layer.w_scales)
-    y = layer.alpha * (deq_a @ deq_w.T) + lr @ layer.L2
+    y = layer.alpha * (deq_a @ layer.deq_w.T) + lr @ layer.L2
     if layer.bias is not None:
         y = y + layer.bias[None, :]
     if epilogue == EPI_GELU_TANH:

@@ -92,11 +92,17 @@ def test_gelu_epilogue_with_bias():
     check_y(case, Y, check_act(case, act), epilogue=S.EPI_GELU_TANH)
 
 
+def _same_act(case, a1, a2, M):
+    """Everything kernel 1 writes (the buffers' padding is never written)."""
+    for x, y in zip(case.unpack(a1, M), case.unpack(a2, M)):
+        np.testing.assert_array_equal(x, y)
+
+
 def test_deterministic_across_runs():
     case = _spec_case(WL.CFG2, M=512)
     act1, Y1 = case.run()
     act2, Y2 = case.run()
-    assert torch.equal(act1, act2)
+    _same_act(case, act1, act2, 512)
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
 
 
@@ -190,4 +196,4 @@ def test_two_calls_share_nothing_between_layers():
     act_a2, Ya2 = a.run()
     assert torch.equal(Ya.view(torch.int16), Ya2.view(torch.int16))
     check_y(b, Yb, check_act(b, act_b))
-    assert torch.equal(act_a, act_a2)
+    _same_act(a, act_a, act_a2, 64)
