@@ -11,15 +11,16 @@
 //   Y    = bf16(act(alpha * acc + b)),  alpha = g_a g_w,  lr' = (X_hat L1) / alpha
 //
 // Design (sm_100a), persistent, one CTA per SM, 128 x 256 output tiles:
-//   * warp 4: one thread fills a 4-stage ring with 1D bulk copies (every
+//   * warp 8: one thread fills a 4-stage ring with 1D bulk copies (every
 //     operand is stored pre-tiled and pre-swizzled, so a stage is 4 copies:
 //     A codes 16 KB, B codes 32 KB, A scales 2 KB, B scales 4 KB); after the K
 //     loop of a tile it loads the lr' and L2^T chunks into the same ring;
-//   * warp 5: one thread copies the stage's block scales into tensor memory
+//   * warp 9: one thread copies the stage's block scales into tensor memory
 //     (tcgen05.cp 32x128b.warpx4), issues 4 block-scaled MMAs per 256-wide
 //     k-tile, then the bf16 MMAs of the fold, and commits stages back;
-//   * warps 0-3: epilogue, one output row per thread, tensor memory ->
-//     registers -> alpha, bias, GELU -> bf16 -> global.
+//   * warps 0-7: epilogue, one output row x 128 columns per thread: tensor
+//     memory -> registers, release the accumulator, then alpha, bias, GELU ->
+//     bf16 -> global while the next tile's K loop runs.
 //   * Tensor memory: accumulator columns [0, 256), scale factors of stage s at
 //     256 + 16 s (A) and 320 + 32 s (B).
 //   * Every wait is bounded (status word + clean exit on timeout).
@@ -37,11 +38,14 @@ namespace {
 using namespace ptx;
 
 constexpr int kStages2 = 4;
-constexpr int kThreads2 = 192;
+constexpr int kThreads2 = 320;  // warps 0-7 epilogue, 8 producer, 9 MMA
+constexpr int kEpiThreads = 256;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr uint32_t kOffA = 0, kOffB = kATileBytes, kOffSFA = kOffB + kBTileBytes;
 constexpr uint32_t kOffSFB = kOffSFA + kSFATileBytes;
 constexpr uint32_t kStage2 = kOffSFB + kSFBTileBytes;  // 55296 bytes
 constexpr uint32_t kCtrl2 = 128;
+constexpr uint32_t kBiasBytes = 8 * 2 * 128 * 4;  // per epilogue warp: 2 tiles x 128 floats
 constexpr uint32_t kTmemCols2 = 512;
 constexpr uint32_t kColSFA = 256, kColSFB = 320;
 
@@ -69,30 +73,16 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return 0.5f * x * (1.0f + tanh_approx(u));
 }
 
-// 32 accumulator columns of one row -> bf16 -> 64 bytes of Y.
-__device__ __forceinline__ void store_chunk(const GemmParams& p, const uint32_t* v, int64_t row, int n0) {
-  float b[32];
-  if (p.bias) {
-    const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 w = __ldg(bp + q);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        b[8 * q + 2 * e] = bf16lo(ws[e]);
-        b[8 * q + 2 * e + 1] = bf16hi(ws[e]);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 32; ++e) b[e] = 0.0f;
-  }
+// 32 accumulator columns of one row -> alpha, bias, act -> bf16 -> 64 bytes of Y.
+// `bias` points at the 32 bias values of these columns in shared memory (or null).
+__device__ __forceinline__ void store_chunk(const GemmParams& p, const uint32_t* v, const float* bias, int64_t row,
+                                            int n0) {
   uint32_t out[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    float y0 = fmaf(p.alpha, __uint_as_float(v[2 * e]), b[2 * e]);
-    float y1 = fmaf(p.alpha, __uint_as_float(v[2 * e + 1]), b[2 * e + 1]);
+    const float b0 = bias ? bias[2 * e] : 0.0f, b1 = bias ? bias[2 * e + 1] : 0.0f;
+    float y0 = fmaf(p.alpha, __uint_as_float(v[2 * e]), b0);
+    float y1 = fmaf(p.alpha, __uint_as_float(v[2 * e + 1]), b1);
     if (p.epilogue == SVDQ_EPI_GELU_TANH) {
       y0 = gelu_tanh(y0);
       y1 = gelu_tanh(y1);
@@ -118,6 +108,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
   const uint32_t ACCF = ctrl_s + 64u, ACCE = ctrl_s + 72u, DRAIN = ctrl_s + 80u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 88);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 92);
+  float* bias_s = reinterpret_cast<float*>(ctrl + kCtrl2);  // [warp][tile parity][128] floats
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
@@ -125,12 +116,12 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
       mbar_init(EMPTY + 8u * s, 1);
     }
     mbar_init(ACCF, 1);
-    mbar_init(ACCE, 128);
+    mbar_init(ACCE, kEpiThreads);
     mbar_init(DRAIN, 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(ctrl_s + 88u, kTmemCols2);
     tmem_relinquish();
   }
@@ -147,7 +138,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
   const int ntiles = p.MT * p.NT;
   const int nlr = (p.r_tot + kRChunk - 1) / kRChunk;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t it = 0;
@@ -190,7 +181,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
         mbar_wait(FULL + 8u * (i % kStages2), (i / kStages2) & 1u, nullptr, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t id_fp4 = idesc_nvfp4(kBN), id_bf16 = idesc_bf16(kBN);
@@ -254,11 +245,24 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
     __syncwarp();
   } else {
     // ------------------------------------------------------------- epilogue
+    // warp w reads TMEM lanes 32 (w % 4) .. +31 (its lane quarter) and
+    // accumulator columns 128 (w / 4) .. +127: the whole 128 x 256 tile is
+    // read into registers, the accumulator is released, then the rows are
+    // finished and stored while the next tile's K loop runs.
     uint32_t tc = 0;
-    const int row_in_tile = warp * 32 + lane;
-    const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
+    const int quarter = warp & 3, colhalf = warp >> 2;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colhalf * 128);
     for (int tile = int(blockIdx.x); tile < ntiles; tile += int(gridDim.x)) {
       const int mt = tile % p.MT, nt = tile / p.MT;
+      // stage this warp's 128 bias values while the K loop runs (warp-private,
+      // double buffered by tile parity: only __syncwarp is needed)
+      float* bias_w = bias_s + (size_t(warp) * 2 + (tc & 1u)) * 128;
+      if (p.bias) {
+        const uint2 w = *reinterpret_cast<const uint2*>(p.bias + size_t(nt) * kBN + colhalf * 128 + lane * 4);
+        *reinterpret_cast<float4*>(bias_w + lane * 4) = make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
+      }
+      __syncwarp();
       bool ok = mbar_wait(ACCF, tc & 1u, abort_flag, p.timeout_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) {
@@ -266,25 +270,21 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
         break;
       }
       tc_fence_after();
+      uint32_t v[128];
+      tmem_ld32(tl, v);
+      tmem_ld32(tl + 32u, v + 32);
+      tmem_ld32(tl + 64u, v + 64);
+      tmem_ld32(tl + 96u, v + 96);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(ACCE);  // the accumulator may be overwritten now
       const int64_t row = int64_t(mt) * kBM + row_in_tile;
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        uint32_t v[128];
-        tmem_ld32(tl + uint32_t(half * 128), v);
-        tmem_ld32(tl + uint32_t(half * 128 + 32), v + 32);
-        tmem_ld32(tl + uint32_t(half * 128 + 64), v + 64);
-        tmem_ld32(tl + uint32_t(half * 128 + 96), v + 96);
-        tmem_wait_ld();
-        if (half == 1) {
-          tc_fence_before();
-          mbar_arrive(ACCE);  // the accumulator may be overwritten now
-        }
-        if (row < p.M) {
+      if (row < p.M) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int n0 = nt * kBN + half * 128 + q * 32;
-            if (n0 < p.N) store_chunk(p, v + 32 * q, row, n0);
-          }
+        for (int q = 0; q < 4; ++q) {
+          const int c0 = colhalf * 128 + q * 32;
+          const int n0 = nt * kBN + c0;
+          if (n0 < p.N) store_chunk(p, v + 32 * q, p.bias ? bias_w + q * 32 : nullptr, row, n0);
         }
       }
       ++tc;
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols2);
   }
@@ -331,7 +331,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
     *why = "too many output tiles";
     return cudaErrorInvalidValue;
   }
-  const size_t smem = size_t(kStages2) * kStage2 + kCtrl2 + 1024;
+  const size_t smem = size_t(kStages2) * kStage2 + kCtrl2 + kBiasBytes + 1024;
   {
     static std::atomic<int> set_on[64];
     int dev = 0;
