@@ -10,14 +10,14 @@
 // and lr' = bf16((x_hat L1) / (g_a g_w)) on the tensor cores.
 //
 // Design (sm_100a):
-//   * CTA = 128 rows of X x a slice of K.  Warp 4 streams X chunks of 128 rows
+//   * CTA = 128 rows of X x a slice of K.  Warp 8 streams X chunks of 128 rows
 //     x 64 columns with a 2D TMA load (128-byte swizzle), the matching
 //     1/lambda slice and L1^T chunk with bulk copies, through a 4-stage
 //     mbarrier ring.
-//   * Warps 0-3: one thread per row converts its 64 elements in shared
-//     memory, writes x_hat back in place (it is the A operand of the MMA),
-//     and stores codes and block scales straight into the GEMM's tiled layout.
-//   * Warp 5: one thread issues tcgen05.mma kind::f16 (M = 128, N = rank)
+//   * Warps 0-7: two threads per row convert 32 elements each in shared
+//     memory, write x_hat back in place (it is the A operand of the MMA),
+//     and store codes and block scales straight into the GEMM's tiled layout.
+//   * Warp 9: one thread issues tcgen05.mma kind::f16 (M = 128, N = rank)
 //     accumulating X_hat L1 in tensor memory.
 //   * K is split across the CTAs of a cluster so that enough CTAs stream HBM;
 //     their partial X_hat L1 tiles are summed in a fixed order through
@@ -40,7 +40,10 @@ namespace {
 using namespace ptx;
 
 constexpr int kStages1 = 4;
-constexpr int kThreads1 = 192;
+constexpr int kThreads1 = 320;  // warps 0-7 convert, 8 produce, 9 issue MMAs
+constexpr int kConvThreads = 256;
+constexpr int kProducerWarp1 = 8, kMmaWarp1 = 9;
+constexpr int kMaxSplits = 8;
 constexpr uint32_t kXBytes = kBM * 128;  // 16 KB: 128 rows x 64 bf16
 constexpr uint32_t kInvSlot = 1024;      // 64 floats of 1/lambda (256 B), padded for alignment
 constexpr uint32_t kCtrlBytes = 128;
@@ -61,7 +64,8 @@ struct ActQuantParams {
 // One 16-element block of one row: read x from the swizzled stage, write
 // x_hat back, return 8 bytes of E2M1 codes and the E4M3 block scale.
 __device__ __forceinline__ void quant_block(uint8_t* xrow, uint32_t t7, int g, const float* inv, float g_a,
-                                            float c_a, uint32_t& w0, uint32_t& w1, uint32_t& scale) {
+                                            float c_a, bool write_back, uint32_t& w0, uint32_t& w1,
+                                            uint32_t& scale) {
   uint4* p0 = reinterpret_cast<uint4*>(xrow + (((2u * g) ^ t7) << 4));
   uint4* p1 = reinterpret_cast<uint4*>(xrow + (((2u * g + 1u) ^ t7) << 4));
   const uint4 a = *p0, b = *p1;
@@ -82,8 +86,10 @@ __device__ __forceinline__ void quant_block(uint8_t* xrow, uint32_t t7, int g, c
     xh[2 * j + 1] = bf16hi(h[j]);
     amax = fmaxf(amax, fmaxf(fabsf(xh[2 * j]), fabsf(xh[2 * j + 1])));
   }
-  *p0 = make_uint4(h[0], h[1], h[2], h[3]);
-  *p1 = make_uint4(h[4], h[5], h[6], h[7]);
+  if (write_back) {  // x_hat is the A operand of the down projection
+    *p0 = make_uint4(h[0], h[1], h[2], h[3]);
+    *p1 = make_uint4(h[4], h[5], h[6], h[7]);
+  }
   const uint32_t sc = f32_to_e4m3(__fmul_rn(amax, c_a));
   const float d = __fmul_rn(e4m3_value(sc), g_a);
   const float rcp = d == 0.0f ? 0.0f : __frcp_rn(d);
@@ -106,7 +112,7 @@ __device__ __forceinline__ void store_lr8(const ActQuantParams& p, int mt, uint3
   *reinterpret_cast<uint4*>(tile + sw128(row, uint32_t(c % kRChunk) * 2u)) = w;
 }
 
-__global__ void __launch_bounds__(kThreads1, 1)
+__global__ void __launch_bounds__(kThreads1, 2)
     act_quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const ActQuantParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -131,7 +137,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages1; ++s) {
       mbar_init(FULL + 8u * s, 1);
-      mbar_init(CONV + 8u * s, 128);
+      mbar_init(CONV + 8u * s, kConvThreads);
       mbar_init(EMPTY + 8u * s, 1);
     }
     mbar_init(ACCF, 1);
@@ -139,7 +145,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp == 5 && lowrank) {
+  if (warp == kMmaWarp1 && lowrank) {
     tmem_alloc(ctrl_s + 112u, p.tmem_cols);
     tmem_relinquish();
   }
@@ -153,7 +159,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
     atomicOr(p.status, code);
   };
 
-  if (warp == 4) {
+  if (warp == kProducerWarp1) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tmap_x);
@@ -181,9 +187,11 @@ __global__ void __launch_bounds__(kThreads1, 1)
         mbar_wait(FULL + 8u * (i % kStages1), uint32_t(i / kStages1) & 1u, nullptr, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ----------------------------------------------------------- converters
-    const uint32_t t = threadIdx.x;  // row inside the 128-row tile
+    // two threads per row: thread (t, h) converts elements 32 h .. 32 h + 31
+    // of row t of each 64-column chunk (two 16-element blocks)
+    const uint32_t t = threadIdx.x & 127u, h = threadIdx.x >> 7;
     const uint32_t t7 = t & 7u;
     for (int i = 0; i < nchunks; ++i) {
       const int s = i % kStages1;
@@ -195,19 +203,21 @@ __global__ void __launch_bounds__(kThreads1, 1)
       uint8_t* stage = smem + size_t(s) * p.stage_bytes;
       uint8_t* xrow = stage + t * 128u;
       const float* inv = reinterpret_cast<const float*>(stage + kXBytes);
-      uint32_t cw[8], sc[4];
+      uint32_t cw[4], sc[2];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) quant_block(xrow, t7, g, inv + 16 * g, p.g_a, p.c_a, cw[2 * g], cw[2 * g + 1], sc[g]);
+      for (int j = 0; j < 2; ++j) {
+        const int g = int(2 * h) + j;
+        quant_block(xrow, t7, g, inv + 16 * g, p.g_a, p.c_a, lowrank, cw[2 * j], cw[2 * j + 1], sc[j]);
+      }
       const int kc = kc0 + i, kt = kc >> 2, sub = kc & 3;
       uint8_t* ctile = p.codes + (size_t(mt) * p.KT + kt) * kATileBytes;
-      *reinterpret_cast<uint4*>(ctile + sw128(t, uint32_t(sub) * 32u)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      *reinterpret_cast<uint4*>(ctile + sw128(t, uint32_t(sub) * 32u + 16u)) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      *reinterpret_cast<uint4*>(ctile + sw128(t, uint32_t(sub) * 32u + h * 16u)) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       uint8_t* stile = p.sf + (size_t(mt) * p.KT + kt) * kSFATileBytes + size_t(sub) * kSFAtomBytes;
-      *reinterpret_cast<uint32_t*>(stile + sf_atom(t, 0)) = sc[0] | (sc[1] << 8) | (sc[2] << 16) | (sc[3] << 24);
-      fence_proxy_async_smem();  // x_hat (generic writes) -> tensor-core reads
+      *reinterpret_cast<uint16_t*>(stile + sf_atom(t, 2u * h)) = uint16_t(sc[0] | (sc[1] << 8));
+      if (lowrank) fence_proxy_async_smem();  // x_hat (generic writes) -> tensor-core reads
       mbar_arrive(CONV + 8u * s);
     }
-  } else {
+  } else if (warp == kMmaWarp1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       bool any = false;
@@ -281,23 +291,35 @@ __global__ void __launch_bounds__(kThreads1, 1)
     }
     if (multi) {
       cluster_sync();  // every partial tile of the cluster is in shared memory
-      if (warp < 4 && *abort_flag == 0u) {
+      if (warp < 8 && *abort_flag == 0u) {
+        // this CTA sums rows [row0, row1) over the cluster, 4 ranks per item;
+        // all peer loads of an item are in flight before the (ordered) adds
         const int rows = (kBM + p.splits - 1) / p.splits;
         const int rank = int(cluster_ctarank());
         const int row0 = rank * rows;
         const int row1 = row0 + rows < kBM ? row0 + rows : kBM;
-        const int groups = p.r_tot / 8;
-        for (int item = int(threadIdx.x); item < (row1 - row0) * groups; item += 128) {
-          const int row = row0 + item / groups, c = (item % groups) * 8;
-          const uint32_t off = uint32_t((row * pstride + c) * 4);
-          float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          for (int q = 0; q < p.splits; ++q) {  // fixed order: deterministic sums
-            const uint32_t a = mapa(sbase + off, uint32_t(q));
-            const float4 v0 = ld_dsmem_f4(a), v1 = ld_dsmem_f4(a + 16u);
-            acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
-            acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
-          }
-          store_lr8(p, mt, uint32_t(row), c, acc);
+        const int groups = p.r_tot / 4;
+        for (int item = int(threadIdx.x); item < (row1 - row0) * groups; item += kConvThreads) {
+          const int row = row0 + item / groups, c = (item % groups) * 4;
+          const uint32_t local = sbase + uint32_t((row * pstride + c) * 4);
+          float4 v[kMaxSplits];
+#pragma unroll
+          for (int q = 0; q < kMaxSplits; ++q)
+            if (q < p.splits) v[q] = ld_dsmem_f4(mapa(local, uint32_t(q)));
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < kMaxSplits; ++q)  // fixed order: deterministic sums
+            if (q < p.splits) {
+              acc.x += v[q].x;
+              acc.y += v[q].y;
+              acc.z += v[q].z;
+              acc.w += v[q].w;
+            }
+          uint2 w;
+          w.x = f32x2_to_bf16x2(__fmul_rn(acc.x, p.inv_alpha), __fmul_rn(acc.y, p.inv_alpha));
+          w.y = f32x2_to_bf16x2(__fmul_rn(acc.z, p.inv_alpha), __fmul_rn(acc.w, p.inv_alpha));
+          uint8_t* tile = p.lr + (size_t(mt) * p.RJ + size_t(c / kRChunk)) * kATileBytes;
+          *reinterpret_cast<uint2*>(tile + sw128(uint32_t(row), uint32_t(c % kRChunk) * 2u)) = w;
         }
       }
       cluster_sync();  // peers keep their shared memory until every read is done
@@ -307,7 +329,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 5 && lowrank) {
+  if (warp == kMmaWarp1 && lowrank) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);
   }
@@ -381,7 +403,7 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   const size_t smem = size_t(kStages1) * p.stage_bytes + kCtrlBytes + 1024;
   const int per_sm = smem <= 113 * 1024 ? 2 : 1;
   int splits = int((int64_t(per_sm) * a.num_sms) / ag.MT);
-  const int max_splits = a.r_tot > 0 ? 8 : 64;  // the cluster reduction needs a portable cluster
+  const int max_splits = a.r_tot > 0 ? kMaxSplits : 64;  // the cluster reduction needs a portable cluster
   if (splits > max_splits) splits = max_splits;
   if (splits > p.KC) splits = p.KC;
   if (splits < 1) splits = 1;
