@@ -183,7 +183,7 @@ svdq_status svdq_w4a4_linear(const svdq_layer* L, const void* act_buf, size_t ac
   if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
   if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU_TANH)
     return fail(SVDQ_ERR_INVALID_ARGUMENT, "unknown epilogue");
-  if (!aligned(Y, 16)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "Y must be 16-byte aligned");
+  if (!aligned(Y, 32)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "Y must be 32-byte aligned");
   if (!aligned(act_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf must be 256-byte aligned");
   const size_t need = svdq::make_act_geom(L->g, M).total;
   if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");

@@ -10,20 +10,33 @@
 //   acc += lr' L2                                 tcgen05.mma kind::f16, same TMEM tile
 //   Y    = bf16(act(alpha * acc + b)),  alpha = g_a g_w,  lr' = (X_hat L1) / alpha
 //
-// Design (sm_100a), persistent, one CTA per SM, 128 x 256 output tiles:
-//   * warp 8: one thread fills a 4-stage ring with 1D bulk copies (every
-//     operand is stored pre-tiled and pre-swizzled, so a stage is 4 copies:
-//     A codes 16 KB, B codes 32 KB, A scales 2 KB, B scales 4 KB); after the K
-//     loop of a tile it loads the lr' and L2^T chunks into the same ring;
-//   * warp 9: one thread copies the stage's block scales into tensor memory
-//     (tcgen05.cp 32x128b.warpx4), issues 4 block-scaled MMAs per 256-wide
-//     k-tile, then the bf16 MMAs of the fold, and commits stages back;
-//   * warps 0-7: epilogue, one output row x 128 columns per thread: tensor
-//     memory -> registers, release the accumulator, then alpha, bias, GELU ->
-//     bf16 -> global while the next tile's K loop runs.
-//   * Tensor memory: accumulator columns [0, 256), scale factors of stage s at
-//     256 + 16 s (A) and 320 + 32 s (B).
-//   * Every wait is bounded (status word + clean exit on timeout).
+// Design (sm_100a): persistent CTA pairs (clusters of 2, one CTA per SM) over
+// 256 x 256 output tiles with the 2-SM MMA (cta_group::2, M = 256):
+//   * CTA v of a pair owns A rows [128 v, 128 v + 128) and B rows (output
+//     features) [128 v, 128 v + 128) of the tile, and holds the tile's rows
+//     [128 v, 128 v + 128) x 256 columns of the accumulator in its tensor
+//     memory.  Sharing B across the pair cuts the operand bytes every SM
+//     streams per FLOP by 30 % against a 128 x 256 one-SM tile; the freed
+//     shared memory buys a fifth pipeline stage.
+//   * warp 8 of each CTA fills a 5-stage ring with tensor loads (one per
+//     operand, 2 KB rows) of the pre-tiled, pre-swizzled operands (A 16 KB, B half 16 KB, A scales 2 KB,
+//     all 256 rows of B scales 4 KB); completion is counted on the leader
+//     CTA's full barrier, which the leader arms with both CTAs' bytes.  After
+//     the K loop of a tile the same ring carries the lr' and L2^T chunks.
+//   * warp 9 of the leader copies each stage's block scales into both CTAs'
+//     tensor memory (tcgen05.cp, cta_group::2), issues 4 block-scaled MMAs per
+//     256-wide k-tile, then the bf16 MMAs of the fold, and commits every stage
+//     back to both CTAs' empty barriers with a multicast commit.
+//   * warps 0-7 of each CTA: epilogue, one output row x 128 columns per
+//     thread: tensor memory -> registers, release the accumulator to the
+//     leader, then alpha, bias, GELU -> bf16 -> global while the next tile's K
+//     loop runs.
+//   * Tensor memory (per CTA): accumulator columns [0, 256), scale factors of
+//     stage s at 256 + 16 s (A) and 336 + 32 s (B).
+//   * Every wait is bounded (status word + clean exit on timeout); the pair
+//     meets at a cluster barrier before freeing tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -37,32 +50,47 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kStages2 = 4;
+constexpr int kStages2 = 5;
 constexpr int kThreads2 = 320;  // warps 0-7 epilogue, 8 producer, 9 MMA
-constexpr int kEpiThreads = 256;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr uint32_t kOffA = 0, kOffB = kATileBytes, kOffSFA = kOffB + kBTileBytes;
-constexpr uint32_t kOffSFB = kOffSFA + kSFATileBytes;
-constexpr uint32_t kStage2 = kOffSFB + kSFBTileBytes;  // 55296 bytes
+constexpr uint32_t kHalf = 128;                          // rows per CTA of A and of B
+constexpr uint32_t kOffA = 0;                            // 16 KB
+constexpr uint32_t kOffB = kHalf * kRowBytes;            // 16 KB
+constexpr uint32_t kOffSFA = 2 * kHalf * kRowBytes;      // 2 KB
+constexpr uint32_t kOffSFB = kOffSFA + kSFATileBytes;    // 4 KB
+constexpr uint32_t kStage2 = kOffSFB + kSFBTileBytes;    // 38912 bytes
+constexpr uint32_t kFoldBytes = 2 * kHalf * kRowBytes;   // lr' 16 KB + L2^T half 16 KB
 constexpr uint32_t kCtrl2 = 128;
-constexpr uint32_t kBiasBytes = 8 * 2 * 128 * 4;  // per epilogue warp: 2 tiles x 128 floats
+constexpr uint32_t kBiasBytes = 8 * 2 * 128 * 4;         // per epilogue warp: 2 tiles x 128 floats
 constexpr uint32_t kTmemCols2 = 512;
-constexpr uint32_t kColSFA = 256, kColSFB = 320;
+constexpr uint32_t kColSFA = 256, kColSFB = kColSFA + 16 * kStages2;
+constexpr uint16_t kPairMask = 0x3;
 
 static_assert(kStage2 % 1024 == 0, "stage must keep 1 KB alignment");
 static_assert(kColSFB + kStages2 * 32 <= kTmemCols2, "tensor memory budget");
 
+// Every pre-tiled operand is viewed by its tensor map as rows of 2 KB (256
+// elements of 8 bytes), so a 16 KB tile is one load of 8 such rows.
+constexpr uint32_t kMapRow = 2048;
+constexpr int kRowsA = kHalf * kRowBytes / kMapRow;         // 8: 128 rows of A (or lr')
+constexpr int kRowsBTile = kBTileBytes / kMapRow;           // 16: a whole 256-row tile
+constexpr int kRowsSFA = kSFATileBytes / kMapRow;           // 1
+constexpr int kRowsSFB = kSFBTileBytes / kMapRow;           // 2
+
+struct alignas(64) GemmMaps {
+  CUtensorMap a;    // act codes, box = 128 rows of one tile (16 KB)
+  CUtensorMap asf;  // act scales, box = one k-tile (2 KB)
+  CUtensorMap lr;   // lr' tiles, box = 16 KB
+  CUtensorMap b;    // weight codes, box = half a 256-row tile (16 KB)
+  CUtensorMap bsf;  // weight scales, box = one k-tile of all 256 rows (4 KB)
+  CUtensorMap l2;   // L2^T tiles, box = half a tile (16 KB)
+};
+
 struct GemmParams {
-  const uint8_t* a_codes;
-  const uint8_t* a_sf;
-  const uint8_t* a_lr;
-  const uint8_t* b_codes;
-  const uint8_t* b_sf;
-  const uint8_t* b_l2t;
   const uint16_t* bias;  // padded to NT * 256, or null
   uint16_t* Y;
   uint32_t* status;
-  int32_t M, N, MT, NT, KT, RJ, r_tot, epilogue;
+  int32_t M, N, MP, NT, KT, RJ, r_tot, epilogue;
   float alpha;
   uint64_t timeout_ns;
 };
@@ -89,12 +117,12 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, const uint32_t*
     }
     out[e] = f32x2_to_bf16x2(y0, y1);
   }
-  uint4* dst = reinterpret_cast<uint4*>(p.Y + row * p.N + n0);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+  uint16_t* dst = p.Y + row * p.N + n0;  // 64 bytes, 64-byte aligned (n0 % 32 == 0, N % 64 == 0)
+  st_global_v8(dst, out);
+  st_global_v8(dst + 16, out + 8);
 }
 
-__global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) {
+__global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -102,31 +130,35 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
   const uint32_t sbase = raw_s + pad;
 
   const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
+  const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int pair = int(blockIdx.x >> 1), npairs = int(gridDim.x >> 1);
+
   uint8_t* ctrl = smem + kStages2 * kStage2;
   const uint32_t ctrl_s = sbase + kStages2 * kStage2;
-  const uint32_t FULL = ctrl_s, EMPTY = ctrl_s + 32u;
-  const uint32_t ACCF = ctrl_s + 64u, ACCE = ctrl_s + 72u, DRAIN = ctrl_s + 80u;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 88);
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 92);
+  const uint32_t FULL = ctrl_s, EMPTY = ctrl_s + 40u;
+  const uint32_t ACCF = ctrl_s + 80u, ACCE = ctrl_s + 88u, DRAIN = ctrl_s + 96u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 104);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 108);
   float* bias_s = reinterpret_cast<float*>(ctrl + kCtrl2);  // [warp][tile parity][128] floats
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
-      mbar_init(FULL + 8u * s, 1);
-      mbar_init(EMPTY + 8u * s, 1);
+      mbar_init(FULL + 8u * s, 1);   // leader: its producer's arrive + both CTAs' bytes
+      mbar_init(EMPTY + 8u * s, 1);  // both: one multicast commit per phase
     }
-    mbar_init(ACCF, 1);
-    mbar_init(ACCE, kEpiThreads);
+    mbar_init(ACCF, 1);   // both: one multicast commit per tile
+    mbar_init(ACCE, 16);  // leader: one arrival per epilogue warp of both CTAs
     mbar_init(DRAIN, 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(ctrl_s + 88u, kTmemCols2);
-    tmem_relinquish();
+    tmem_alloc_pair(ctrl_s + 104u, kTmemCols2);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -135,16 +167,20 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
     atomicOr(p.status, code);
   };
 
-  const int ntiles = p.MT * p.NT;
+  const int ntiles = p.MP * p.NT;
   const int nlr = (p.r_tot + kRChunk - 1) / kRChunk;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      prefetch_tensormap(&maps.a);
+      prefetch_tensormap(&maps.b);
+      prefetch_tensormap(&maps.asf);
+      prefetch_tensormap(&maps.bsf);
       uint32_t it = 0;
       bool stop = false;
-      for (int tile = int(blockIdx.x); tile < ntiles && !stop; tile += int(gridDim.x)) {
-        const int mt = tile % p.MT, nt = tile / p.MT;
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+        const int mt = 2 * (tile % p.MP) + int(rank), nt = tile / p.MP;
         for (int kt = 0; kt < p.KT; ++kt) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
@@ -153,12 +189,12 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
             break;
           }
           const uint32_t st = sbase + s * kStage2;
-          const uint32_t bar = FULL + 8u * s;
-          mbar_expect_tx(bar, kStage2);
-          bulk_g2s(st + kOffA, p.a_codes + (size_t(mt) * p.KT + kt) * kATileBytes, kATileBytes, bar);
-          bulk_g2s(st + kOffB, p.b_codes + (size_t(nt) * p.KT + kt) * kBTileBytes, kBTileBytes, bar);
-          bulk_g2s(st + kOffSFA, p.a_sf + (size_t(mt) * p.KT + kt) * kSFATileBytes, kSFATileBytes, bar);
-          bulk_g2s(st + kOffSFB, p.b_sf + (size_t(nt) * p.KT + kt) * kSFBTileBytes, kSFBTileBytes, bar);
+          const uint32_t bar = mapa(FULL + 8u * s, 0u);
+          if (leader) mbar_expect_tx(FULL + 8u * s, 2u * kStage2);
+          tma_load_2d_pair(st + kOffA, &maps.a, 0, (mt * p.KT + kt) * kRowsA, bar);
+          tma_load_2d_pair(st + kOffB, &maps.b, 0, (nt * p.KT + kt) * kRowsBTile + int(rank) * kRowsA, bar);
+          tma_load_2d_pair(st + kOffSFA, &maps.asf, 0, (mt * p.KT + kt) * kRowsSFA, bar);
+          tma_load_2d_pair(st + kOffSFB, &maps.bsf, 0, (nt * p.KT + kt) * kRowsSFB, bar);
           ++it;
         }
         for (int j = 0; j < nlr && !stop; ++j) {
@@ -169,25 +205,26 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
             break;
           }
           const uint32_t st = sbase + s * kStage2;
-          const uint32_t bar = FULL + 8u * s;
-          mbar_expect_tx(bar, kATileBytes + kBTileBytes);
-          bulk_g2s(st + kOffA, p.a_lr + (size_t(mt) * p.RJ + j) * kATileBytes, kATileBytes, bar);
-          bulk_g2s(st + kOffB, p.b_l2t + (size_t(nt) * p.RJ + j) * kBTileBytes, kBTileBytes, bar);
+          const uint32_t bar = mapa(FULL + 8u * s, 0u);
+          if (leader) mbar_expect_tx(FULL + 8u * s, 2u * kFoldBytes);
+          tma_load_2d_pair(st + kOffA, &maps.lr, 0, (mt * p.RJ + j) * kRowsA, bar);
+          tma_load_2d_pair(st + kOffB, &maps.l2, 0, (nt * p.RJ + j) * kRowsBTile + int(rank) * kRowsA, bar);
           ++it;
         }
       }
-      // every issued copy must land before this CTA may exit
-      for (uint32_t i = it > kStages2 ? it - kStages2 : 0; i < it; ++i)
-        mbar_wait(FULL + 8u * (i % kStages2), (i / kStages2) & 1u, nullptr, p.timeout_ns);
+      // every issued copy (of both CTAs) must land before the pair may exit
+      if (leader)
+        for (uint32_t i = it > kStages2 ? it - kStages2 : 0; i < it; ++i)
+          mbar_wait(FULL + 8u * (i % kStages2), (i / kStages2) & 1u, nullptr, p.timeout_ns);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      const uint32_t id_fp4 = idesc_nvfp4(kBN), id_bf16 = idesc_bf16(kBN);
+    // ------------------------------------------------------ MMA issue (leader)
+    if (leader && lane == 0) {
+      const uint32_t id_fp4 = idesc_nvfp4_m256(kBN), id_bf16 = idesc_bf16_m256(kBN);
       uint32_t it = 0, tc = 0;
       bool stop = false, any = false;
-      for (int tile = int(blockIdx.x); tile < ntiles && !stop; tile += int(gridDim.x)) {
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
         if (!mbar_wait(ACCE, (tc & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
           fail(0x20u);
           break;
@@ -205,15 +242,15 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
           const uint32_t sfa = tmem + kColSFA + 16u * s, sfb = tmem + kColSFB + 32u * s;
 #pragma unroll
           for (uint32_t kb = 0; kb < 4; ++kb) {
-            tc_cp_32x128b_warpx4(sfa + 4u * kb, sdesc_sf(st + kOffSFA + kb * kSFAtomBytes));
-            tc_cp_32x128b_warpx4(sfb + 8u * kb, sdesc_sf(st + kOffSFB + (2u * kb) * kSFAtomBytes));
-            tc_cp_32x128b_warpx4(sfb + 8u * kb + 4u, sdesc_sf(st + kOffSFB + (2u * kb + 1u) * kSFAtomBytes));
+            tc_cp_32x128b_warpx4_pair(sfa + 4u * kb, sdesc_sf(st + kOffSFA + kb * kSFAtomBytes));
+            tc_cp_32x128b_warpx4_pair(sfb + 8u * kb, sdesc_sf(st + kOffSFB + (2u * kb) * kSFAtomBytes));
+            tc_cp_32x128b_warpx4_pair(sfb + 8u * kb + 4u, sdesc_sf(st + kOffSFB + (2u * kb + 1u) * kSFAtomBytes));
           }
 #pragma unroll
           for (uint32_t kb = 0; kb < 4; ++kb)
-            umma_nvfp4(tmem, sdesc_sw128(st + kOffA + 32u * kb), sdesc_sw128(st + kOffB + 32u * kb), id_fp4,
-                       sfa + 4u * kb, sfb + 8u * kb, (kt | int(kb)) ? 1u : 0u);
-          tc_commit(EMPTY + 8u * s);
+            umma_nvfp4_pair(tmem, sdesc_sw128(st + kOffA + 32u * kb), sdesc_sw128(st + kOffB + 32u * kb), id_fp4,
+                            sfa + 4u * kb, sfb + 8u * kb, (kt | int(kb)) ? 1u : 0u);
+          tc_commit_pair_mc(EMPTY + 8u * s, kPairMask);
           any = true;
           ++it;
         }
@@ -229,34 +266,33 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
           const int left = p.r_tot - kRChunk * j;
           const int nks = (left < kRChunk ? left : kRChunk) / 16;
           for (int ks = 0; ks < nks; ++ks)
-            umma_bf16(tmem, sdesc_sw128(st + kOffA + 32u * ks), sdesc_sw128(st + kOffB + 32u * ks), id_bf16, 1u);
-          tc_commit(EMPTY + 8u * s);
+            umma_bf16_pair(tmem, sdesc_sw128(st + kOffA + 32u * ks), sdesc_sw128(st + kOffB + 32u * ks), id_bf16, 1u);
+          tc_commit_pair_mc(EMPTY + 8u * s, kPairMask);
           ++it;
         }
         if (stop) break;
-        tc_commit(ACCF);
+        tc_commit_pair_mc(ACCF, kPairMask);
         ++tc;
       }
       if (any) {
-        tc_commit(DRAIN);
+        tc_commit_pair(DRAIN);
         mbar_wait(DRAIN, 0u, nullptr, p.timeout_ns);
       }
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------- epilogue
-    // warp w reads TMEM lanes 32 (w % 4) .. +31 (its lane quarter) and
-    // accumulator columns 128 (w / 4) .. +127: the whole 128 x 256 tile is
-    // read into registers, the accumulator is released, then the rows are
+    // warp w reads TMEM lanes 32 (w % 4) .. +31 and accumulator columns
+    // 128 (w / 4) .. +127: the whole 128 x 256 share of the tile goes to
+    // registers, the accumulator is released to the leader, then the rows are
     // finished and stored while the next tile's K loop runs.
     uint32_t tc = 0;
     const int quarter = warp & 3, colhalf = warp >> 2;
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colhalf * 128);
-    for (int tile = int(blockIdx.x); tile < ntiles; tile += int(gridDim.x)) {
-      const int mt = tile % p.MT, nt = tile / p.MT;
-      // stage this warp's 128 bias values while the K loop runs (warp-private,
-      // double buffered by tile parity: only __syncwarp is needed)
+    for (int tile = pair; tile < ntiles; tile += npairs) {
+      const int mt = 2 * (tile % p.MP) + int(rank), nt = tile / p.MP;
+      // stage this warp's 128 bias values (warp-private, double buffered)
       float* bias_w = bias_s + (size_t(warp) * 2 + (tc & 1u)) * 128;
       if (p.bias) {
         const uint2 w = *reinterpret_cast<const uint2*>(p.bias + size_t(nt) * kBN + colhalf * 128 + lane * 4);
@@ -277,7 +313,8 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
       tmem_ld32(tl + 96u, v + 96);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(ACCE);  // the accumulator may be overwritten now
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
       const int64_t row = int64_t(mt) * kBM + row_in_tile;
       if (row < p.M) {
 #pragma unroll
@@ -293,11 +330,36 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
 
   // ------------------------------------------------------------ teardown
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs are done with every MMA, copy and tensor-memory read
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols2);
+    tmem_dealloc_pair(tmem, kTmemCols2);
   }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// A pre-tiled operand of `bytes` bytes viewed as rows of 2 KB; one load = `box` rows.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t bytes, uint32_t box) {
+  auto enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {kMapRow / 8u, bytes / kMapRow};
+  const cuuint64_t strides[1] = {kMapRow};
+  const cuuint32_t boxd[2] = {kMapRow / 8u, box};
+  const cuuint32_t es[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(base), dims, strides, boxd, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -305,19 +367,31 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const GemmParams p) 
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   const LayerGeom& lg = a.lg;
   const ActGeom ag = make_act_geom(lg, a.M);
+  GemmMaps maps;
+  const uint8_t* act = a.act;
+  const uint8_t* lay = a.layer;
+  bool ok = encode_rows(&maps.a, act + ag.off_codes, uint64_t(ag.MT) * ag.KT * kATileBytes, kRowsA) &&
+            encode_rows(&maps.asf, act + ag.off_sf, uint64_t(ag.MT) * ag.KT * kSFATileBytes, kRowsSFA) &&
+            encode_rows(&maps.b, lay + lg.off_bcodes, uint64_t(lg.NT) * lg.KT * kBTileBytes, kRowsA) &&
+            encode_rows(&maps.bsf, lay + lg.off_sfb, uint64_t(lg.NT) * lg.KT * kSFBTileBytes, kRowsSFB);
+  if (ok && lg.RJ > 0) {
+    ok = encode_rows(&maps.lr, act + ag.off_lr, uint64_t(ag.MT) * ag.RJ * kATileBytes, kRowsA) &&
+         encode_rows(&maps.l2, lay + lg.off_l2t, uint64_t(lg.NT) * lg.RJ * kBTileBytes, kRowsA);
+  } else {
+    maps.lr = maps.a;  // never read without low-rank chunks
+    maps.l2 = maps.b;
+  }
+  if (!ok) {
+    *why = "cuTensorMapEncodeTiled rejected a GEMM operand";
+    return cudaErrorInvalidValue;
+  }
   GemmParams p{};
-  p.a_codes = a.act + ag.off_codes;
-  p.a_sf = a.act + ag.off_sf;
-  p.a_lr = a.act + ag.off_lr;
-  p.b_codes = a.layer + lg.off_bcodes;
-  p.b_sf = a.layer + lg.off_sfb;
-  p.b_l2t = a.layer + lg.off_l2t;
-  p.bias = a.has_bias ? reinterpret_cast<const uint16_t*>(a.layer + lg.off_bias) : nullptr;
+  p.bias = a.has_bias ? reinterpret_cast<const uint16_t*>(lay + lg.off_bias) : nullptr;
   p.Y = static_cast<uint16_t*>(a.Y);
-  p.status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.layer) + lg.off_status);
+  p.status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(lay) + lg.off_status);
   p.M = int32_t(a.M);
   p.N = int32_t(lg.N);
-  p.MT = int32_t(ag.MT);
+  p.MP = int32_t(ag.MT / 2);
   p.NT = int32_t(lg.NT);
   p.KT = int32_t(lg.KT);
   p.RJ = int32_t(lg.RJ);
@@ -326,28 +400,55 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   p.alpha = a.alpha;
   p.timeout_ns = a.timeout_ns;
 
-  const int64_t ntiles = ag.MT * lg.NT;
+  const int64_t ntiles = int64_t(p.MP) * lg.NT;
   if (ntiles > (int64_t(1) << 30)) {
-    *why = "too many output tiles";
+    *why = "problem too large for one launch";
     return cudaErrorInvalidValue;
   }
   const size_t smem = size_t(kStages2) * kStage2 + kCtrl2 + kBiasBytes + 1024;
-  {
-    static std::atomic<int> set_on[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!set_on[dev & 63].load()) {
-      cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      if (e != cudaSuccess) {
-        *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
-        return e;
-      }
-      set_on[dev & 63].store(1);
+  static std::atomic<int> max_pairs[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (max_pairs[dev & 63].load() == 0) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) {
+      *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
+      return e;
     }
+    cudaLaunchConfig_t q{};
+    q.gridDim = dim3(2 * unsigned(a.num_sms / 2), 1, 1);
+    q.blockDim = dim3(kThreads2, 1, 1);
+    q.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    q.attrs = at;
+    q.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel, &q);
+    if (e != cudaSuccess || clusters < 1) {
+      *why = "no CTA pair of the GEMM fits on this device";
+      return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+    }
+    max_pairs[dev & 63].store(clusters);
   }
-  const int grid = int(ntiles < a.num_sms ? ntiles : a.num_sms);
-  gemm_kernel<<<grid, kThreads2, smem, s>>>(p);
-  cudaError_t e = cudaGetLastError();
+  const int cap = max_pairs[dev & 63].load();
+  const int pairs = int(ntiles < cap ? ntiles : cap);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(kThreads2, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, maps, p);
   if (e != cudaSuccess) *why = "launch of the GEMM kernel failed";
   return e;
 }

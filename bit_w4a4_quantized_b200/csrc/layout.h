@@ -112,6 +112,8 @@ SVDQ_HD size_t l2t_off(const LayerGeom& g, int64_t n, int64_t rho) {
 }
 
 // ---------------------------------------------------------- activation buffer
+// Rows are padded to an even number of 128-row tiles; the padding rows hold
+// zero codes and scales (kernel 1 reads them as zeros past the end of X).
 struct ActGeom {
   int64_t M, MT, KT, RJ;
   size_t off_codes, off_sf, off_lr, total;
@@ -120,7 +122,7 @@ struct ActGeom {
 SVDQ_HD ActGeom make_act_geom(const LayerGeom& lg, int64_t M) {
   ActGeom a{};
   a.M = M;
-  a.MT = ceil_div(M, kBM);
+  a.MT = round_up(ceil_div(M, kBM), 2);  // the GEMM works on pairs of 128-row tiles
   a.KT = lg.KT;
   a.RJ = lg.RJ;
   size_t o = 0;

@@ -165,7 +165,7 @@ SVDQ_API svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, i
  * block-scaled MMA and the bf16 up projection accumulating into the same
  * tensor-memory tile.
  * act_buf: the buffer svdq_quantize_act filled for the same M.
- * Y: device bf16 [M, N] row-major, 16-byte aligned.
+ * Y: device bf16 [M, N] row-major, 32-byte aligned.
  * epilogue: SVDQ_EPI_NONE or SVDQ_EPI_GELU_TANH (bias is added first).
  */
 SVDQ_API svdq_status svdq_w4a4_linear(const svdq_layer* layer, const void* act_buf, size_t act_buf_bytes,

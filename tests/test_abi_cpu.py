@@ -107,9 +107,11 @@ def test_buffer_sizes_follow_tiling():
     spec = WL.CFG1
     X = spec.x()
     layer = svdq.Layer(spec.w(), np.max(np.abs(X.astype(np.float32)), 0), 16, rank_capacity=48)
-    # activation tiles: 128 rows x (256 K -> 16 KB codes + 2 KB scales) + 1 chunk of 64 ranks (16 KB)
-    assert layer.act_buffer_bytes(1) == 16384 + 2048 + 16384
-    assert layer.act_buffer_bytes(129) == 2 * (16384 + 2048 + 16384)
+    # activation tiles of 128 rows, an even number of them: (256 K -> 16 KB codes
+    # + 2 KB scales) + 1 chunk of 64 ranks (16 KB) per tile
+    assert layer.act_buffer_bytes(1) == 2 * (16384 + 2048 + 16384)
+    assert layer.act_buffer_bytes(256) == 2 * (16384 + 2048 + 16384)
+    assert layer.act_buffer_bytes(257) == 4 * (16384 + 2048 + 16384)
     info = layer.info()
     assert (info.K, info.N, info.rank, info.rank_total, info.rank_capacity) == (256, 256, 16, 16, 48)
     assert info.dev_buf is None and info.device == -1
