@@ -20,7 +20,8 @@ the prepared layer) whose total exceeds the 126 MB L2, so every step reads
 its operands from HBM.  CUDA events on the launching stream, max over ranks.
 value = 2 M N K / step time, summed over ranks (weak scaling: every rank
 runs its own batch; the layer has no cross-GPU exchange, so ranks are
-replicas).  See the design doc for the roofline accounting.
+replicas).  The roofline of each kernel counts its algorithmic bytes or
+flops per launch (the formulas are in layer_flops and run_ours).
 """
 
 import argparse
@@ -167,6 +168,47 @@ def measured_peaks():
         d = json.load(open(p))
         return d.get("bf16_tflops"), d.get("hbm_gbs"), "measured"
     return 1590.0, 6650.0, "fallback"
+
+
+KERNEL_SOURCES = {
+    "gemm_kernel": ("gemm.cu", "ptx.cuh", "layout.h", "kernels.h"),
+    "act_quant_kernel": ("act_quant.cu", "ptx.cuh", "layout.h", "kernels.h"),
+}
+PROFILE_FILES = {
+    "gemm_kernel": "gemm_kernel_attention_projection.md",
+    "act_quant_kernel": "act_quant_kernel_attention_projection.md",
+}
+
+
+def kernel_source_hash(kernel):
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "bit_w4a4_quantized_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from the committed ncu summary,
+    or None if the summary is for another workload or the kernel's source changed since the capture."""
+    if workload != "attn_proj_M4096_K3072_N3072_r32":
+        return None
+    path = os.path.join(ROOT, "profiles", PROFILE_FILES[kernel])
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if "=" in line:
+            k, _, v = line.strip().partition("=")
+            fields[k.strip()] = v.strip()
+    if fields.get("source_sha256_16") != kernel_source_hash(kernel):
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 # -------------------------------------------------------------- CPU oracle
@@ -361,13 +403,17 @@ def run_ours(args):
     k1_bytes = 2 * M * K + M * K // 2 + M * K // 16 + 2 * M * r_tot + 2 * K * r_tot + 4 * K
     if per_k2 >= per_k1:
         roof = {"kernel": "svdq_gemm (kernel 2)", "bound": "tensor", "achieved": k2_flops / per_k2 / 1e12,
-                "peak": k2_flops / k2_roof_s / 1e12, "unit": "TFLOP/s", "traffic": None}
+                "peak": k2_flops / k2_roof_s / 1e12, "unit": "TFLOP/s",
+                "traffic": profiled_traffic("gemm_kernel", spec.name),
+                "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture "
+                                  "(profiles/gemm_kernel_attention_projection.md); Y stays in L2 during the kernel"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["peak_basis"] = (f"{peak_src} bf16 {bf16_peak} TF/s x 4 (nominal FP4:BF16) for the FP4 flops, "
                               f"bf16 {bf16_peak} TF/s for the fold")
     else:
         roof = {"kernel": "act_quant (kernel 1)", "bound": "hbm", "achieved": k1_bytes / per_k1 / 1e9,
-                "peak": hbm_peak, "unit": "GB/s", "traffic": None, "peak_basis": f"{peak_src} HBM copy"}
+                "peak": hbm_peak, "unit": "GB/s", "traffic": profiled_traffic("act_quant_kernel", spec.name),
+                "peak_basis": f"{peak_src} HBM copy"}
         roof["frac"] = roof["achieved"] / roof["peak"]
 
     clocks = clk.summary()
@@ -406,6 +452,158 @@ def run_ours(args):
     return 0
 
 
+# ------------------------------------------------------------------ sweep
+def _graph_seconds(graphs, steps, stream, device):
+    """Mean seconds per replay of `graphs` (rotated), CUDA events on `stream`."""
+    import torch
+
+    with torch.cuda.stream(stream):
+        for i in range(3 * len(graphs)):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize(device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    return e0.elapsed_time(e1) / 1e3 / steps
+
+
+def _capture(fns, stream):
+    import torch
+
+    graphs = []
+    for fn in fns:
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=stream, capture_error_mode="thread_local"):
+            fn()
+        graphs.append(cg)
+    return graphs
+
+
+def sweep_point(spec, device, steps, factors_cache):
+    """Kernel times of one shape at its rank and at rank 0, next to a bf16 cuBLAS linear.
+
+    Low-rank factors come from one library SVD per (K, N) at the largest rank
+    swept, truncated to each rank (timing does not depend on their values)."""
+    import torch
+    import torch.nn.functional as F
+
+    from bit_w4a4_quantized_b200 import svdq
+    from bit_w4a4_quantized_b200 import workloads as WL
+
+    M, K, N = spec.M, spec.K, spec.N
+    r = spec.rank + (spec.lora_rank or 0)  # an attached adapter only adds ranks to the branch
+    X = WL.make_x(M, K, spec.seed, spec.x_dist, spec.x_outliers, spec.x_outlier_scale)
+    W = spec.w()
+    bias = spec.b()
+    amax = svdq.calibrate_amax(X)
+    key = (K, N)
+    r_max = max(64, r)
+    if r > 0 and key not in factors_cache:
+        base = svdq.Layer(W, amax, r_max, device=None)
+        factors_cache[key] = (base.export(svdq.EXPORT_L1), base.export(svdq.EXPORT_L2))
+        base.close()
+    epi = svdq.EPI_GELU_TANH if spec.gelu else svdq.EPI_NONE
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.uint16).astype(np.int16)).view(
+        torch.bfloat16).to(device)
+    Xd = to_dev(X)
+    stream = torch.cuda.Stream(device)
+    out = {"workload": spec.name, "M": M, "K": K, "N": N, "rank": spec.rank, "rank_total": r,
+           "epilogue": "gelu_tanh" if spec.gelu else "none", "bias": bias is not None}
+
+    def layer_at(rank):
+        fac = None
+        if rank > 0:
+            L1, L2 = factors_cache[key]
+            fac = (np.ascontiguousarray(L1[:, :rank]), np.ascontiguousarray(L2[:rank]))
+        return svdq.Layer(W, amax, rank, bias=bias, factors=fac, device=device)
+
+    per_set = None
+    for rank, tag in ((r, "fused"), (0, "plain")) if r > 0 else ((0, "plain"),):
+        L0 = layer_at(rank)
+        per_set = L0.device_bytes + L0.act_buffer_bytes(M) + 2 * M * K + 2 * M * N
+        nsets = int(min(8, max(2, math.ceil(3 * L2_BYTES / per_set))))
+        layers = [L0] + [layer_at(rank) for _ in range(nsets - 1)]
+        Xs = [Xd] + [Xd.clone() for _ in range(nsets - 1)]
+        acts = [L.new_act_buffer(M) for L in layers]
+        Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+        with torch.cuda.stream(stream):
+            for i in range(nsets):
+                layers[i].quantize_act(Xs[i], acts[i])
+                layers[i].linear(acts[i], M, out=Ys[i], epilogue=epi)
+            stream.synchronize()
+        k1 = _capture([lambda i=i: layers[i].quantize_act(Xs[i], acts[i]) for i in range(nsets)], stream)
+        k2 = _capture([lambda i=i: layers[i].linear(acts[i], M, out=Ys[i], epilogue=epi) for i in range(nsets)],
+                      stream)
+        t1 = _graph_seconds(k1, steps, stream, device)
+        t2 = _graph_seconds(k2, steps, stream, device)
+        for L in layers:
+            L.poll_status()
+        out[f"{tag}_act_us"] = round(t1 * 1e6, 3)
+        out[f"{tag}_gemm_us"] = round(t2 * 1e6, 3)
+        out[f"{tag}_layer_us"] = round((t1 + t2) * 1e6, 3)
+        out[f"{tag}_gemm_TFLOPs"] = round(2 * M * N * K / t2 / 1e12, 1)
+        out[f"{tag}_layer_TFLOPs"] = round(2 * M * N * K / (t1 + t2) / 1e12, 1)
+        del k1, k2
+        for L in layers:
+            L.close()
+        del layers, acts, Ys, Xs
+    # bf16 cuBLAS dense GEMM of the same shape (X W^T, no bias or activation)
+    Wd = to_dev(W)
+    nsets = int(min(8, max(2, math.ceil(3 * L2_BYTES / (2 * (M * K + N * K + M * N))))))
+    Xs = [Xd] + [Xd.clone() for _ in range(nsets - 1)]
+    Ws = [Wd] + [Wd.clone() for _ in range(nsets - 1)]
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+
+    mm = [lambda i=i: torch.matmul(Xs[i], Ws[i].t(), out=Ys[i]) for i in range(nsets)]
+    with torch.cuda.stream(stream):
+        for f in mm:
+            f()
+        stream.synchronize()
+    gl = _capture(mm, stream)
+    t_cb = _graph_seconds(gl, steps, stream, device)
+    out["cublas_bf16_us"] = round(t_cb * 1e6, 3)
+    out["cublas_bf16_TFLOPs"] = round(2 * M * N * K / t_cb / 1e12, 1)
+    if r > 0:
+        out["lowrank_overhead_layer"] = round(out["fused_layer_us"] / out["plain_layer_us"] - 1, 4)
+        out["lowrank_overhead_gemm"] = round(out["fused_gemm_us"] / out["plain_gemm_us"] - 1, 4)
+        out["speedup_vs_cublas_bf16"] = round(t_cb / (out["fused_layer_us"] * 1e-6), 3)
+    else:
+        out["speedup_vs_cublas_bf16"] = round(t_cb / (out["plain_layer_us"] * 1e-6), 3)
+    del gl
+    return out
+
+
+def run_sweep(args):
+    import torch
+
+    from bit_w4a4_quantized_b200 import workloads as WL
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    names = args.sweep.split(",")
+    specs = []
+    for n in names:
+        if n == "all":
+            specs += [WL.CFG2, WL.CFG3_FC1, WL.CFG3_FC2, WL.CFG4] + WL.sweep()
+        elif n == "sweep":
+            specs += WL.sweep()
+        else:
+            specs.append(workload_spec(n))
+    cache = {}
+    props = torch.cuda.get_device_properties(device)
+    for spec in specs:
+        with ClockSampler(getattr(props, "uuid", None)) as clk:
+            row = sweep_point(spec, device, args.sweep_steps, cache)
+        row["clocks"] = clk.summary()
+        print(json.dumps(row), flush=True)
+        torch.cuda.empty_cache()
+    return 0
+
+
 # --------------------------------------------------------- reference arm
 def run_reference(args):
     rank, world, _ = dist_env()
@@ -439,7 +637,12 @@ def main(argv=None):
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", default=None,
+                    help="per-shape report instead of the bench line: 'all', 'sweep' or workload names, comma separated")
+    ap.add_argument("--sweep-steps", type=int, default=50)
     args = ap.parse_args(argv)
+    if args.sweep:
+        return run_sweep(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     _, world, _ = dist_env()

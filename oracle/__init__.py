@@ -20,7 +20,7 @@ low-rank branch without re-quantizing R.  The Diffusers/Nunchaku page adds:
 NVFP4 (Blackwell), compute dtype bfloat16, QKV fusion along the output dim.
 
 Every reading the pages leave open (NVFP4 two-level scales, rounding, sign of
-zero, static activation scale, ...) is listed in the design doc and in the
+zero, static activation scale, ...) is stated in the
 docstrings of ``formats`` and ``svdquant``.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``

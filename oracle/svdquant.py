@@ -14,7 +14,7 @@ scales input channel j of both X and W^T:
                                                  (section 4.2, eq. W_hat = L1 L2 + R)
     Y       = Q(X_hat) Q(R) + (X_hat L1) L2 + b  (section 4.2, decomposition of XW)
 
-Readings of what the pages leave open (also listed in the design doc):
+Readings of what the pages leave open:
   * lambda_j = sqrt(max|X_:,j| / max|W_:,j|) (SmoothQuant migration strength
     1/2), 1 where either maximum is 0; every step correctly rounded float32.
   * Sigma goes wholly into L1 (L1 = U Sigma_r, as the page writes it); L1 and
