@@ -297,11 +297,9 @@ def run_ours(args):
     act_bytes = layer0.act_buffer_bytes(M)
     per_set = layer0.device_bytes + act_bytes + 2 * M * K + 2 * M * N
     nsets = int(min(16, max(2, math.ceil(3 * L2_BYTES / per_set))))
-    factors = (layer0.export(svdq.EXPORT_L1), layer0.export(svdq.EXPORT_L2)) if spec.rank else None
     layers = [layer0]
-    for _ in range(nsets - 1):
-        L = svdq.Layer(W, amax, spec.rank, rank_capacity=layer0.info().rank_capacity, bias=bias, factors=factors,
-                       device=device)
+    for _ in range(nsets - 1):  # device copies of the same prepared layer
+        L = layer0.clone(device=device)
         if spec.lora_rank:
             L.lora_swap(*lora_dev)
         layers.append(L)
@@ -496,11 +494,20 @@ def sweep_point(spec, device, steps, factors_cache):
 
     M, K, N = spec.M, spec.K, spec.N
     r = spec.rank + (spec.lora_rank or 0)  # an attached adapter only adds ranks to the branch
-    X = WL.make_x(M, K, spec.seed, spec.x_dist, spec.x_outliers, spec.x_outlier_scale)
-    W = spec.w()
+    cache = factors_cache
+    xkey = (M, K, spec.seed, spec.x_dist, spec.x_outliers, spec.x_outlier_scale)
+    if cache.get("x_key") != xkey:  # consecutive points often share X (and W)
+        cache["x_key"], cache["x"] = xkey, None
+        cache["x"] = WL.make_x(M, K, spec.seed, spec.x_dist, spec.x_outliers, spec.x_outlier_scale)
+        cache["amax"] = svdq.calibrate_amax(cache["x"])
+    X, amax = cache["x"], cache["amax"]
+    wkey = (N, K, spec.seed, spec.w_outliers, spec.w_outlier_scale, spec.w_stream, spec.w_outlier_stream)
+    if cache.get("w_key") != wkey:
+        cache["w_key"], cache["w"] = wkey, None
+        cache["w"] = spec.w()
+    W = cache["w"]
     bias = spec.b()
-    amax = svdq.calibrate_amax(X)
-    key = (K, N)
+    key = (K, N, spec.seed)  # one SVD per weight; its factors serve every M (timing ignores their values)
     r_max = max(64, r)
     if r > 0 and key not in factors_cache:
         base = svdq.Layer(W, amax, r_max, device=None)
@@ -526,7 +533,7 @@ def sweep_point(spec, device, steps, factors_cache):
         L0 = layer_at(rank)
         per_set = L0.device_bytes + L0.act_buffer_bytes(M) + 2 * M * K + 2 * M * N
         nsets = int(min(8, max(2, math.ceil(3 * L2_BYTES / per_set))))
-        layers = [L0] + [layer_at(rank) for _ in range(nsets - 1)]
+        layers = [L0] + [L0.clone(device=device) for _ in range(nsets - 1)]
         Xs = [Xd] + [Xd.clone() for _ in range(nsets - 1)]
         acts = [L.new_act_buffer(M) for L in layers]
         Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]

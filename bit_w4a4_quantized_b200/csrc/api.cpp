@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <new>
 #include <string>
 
 #include "kernels.h"
@@ -282,6 +283,23 @@ svdq_status svdq_poll_status(const svdq_layer* L, void* stream) {
 }
 
 void svdq_layer_destroy(svdq_layer* L) { delete L; }
+
+svdq_status svdq_layer_clone(const svdq_layer* L, svdq_layer** out) {
+  if (!L || !out) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and out are required");
+  svdq_layer* c = nullptr;
+  try {
+    c = new svdq_layer(*L);
+  } catch (const std::bad_alloc&) {
+    return fail(SVDQ_ERR_HOST_ALLOC, "host allocation failed while copying the layer");
+  }
+  c->dev_buf = nullptr;
+  c->dev_bytes = 0;
+  c->device = -1;
+  c->num_sms = 0;
+  c->r_tot = c->g.rank;
+  *out = c;
+  return SVDQ_OK;
+}
 
 void svdq_test_override_device_arch(int sm) { g_arch_override.store(sm); }
 

@@ -127,7 +127,7 @@ void quantize_row(const float* t, int64_t k, float g, float c, PutByte&& put_byt
 
 template <class F>
 void parallel_rows(int64_t n, int threads, F&& f) {
-  if (threads <= 1 || n < 64) {
+  if (threads <= 1 || n < 2) {
     f(int64_t(0), n);
     return;
   }
@@ -196,12 +196,13 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
 
     // 2. smoothed weight W_hat^T [K, N] in float64 (exact: float32 x bf16)
     std::vector<double> R(size_t(K) * N);
-    parallel_rows(K, threads, [&](int64_t k0, int64_t k1) {
-      for (int64_t k = k0; k < k1; ++k) {
-        const double lam = L->lam[k];
-        double* row = &R[size_t(k) * N];
-        for (int64_t n = 0; n < N; ++n) row[n] = lam * double(bf16_bits_to_f32(d->W[n * K + k]));
-      }
+    //    (transposed in 64 x 64 blocks so both sides stay in cache)
+    parallel_rows(ceil_div(K, 64), threads, [&](int64_t b0, int64_t b1) {
+      for (int64_t kb = b0 * 64; kb < std::min(K, b1 * 64); kb += 64)
+        for (int64_t nb = 0; nb < N; nb += 64)
+          for (int64_t n = nb; n < std::min(N, nb + 64); ++n)
+            for (int64_t k = kb; k < std::min(K, kb + 64); ++k)
+              R[size_t(k) * N + n] = double(L->lam[k]) * double(bf16_bits_to_f32(d->W[n * K + k]));
     });
 
     // 3. low-rank factors, bf16 [K, r] and [r, N]
@@ -265,9 +266,11 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
 
     // 5. R^T as float32 [N, K], tensor scale, NVFP4 codes into the image
     std::vector<float> rt(size_t(N) * K);
-    parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
-      for (int64_t n = n0; n < n1; ++n)
-        for (int64_t k = 0; k < K; ++k) rt[size_t(n) * K + k] = float(R[size_t(k) * N + n]);
+    parallel_rows(ceil_div(N, 64), threads, [&](int64_t b0, int64_t b1) {
+      for (int64_t nb = b0 * 64; nb < std::min(N, b1 * 64); nb += 64)
+        for (int64_t kb = 0; kb < K; kb += 64)
+          for (int64_t k = kb; k < std::min(K, kb + 64); ++k)
+            for (int64_t n = nb; n < std::min(N, nb + 64); ++n) rt[size_t(n) * K + k] = float(R[size_t(k) * N + n]);
     });
     if (d->flags & SVDQ_PREPARE_KEEP_R) {
       L->r32.resize(size_t(K) * N);

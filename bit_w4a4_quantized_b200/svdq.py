@@ -46,7 +46,7 @@ EXPORTED_SYMBOLS = (
     "svdq_prepare_host", "svdq_layer_upload", "svdq_prepare_weights", "svdq_act_buffer_bytes",
     "svdq_quantize_act", "svdq_w4a4_linear", "svdq_lora_swap", "svdq_layer_export", "svdq_act_unpack",
     "svdq_get_layer_info", "svdq_poll_status", "svdq_layer_destroy", "svdq_test_override_device_arch",
-    "svdq_test_bounded_wait",
+    "svdq_test_bounded_wait", "svdq_layer_clone",
 )
 
 
@@ -108,6 +108,7 @@ def lib():
         "svdq_get_layer_info": ([vp, ctypes.POINTER(LayerInfo)], st),
         "svdq_poll_status": ([vp, vp], st),
         "svdq_layer_destroy": ([vp], None),
+        "svdq_layer_clone": ([vp, ctypes.POINTER(vp)], st),
         "svdq_test_override_device_arch": ([ctypes.c_int], None),
         "svdq_test_bounded_wait": ([ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32), vp], st),
     }
@@ -210,6 +211,17 @@ class Layer:
         self.dev_buf = None
         if device is not None:
             self.upload(device, stream)
+
+    def clone(self, device=None, stream=None):
+        """A second handle with the same prepared weights (base rank, no adapter), optionally uploaded."""
+        h = ctypes.c_void_p()
+        check(lib().svdq_layer_clone(self._h, ctypes.byref(h)))
+        c = Layer.__new__(Layer)
+        c._h, c._keep, c.desc = h, None, self.desc
+        c.N, c.K, c.rank, c.device_bytes, c.dev_buf = self.N, self.K, self.rank, self.device_bytes, None
+        if device is not None:
+            c.upload(device, stream)
+        return c
 
     # ------------------------------------------------------------- device side
     def upload(self, device="cuda", stream=None):

@@ -233,6 +233,16 @@ SVDQ_API svdq_status svdq_poll_status(const svdq_layer* layer, void* stream);
 SVDQ_API void svdq_layer_destroy(svdq_layer* layer);
 
 /*
+ * Host-only copy of a prepared layer: the packed image in its base state
+ * (rank r, no adapter), lambda, the factors and the scalars, not bound to any
+ * device buffer.  Upload the copy to another buffer or another GPU (one
+ * replica per GPU, or several copies on one GPU) without repeating the
+ * preparation.  Attached adapters are not copied.  *out must be released
+ * with svdq_layer_destroy.  No CUDA call.
+ */
+SVDQ_API svdq_status svdq_layer_clone(const svdq_layer* layer, svdq_layer** out);
+
+/*
  * Test hooks.
  * svdq_test_override_device_arch: pretend the device reports this sm version
  * (e.g. 90) in the capability checks; 0 restores the real query.

@@ -116,3 +116,19 @@ def test_buffer_sizes_follow_tiling():
     assert (info.K, info.N, info.rank, info.rank_total, info.rank_capacity) == (256, 256, 16, 16, 48)
     assert info.dev_buf is None and info.device == -1
     assert info.device_bytes == layer.device_bytes > 0
+
+
+def test_clone_copies_the_prepared_layer_and_outlives_it():
+    spec = WL.CFG1
+    X = spec.x()
+    layer = svdq.Layer(spec.w(), svdq.calibrate_amax(X), spec.rank)
+    twin = layer.clone()
+    want = {e: layer.export(e) for e in (svdq.EXPORT_LAMBDA, svdq.EXPORT_L1, svdq.EXPORT_L2, svdq.EXPORT_W_CODES,
+                                         svdq.EXPORT_W_SCALES, svdq.EXPORT_SCALARS)}
+    layer.close()
+    for e, v in want.items():
+        np.testing.assert_array_equal(twin.export(e), v)
+    assert twin.info().rank_total == spec.rank
+    # not bound to a device buffer: launching must be refused, not crash
+    st = svdq.lib().svdq_quantize_act(twin._h, 1, 1, 1, 1, None)
+    assert st == svdq.ERR_INVALID_ARGUMENT

@@ -197,3 +197,20 @@ def test_two_calls_share_nothing_between_layers():
     assert torch.equal(Ya.view(torch.int16), Ya2.view(torch.int16))
     check_y(b, Yb, check_act(b, act_b))
     _same_act(a, act_a, act_a2, 64)
+
+
+def test_clone_on_another_buffer_gives_identical_output():
+    spec = WL.CFG1
+    case = _spec_case(spec, rank_capacity=spec.rank + 16)
+    _, Y0 = case.run()
+    A, B = WL.make_lora(spec.K, spec.N, 16, seed=1)
+    Ad = torch.from_numpy(A.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    Bd = torch.from_numpy(B.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    case.layer.lora_swap(Ad, Bd)  # the clone must not inherit the adapter
+    twin = case.layer.clone(device="cuda")
+    assert twin.info().rank_total == spec.rank
+    act = twin.quantize_act(case.Xd)
+    Y1 = twin.linear(act, spec.M)
+    torch.cuda.synchronize()
+    assert torch.equal(Y0.view(torch.int16), Y1.view(torch.int16))
+    twin.poll_status()
