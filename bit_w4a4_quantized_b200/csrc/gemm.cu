@@ -19,14 +19,19 @@
 //     streams per FLOP by 30 % against a 128 x 256 one-SM tile; the freed
 //     shared memory buys a fifth pipeline stage.
 //   * warp 8 of each CTA fills a 5-stage ring with tensor loads (one per
-//     operand, 2 KB rows) of the pre-tiled, pre-swizzled operands (A 16 KB, B half 16 KB, A scales 2 KB,
-//     all 256 rows of B scales 4 KB); completion is counted on the leader
-//     CTA's full barrier, which the leader arms with both CTAs' bytes.  After
-//     the K loop of a tile the same ring carries the lr' and L2^T chunks.
-//   * warp 9 of the leader copies each stage's block scales into both CTAs'
-//     tensor memory (tcgen05.cp, cta_group::2), issues 4 block-scaled MMAs per
-//     256-wide k-tile, then the bf16 MMAs of the fold, and commits every stage
-//     back to both CTAs' empty barriers with a multicast commit.
+//     operand, 2 KB rows) of the pre-tiled, pre-swizzled operands: A 16 KB and
+//     the B half 16 KB counted on the leader CTA's full barrier (armed by the
+//     leader with both CTAs' bytes), A scales 2 KB and all 256 rows of B scales
+//     4 KB counted on the CTA's own scale barrier.  After the K loop of a tile
+//     the same ring carries the lr' and L2^T chunks.
+//   * warps 10-13 of each CTA (one per tensor-memory lane quarter) move each
+//     stage's block scales from shared memory into their CTA's tensor memory
+//     with tcgen05.st, in the replicated layout the block-scaled MMA reads,
+//     then arrive on the leader's full barrier.  Scale staging therefore
+//     never occupies the tensor pipe, which issues nothing but MMAs.
+//   * warp 9 of the leader issues 4 block-scaled MMAs per 256-wide k-tile,
+//     then the bf16 MMAs of the fold, and commits every stage back to both
+//     CTAs' empty barriers with a multicast commit.
 //   * warps 0-7 of each CTA: epilogue, one output row x 128 columns per
 //     thread: tensor memory -> registers, release the accumulator to the
 //     leader, then alpha, bias, GELU -> bf16 -> global while the next tile's K
@@ -51,8 +56,9 @@ namespace {
 using namespace ptx;
 
 constexpr int kStages2 = 5;
-constexpr int kThreads2 = 320;  // warps 0-7 epilogue, 8 producer, 9 MMA
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads2 = 448;  // warps 0-7 epilogue, 8 producer, 9 MMA, 10-13 scales
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kScaleWarp0 = 10;
+constexpr int kFullArrivals = 1 + 2 * 4;  // leader producer + the scale warps of both CTAs
 constexpr uint32_t kHalf = 128;                          // rows per CTA of A and of B
 constexpr uint32_t kOffA = 0;                            // 16 KB
 constexpr uint32_t kOffB = kHalf * kRowBytes;            // 16 KB
@@ -60,7 +66,7 @@ constexpr uint32_t kOffSFA = 2 * kHalf * kRowBytes;      // 2 KB
 constexpr uint32_t kOffSFB = kOffSFA + kSFATileBytes;    // 4 KB
 constexpr uint32_t kStage2 = kOffSFB + kSFBTileBytes;    // 38912 bytes
 constexpr uint32_t kFoldBytes = 2 * kHalf * kRowBytes;   // lr' 16 KB + L2^T half 16 KB
-constexpr uint32_t kCtrl2 = 128;
+constexpr uint32_t kCtrl2 = 256;
 constexpr uint32_t kBiasBytes = 8 * 2 * 128 * 4;         // per epilogue warp: 2 tiles x 128 floats
 constexpr uint32_t kTmemCols2 = 512;
 constexpr uint32_t kColSFA = 256, kColSFB = kColSFA + 16 * kStages2;
@@ -101,11 +107,9 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return 0.5f * x * (1.0f + tanh_approx(u));
 }
 
-// 32 accumulator columns of one row -> alpha, bias, act -> bf16 -> 64 bytes of Y.
+// 32 accumulator columns of one row -> alpha, bias, act -> 16 words of bf16 pairs.
 // `bias` points at the 32 bias values of these columns in shared memory (or null).
-__device__ __forceinline__ void store_chunk(const GemmParams& p, const uint32_t* v, const float* bias, int64_t row,
-                                            int n0) {
-  uint32_t out[16];
+__device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t* v, const float* bias, uint32_t* out) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const float b0 = bias ? bias[2 * e] : 0.0f, b1 = bias ? bias[2 * e + 1] : 0.0f;
@@ -117,9 +121,6 @@ __device__ __forceinline__ void store_chunk(const GemmParams& p, const uint32_t*
     }
     out[e] = f32x2_to_bf16x2(y0, y1);
   }
-  uint16_t* dst = p.Y + row * p.N + n0;  // 64 bytes, 64-byte aligned (n0 % 32 == 0, N % 64 == 0)
-  st_global_v8(dst, out);
-  st_global_v8(dst + 16, out + 8);
 }
 
 __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
@@ -140,12 +141,14 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   const uint32_t ACCF = ctrl_s + 80u, ACCE = ctrl_s + 88u, DRAIN = ctrl_s + 96u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 104);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 108);
+  const uint32_t SFULL = ctrl_s + 112u;  // 5 barriers: this CTA's scales of a stage have landed
   float* bias_s = reinterpret_cast<float*>(ctrl + kCtrl2);  // [warp][tile parity][128] floats
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
-      mbar_init(FULL + 8u * s, 1);   // leader: its producer's arrive + both CTAs' bytes
-      mbar_init(EMPTY + 8u * s, 1);  // both: one multicast commit per phase
+      mbar_init(FULL + 8u * s, kFullArrivals);  // leader: producer (+ both CTAs' A/B bytes) + 8 scale warps
+      mbar_init(EMPTY + 8u * s, 1);             // both: one multicast commit per phase
+      mbar_init(SFULL + 8u * s, 1);             // both: own producer (+ own scale bytes)
     }
     mbar_init(ACCF, 1);   // both: one multicast commit per tile
     mbar_init(ACCE, 16);  // leader: one arrival per epilogue warp of both CTAs
@@ -190,11 +193,12 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           }
           const uint32_t st = sbase + s * kStage2;
           const uint32_t bar = mapa(FULL + 8u * s, 0u);
-          if (leader) mbar_expect_tx(FULL + 8u * s, 2u * kStage2);
+          if (leader) mbar_expect_tx(FULL + 8u * s, 2u * kOffSFA);
+          mbar_expect_tx(SFULL + 8u * s, kStage2 - kOffSFA);
           tma_load_2d_pair(st + kOffA, &maps.a, 0, (mt * p.KT + kt) * kRowsA, bar);
           tma_load_2d_pair(st + kOffB, &maps.b, 0, (nt * p.KT + kt) * kRowsBTile + int(rank) * kRowsA, bar);
-          tma_load_2d_pair(st + kOffSFA, &maps.asf, 0, (mt * p.KT + kt) * kRowsSFA, bar);
-          tma_load_2d_pair(st + kOffSFB, &maps.bsf, 0, (nt * p.KT + kt) * kRowsSFB, bar);
+          tma_load_2d(st + kOffSFA, &maps.asf, 0, (mt * p.KT + kt) * kRowsSFA, SFULL + 8u * s);
+          tma_load_2d(st + kOffSFB, &maps.bsf, 0, (nt * p.KT + kt) * kRowsSFB, SFULL + 8u * s);
           ++it;
         }
         for (int j = 0; j < nlr && !stop; ++j) {
@@ -207,15 +211,17 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           const uint32_t st = sbase + s * kStage2;
           const uint32_t bar = mapa(FULL + 8u * s, 0u);
           if (leader) mbar_expect_tx(FULL + 8u * s, 2u * kFoldBytes);
+          mbar_arrive(SFULL + 8u * s);  // no scales in a fold stage: the scale warps only pass it on
           tma_load_2d_pair(st + kOffA, &maps.lr, 0, (mt * p.RJ + j) * kRowsA, bar);
           tma_load_2d_pair(st + kOffB, &maps.l2, 0, (nt * p.RJ + j) * kRowsBTile + int(rank) * kRowsA, bar);
           ++it;
         }
       }
       // every issued copy (of both CTAs) must land before the pair may exit
-      if (leader)
-        for (uint32_t i = it > kStages2 ? it - kStages2 : 0; i < it; ++i)
-          mbar_wait(FULL + 8u * (i % kStages2), (i / kStages2) & 1u, nullptr, p.timeout_ns);
+      for (uint32_t i = it > kStages2 ? it - kStages2 : 0; i < it; ++i) {
+        mbar_wait(SFULL + 8u * (i % kStages2), (i / kStages2) & 1u, nullptr, p.timeout_ns);
+        if (leader) mbar_wait_cluster(FULL + 8u * (i % kStages2), (i / kStages2) & 1u, nullptr, p.timeout_ns);
+      }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         tc_fence_after();
         for (int kt = 0; kt < p.KT; ++kt) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
-          if (!mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
+          if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
             fail(0x20u);
             stop = true;
             break;
@@ -240,12 +246,6 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           tc_fence_after();
           const uint32_t st = sbase + s * kStage2;
           const uint32_t sfa = tmem + kColSFA + 16u * s, sfb = tmem + kColSFB + 32u * s;
-#pragma unroll
-          for (uint32_t kb = 0; kb < 4; ++kb) {
-            tc_cp_32x128b_warpx4_pair(sfa + 4u * kb, sdesc_sf(st + kOffSFA + kb * kSFAtomBytes));
-            tc_cp_32x128b_warpx4_pair(sfb + 8u * kb, sdesc_sf(st + kOffSFB + (2u * kb) * kSFAtomBytes));
-            tc_cp_32x128b_warpx4_pair(sfb + 8u * kb + 4u, sdesc_sf(st + kOffSFB + (2u * kb + 1u) * kSFAtomBytes));
-          }
 #pragma unroll
           for (uint32_t kb = 0; kb < 4; ++kb)
             umma_nvfp4_pair(tmem, sdesc_sw128(st + kOffA + 32u * kb), sdesc_sw128(st + kOffB + 32u * kb), id_fp4,
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         }
         for (int j = 0; j < nlr && !stop; ++j) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
-          if (!mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
+          if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
             fail(0x20u);
             stop = true;
             break;
@@ -280,12 +280,57 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       }
     }
     __syncwarp();
+  } else if (warp >= kScaleWarp0) {
+    // --------------------------------------------------------- scale warps
+    // Warp w writes tensor-memory lanes 32 q .. 32 q + 31, q = w % 4.  For k block
+    // kb the MMA reads A scales at column 256 + 16 s + 4 kb and B scales at
+    // 336 + 32 s + 8 kb (B rows 0-127) and + 4 (rows 128-255), with lane i of
+    // every quarter holding word w = row i + 32 w of each 512-byte atom: the
+    // atom's 16-byte row i replicated into every quarter.
+    const uint32_t q = uint32_t(warp & 3);
+    const uint32_t lanes = (32u * q) << 16;
+    uint32_t it = 0;
+    bool stop = false;
+    for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+      for (int k = 0; k < p.KT + nlr && !stop; ++k) {
+        const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
+        bool ok = mbar_wait(SFULL + 8u * s, ph, abort_flag, p.timeout_ns);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0 && *abort_flag == 0u) fail(0x80u);
+          stop = true;
+          break;
+        }
+        if (k < p.KT) {
+          const uint8_t* st = smem + s * kStage2;
+          uint32_t ra[16], rb[32];
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 a = *reinterpret_cast<const uint4*>(st + kOffSFA + kb * kSFAtomBytes + lane * 16);
+            ra[4 * kb] = a.x, ra[4 * kb + 1] = a.y, ra[4 * kb + 2] = a.z, ra[4 * kb + 3] = a.w;
+          }
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            const uint4 b = *reinterpret_cast<const uint4*>(st + kOffSFB + h * kSFAtomBytes + lane * 16);
+            rb[4 * h] = b.x, rb[4 * h + 1] = b.y, rb[4 * h + 2] = b.z, rb[4 * h + 3] = b.w;
+          }
+          tmem_st16(tmem + lanes + kColSFA + 16u * s, ra);
+          tmem_st32(tmem + lanes + kColSFB + 32u * s, rb);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(FULL + 8u * s, 0u);
+        ++it;
+      }
+    }
   } else {
     // ------------------------------------------------------------- epilogue
     // warp w reads TMEM lanes 32 (w % 4) .. +31 and accumulator columns
-    // 128 (w / 4) .. +127: the whole 128 x 256 share of the tile goes to
-    // registers, the accumulator is released to the leader, then the rows are
-    // finished and stored while the next tile's K loop runs.
+    // 128 (w / 4) .. +127, 64 columns at a time, and keeps the finished row
+    // as 64 words of bf16 pairs; the accumulator is released to the leader
+    // before the 256 bytes of each row are stored, while the next tile's K
+    // loop runs.
     uint32_t tc = 0;
     const int quarter = warp & 3, colhalf = warp >> 2;
     const int row_in_tile = quarter * 32 + lane;
@@ -306,12 +351,16 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         break;
       }
       tc_fence_after();
-      uint32_t v[128];
-      tmem_ld32(tl, v);
-      tmem_ld32(tl + 32u, v + 32);
-      tmem_ld32(tl + 64u, v + 64);
-      tmem_ld32(tl + 96u, v + 96);
-      tmem_wait_ld();
+      uint32_t out[64];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[64];
+        tmem_ld32(tl + 64u * h, v);
+        tmem_ld32(tl + 64u * h + 32u, v + 32);
+        tmem_wait_ld();
+        finish_chunk(p, v, p.bias ? bias_w + h * 64 : nullptr, out + 32 * h);
+        finish_chunk(p, v + 32, p.bias ? bias_w + h * 64 + 32 : nullptr, out + 32 * h + 16);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
@@ -319,9 +368,13 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       if (row < p.M) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int c0 = colhalf * 128 + q * 32;
-          const int n0 = nt * kBN + c0;
-          if (n0 < p.N) store_chunk(p, v + 32 * q, p.bias ? bias_w + q * 32 : nullptr, row, n0);
+          const int n0 = nt * kBN + colhalf * 128 + q * 32;
+          // 64 bytes at a 32-byte aligned address (n0 % 32 == 0, N % 64 == 0, Y 32-byte aligned)
+          uint16_t* dst = p.Y + row * p.N + n0;
+          if (n0 < p.N) {
+            st_global_v8(dst, out + 16 * q);
+            st_global_v8(dst + 16, out + 16 * q + 8);
+          }
         }
       }
       ++tc;
