@@ -56,8 +56,9 @@ namespace {
 using namespace ptx;
 
 constexpr int kStages2 = 5;
-constexpr int kThreads2 = 448;  // warps 0-7 epilogue, 8 producer, 9 MMA, 10-13 scales
-constexpr int kProducerWarp = 8, kMmaWarp = 9, kScaleWarp0 = 10;
+constexpr int kEpiWarps = 16;    // warp w: lane quarter w % 4, accumulator columns 64 (w / 4) .. +63
+constexpr int kThreads2 = 704;  // warps 0-15 epilogue, 16-19 scales, 20 producer, 21 MMA
+constexpr int kScaleWarp0 = 16, kProducerWarp = 20, kMmaWarp = 21;
 constexpr int kFullArrivals = 1 + 2 * 4;  // leader producer + the scale warps of both CTAs
 constexpr uint32_t kHalf = 128;                          // rows per CTA of A and of B
 constexpr uint32_t kOffA = 0;                            // 16 KB
@@ -67,7 +68,7 @@ constexpr uint32_t kOffSFB = kOffSFA + kSFATileBytes;    // 4 KB
 constexpr uint32_t kStage2 = kOffSFB + kSFBTileBytes;    // 38912 bytes
 constexpr uint32_t kFoldBytes = 2 * kHalf * kRowBytes;   // lr' 16 KB + L2^T half 16 KB
 constexpr uint32_t kCtrl2 = 256;
-constexpr uint32_t kBiasBytes = 8 * 2 * 128 * 4;         // per epilogue warp: 2 tiles x 128 floats
+constexpr uint32_t kBiasBytes = kEpiWarps * 2 * 64 * 4;  // per epilogue warp: 2 tiles x 64 floats
 constexpr uint32_t kTmemCols2 = 512;
 constexpr uint32_t kColSFA = 256, kColSFB = kColSFA + 16 * kStages2;
 constexpr uint16_t kPairMask = 0x3;
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 104);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 108);
   const uint32_t SFULL = ctrl_s + 112u;  // 5 barriers: this CTA's scales of a stage have landed
-  float* bias_s = reinterpret_cast<float*>(ctrl + kCtrl2);  // [warp][tile parity][128] floats
+  float* bias_s = reinterpret_cast<float*>(ctrl + kCtrl2);  // [warp][tile parity][64] floats
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       mbar_init(SFULL + 8u * s, 1);             // both: own producer (+ own scale bytes)
     }
     mbar_init(ACCF, 1);   // both: one multicast commit per tile
-    mbar_init(ACCE, 16);  // leader: one arrival per epilogue warp of both CTAs
+    mbar_init(ACCE, 2 * kEpiWarps);  // leader: one arrival per epilogue warp of both CTAs
     mbar_init(DRAIN, 1);
     *abort_flag = 0u;
     fence_mbar_init();
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       }
     }
     __syncwarp();
-  } else if (warp >= kScaleWarp0) {
+  } else if (warp >= kScaleWarp0) {  // warps 16-19
     // --------------------------------------------------------- scale warps
     // Warp w writes tensor-memory lanes 32 q .. 32 q + 31, q = w % 4.  For k block
     // kb the MMA reads A scales at column 256 + 16 s + 4 kb and B scales at
@@ -303,19 +304,25 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         }
         if (k < p.KT) {
           const uint8_t* st = smem + s * kStage2;
-          uint32_t ra[16], rb[32];
+          {
+            uint32_t r[16];
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint4 a = *reinterpret_cast<const uint4*>(st + kOffSFA + kb * kSFAtomBytes + lane * 16);
-            ra[4 * kb] = a.x, ra[4 * kb + 1] = a.y, ra[4 * kb + 2] = a.z, ra[4 * kb + 3] = a.w;
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint4 a = *reinterpret_cast<const uint4*>(st + kOffSFA + kb * kSFAtomBytes + lane * 16);
+              r[4 * kb] = a.x, r[4 * kb + 1] = a.y, r[4 * kb + 2] = a.z, r[4 * kb + 3] = a.w;
+            }
+            tmem_st16(tmem + lanes + kColSFA + 16u * s, r);
           }
 #pragma unroll
-          for (int h = 0; h < 8; ++h) {
-            const uint4 b = *reinterpret_cast<const uint4*>(st + kOffSFB + h * kSFAtomBytes + lane * 16);
-            rb[4 * h] = b.x, rb[4 * h + 1] = b.y, rb[4 * h + 2] = b.z, rb[4 * h + 3] = b.w;
+          for (int half = 0; half < 2; ++half) {
+            uint32_t r[16];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const uint4 b = *reinterpret_cast<const uint4*>(st + kOffSFB + (4 * half + h) * kSFAtomBytes + lane * 16);
+              r[4 * h] = b.x, r[4 * h + 1] = b.y, r[4 * h + 2] = b.z, r[4 * h + 3] = b.w;
+            }
+            tmem_st16(tmem + lanes + kColSFB + 32u * s + 16u * half, r);
           }
-          tmem_st16(tmem + lanes + kColSFA + 16u * s, ra);
-          tmem_st32(tmem + lanes + kColSFB + 32u * s, rb);
           tmem_wait_st();
         }
         tc_fence_before();
@@ -327,21 +334,20 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   } else {
     // ------------------------------------------------------------- epilogue
     // warp w reads TMEM lanes 32 (w % 4) .. +31 and accumulator columns
-    // 128 (w / 4) .. +127, 64 columns at a time, and keeps the finished row
-    // as 64 words of bf16 pairs; the accumulator is released to the leader
-    // before the 256 bytes of each row are stored, while the next tile's K
-    // loop runs.
+    // 64 (w / 4) .. +63: its share of the tile goes to registers, the
+    // accumulator is released to the leader, then the rows are finished and
+    // stored while the next tile's K loop runs.
     uint32_t tc = 0;
-    const int quarter = warp & 3, colhalf = warp >> 2;
+    const int quarter = warp & 3, colq = warp >> 2;
     const int row_in_tile = quarter * 32 + lane;
-    const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colhalf * 128);
+    const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colq * 64);
     for (int tile = pair; tile < ntiles; tile += npairs) {
       const int mt = 2 * (tile % p.MP) + int(rank), nt = tile / p.MP;
-      // stage this warp's 128 bias values (warp-private, double buffered)
-      float* bias_w = bias_s + (size_t(warp) * 2 + (tc & 1u)) * 128;
+      // stage this warp's 64 bias values (warp-private, double buffered)
+      float* bias_w = bias_s + (size_t(warp) * 2 + (tc & 1u)) * 64;
       if (p.bias) {
-        const uint2 w = *reinterpret_cast<const uint2*>(p.bias + size_t(nt) * kBN + colhalf * 128 + lane * 4);
-        *reinterpret_cast<float4*>(bias_w + lane * 4) = make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p.bias + size_t(nt) * kBN + colq * 64 + lane * 2);
+        *reinterpret_cast<float2*>(bias_w + lane * 2) = make_float2(bf16lo(w), bf16hi(w));
       }
       __syncwarp();
       bool ok = mbar_wait(ACCF, tc & 1u, abort_flag, p.timeout_ns);
@@ -351,29 +357,25 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         break;
       }
       tc_fence_after();
-      uint32_t out[64];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t v[64];
-        tmem_ld32(tl + 64u * h, v);
-        tmem_ld32(tl + 64u * h + 32u, v + 32);
-        tmem_wait_ld();
-        finish_chunk(p, v, p.bias ? bias_w + h * 64 : nullptr, out + 32 * h);
-        finish_chunk(p, v + 32, p.bias ? bias_w + h * 64 + 32 : nullptr, out + 32 * h + 16);
-      }
+      uint32_t v[64];
+      tmem_ld32(tl, v);
+      tmem_ld32(tl + 32u, v + 32);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
       const int64_t row = int64_t(mt) * kBM + row_in_tile;
       if (row < p.M) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int n0 = nt * kBN + colhalf * 128 + q * 32;
-          // 64 bytes at a 32-byte aligned address (n0 % 32 == 0, N % 64 == 0, Y 32-byte aligned)
-          uint16_t* dst = p.Y + row * p.N + n0;
+        for (int q = 0; q < 2; ++q) {
+          const int n0 = nt * kBN + colq * 64 + q * 32;
           if (n0 < p.N) {
-            st_global_v8(dst, out + 16 * q);
-            st_global_v8(dst + 16, out + 16 * q + 8);
+            uint32_t out[16];
+            finish_chunk(p, v + 32 * q, p.bias ? bias_w + q * 32 : nullptr, out);
+            // 64 bytes at a 32-byte aligned address (n0 % 32 == 0, N % 64 == 0, Y 32-byte aligned)
+            uint16_t* dst = p.Y + row * p.N + n0;
+            st_global_v8(dst, out);
+            st_global_v8(dst + 16, out + 8);
           }
         }
       }
