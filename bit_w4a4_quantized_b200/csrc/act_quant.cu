@@ -112,6 +112,9 @@ __device__ __forceinline__ void store_lr8(const ActQuantParams& p, int mt, uint3
   *reinterpret_cast<uint4*>(tile + sw128(row, uint32_t(c % kRChunk) * 2u)) = w;
 }
 
+// kLowRank = false (rank 0) leaves out every tensor-core instruction: a kernel
+// that allocates tensor memory runs one CTA per SM, the plain quantizer two.
+template <bool kLowRank>
 __global__ void __launch_bounds__(kThreads1, 2)
     act_quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const ActQuantParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kThreads1, 2)
   const int kc0 = int(int64_t(split) * p.KC / p.splits);
   const int kc1 = int(int64_t(split + 1) * p.KC / p.splits);
   const int nchunks = kc1 - kc0;
-  const bool lowrank = p.r_tot > 0;
+  constexpr bool lowrank = kLowRank;
 
   uint8_t* ctrl = smem + kStages1 * p.stage_bytes;
   const uint32_t ctrl_s = sbase + kStages1 * p.stage_bytes;
@@ -149,10 +152,13 @@ __global__ void __launch_bounds__(kThreads1, 2)
     tmem_alloc(ctrl_s + 112u, p.tmem_cols);
     tmem_relinquish();
   }
-  tc_fence_before();
+  if (lowrank) tc_fence_before();
   __syncthreads();
-  tc_fence_after();
+  if (lowrank) tc_fence_after();
   const uint32_t tmem = lowrank ? *tmem_slot : 0u;
+  // X may be the previous kernel's output and the activation buffer its input
+  griddep_wait();
+  griddep_launch_dependents();
 
   auto fail = [&](uint32_t code) {
     *abort_flag = 1u;
@@ -327,7 +333,7 @@ __global__ void __launch_bounds__(kThreads1, 2)
   }
 
   // ------------------------------------------------------------ teardown
-  tc_fence_before();
+  if (lowrank) tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp1 && lowrank) {
     tc_fence_after();
@@ -409,16 +415,21 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   if (splits < 1) splits = 1;
   p.splits = splits;
 
+  const bool lowrank = a.r_tot > 0;
+  auto kernel = lowrank ? act_quant_kernel<true> : act_quant_kernel<false>;
   {
-    // the attribute is per device: remember the largest value set on each
-    static std::atomic<size_t> smem_set[64];
+    // the attributes are per device and kernel: remember the largest size set on each
+    static std::atomic<size_t> smem_set[2][64];
     int dev = 0;
     cudaGetDevice(&dev);
-    std::atomic<size_t>& done = smem_set[dev & 63];
+    std::atomic<size_t>& done = smem_set[lowrank ? 1 : 0][dev & 63];
     if (smem > done.load()) {
-      cudaError_t e = cudaFuncSetAttribute(act_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+      if (e == cudaSuccess)  // all of the unified L1 as shared memory: two CTAs per SM must fit
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 int(cudaSharedmemCarveoutMaxShared));
       if (e != cudaSuccess) {
-        *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
+        *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
         return e;
       }
       done.store(smem);
@@ -429,16 +440,19 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   cfg.blockDim = dim3(kThreads1, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  if (a.r_tot > 0 && splits > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = unsigned(splits);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (lowrank && splits > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = unsigned(splits);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, act_quant_kernel, map, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, map, p);
   if (e != cudaSuccess) *why = "launch of the activation kernel failed";
   return e;
 }

@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the activation buffer is the previous kernel's output, Y may be its input
+  griddep_wait();
+  griddep_launch_dependents();
 
   auto fail = [&](uint32_t code) {
     *abort_flag = 1u;
@@ -466,8 +469,11 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   cudaGetDevice(&dev);
   if (max_pairs[dev & 63].load() == 0) {
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               int(cudaSharedmemCarveoutMaxShared));
     if (e != cudaSuccess) {
-      *why = "cudaFuncSetAttribute(max dynamic shared memory) failed";
+      *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
       return e;
     }
     cudaLaunchConfig_t q{};
@@ -496,13 +502,15 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   cfg.blockDim = dim3(kThreads2, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, maps, p);
   if (e != cudaSuccess) *why = "launch of the GEMM kernel failed";
   return e;
