@@ -325,35 +325,47 @@ def run_ours(args):
             L.poll_status()
 
     def capture(fn):
-        graphs = []
+        """One graph running fn over every buffer set in turn (launch cost amortised over nsets
+        steps), and one graph per set for a remainder."""
+        whole = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(whole, stream=stream, capture_error_mode="thread_local"):
+            for i in range(nsets):
+                fn(i)
+        singles = []
         for i in range(nsets):
             cg = torch.cuda.CUDAGraph()
             with torch.cuda.graph(cg, stream=stream, capture_error_mode="thread_local"):
                 fn(i)
-            graphs.append(cg)
-        return graphs
+            singles.append(cg)
+        return whole, singles
 
     step_graphs = capture(lambda i: (q(i), g(i)))
     k1_graphs = capture(q)
     k2_graphs = capture(g)
 
-    def timed(graphs, steps, sampler=None):
+    def replay(graphs, steps):
+        whole, singles = graphs
+        for _ in range(steps // nsets):
+            whole.replay()
+        for i in range(steps % nsets):
+            singles[i].replay()
+
+    def timed(graphs, steps):
+        """Seconds for exactly `steps` steps, CUDA events on the launching stream."""
         with torch.cuda.stream(stream):
             barrier(device)
             torch.cuda.synchronize(device)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for i in range(steps):
-                graphs[i % nsets].replay()
+            replay(graphs, steps)
             e1.record(stream)
             torch.cuda.synchronize(device)
             barrier(device)
         return e0.elapsed_time(e1) / 1e3
 
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            step_graphs[i % nsets].replay()
+        replay(step_graphs, args.warmup)
     props = torch.cuda.get_device_properties(device)
     with ClockSampler(getattr(props, "uuid", None)) as clk:
         t_step = timed(step_graphs, args.steps)
@@ -424,7 +436,8 @@ def run_ours(args):
                    "bias": bias is not None, "epilogue": "gelu_tanh" if spec.gelu else "none",
                    "lora": lora_note, "parallelism": f"replicas x{world} (no collective on the data path)",
                    "l2": f"rotating {nsets} buffer sets of {per_set / 2**20:.1f} MiB (X, act, Y, layer copy): "
-                         f"{nsets * per_set / 2**20:.0f} MiB > L2", "timing": "CUDA graph per step, CUDA events"},
+                         f"{nsets * per_set / 2**20:.0f} MiB > L2",
+                   "timing": f"CUDA graphs of {nsets} steps (one per buffer set), CUDA events"},
         "kernels": {"act_quant_us": round(per_k1 * 1e6, 3), "gemm_us": round(per_k2 * 1e6, 3),
                     "act_quant_GBps": round(k1_bytes / per_k1 / 1e9, 1),
                     "gemm_TFLOPs": round(k2_flops / per_k2 / 1e12, 1), "flops_fp4": fp4,
@@ -443,42 +456,42 @@ def run_ours(args):
                                          f"host has {os.cpu_count()} logical cores"}
     if rank == 0:
         print(json.dumps(out), flush=True)
-    for cg in step_graphs + k1_graphs + k2_graphs:
-        del cg
+    del step_graphs, k1_graphs, k2_graphs
     if world > 1:
         dist.destroy_process_group()
     return 0
 
 
 # ------------------------------------------------------------------ sweep
-def _graph_seconds(graphs, steps, stream, device):
-    """Mean seconds per replay of `graphs` (rotated), CUDA events on `stream`."""
+def _graph_seconds(graph, launches, steps, stream, device):
+    """Mean seconds per launch: `graph` holds `launches` launches (one per buffer set) and is
+    replayed until about `steps` launches ran; CUDA events on `stream`."""
     import torch
 
+    reps = max(1, steps // launches)
     with torch.cuda.stream(stream):
-        for i in range(3 * len(graphs)):
-            graphs[i % len(graphs)].replay()
+        for _ in range(3):
+            graph.replay()
         torch.cuda.synchronize(device)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(steps):
-            graphs[i % len(graphs)].replay()
+        for _ in range(reps):
+            graph.replay()
         e1.record(stream)
         torch.cuda.synchronize(device)
-    return e0.elapsed_time(e1) / 1e3 / steps
+    return e0.elapsed_time(e1) / 1e3 / (reps * launches)
 
 
 def _capture(fns, stream):
+    """One CUDA graph running every fn in turn."""
     import torch
 
-    graphs = []
-    for fn in fns:
-        cg = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(cg, stream=stream, capture_error_mode="thread_local"):
+    cg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(cg, stream=stream, capture_error_mode="thread_local"):
+        for fn in fns:
             fn()
-        graphs.append(cg)
-    return graphs
+    return cg
 
 
 def sweep_point(spec, device, steps, factors_cache):
@@ -545,8 +558,8 @@ def sweep_point(spec, device, steps, factors_cache):
         k1 = _capture([lambda i=i: layers[i].quantize_act(Xs[i], acts[i]) for i in range(nsets)], stream)
         k2 = _capture([lambda i=i: layers[i].linear(acts[i], M, out=Ys[i], epilogue=epi) for i in range(nsets)],
                       stream)
-        t1 = _graph_seconds(k1, steps, stream, device)
-        t2 = _graph_seconds(k2, steps, stream, device)
+        t1 = _graph_seconds(k1, nsets, steps, stream, device)
+        t2 = _graph_seconds(k2, nsets, steps, stream, device)
         for L in layers:
             L.poll_status()
         out[f"{tag}_act_us"] = round(t1 * 1e6, 3)
@@ -571,7 +584,7 @@ def sweep_point(spec, device, steps, factors_cache):
             f()
         stream.synchronize()
     gl = _capture(mm, stream)
-    t_cb = _graph_seconds(gl, steps, stream, device)
+    t_cb = _graph_seconds(gl, nsets, steps, stream, device)
     out["cublas_bf16_us"] = round(t_cb * 1e6, 3)
     out["cublas_bf16_TFLOPs"] = round(2 * M * N * K / t_cb / 1e12, 1)
     if r > 0:
