@@ -56,7 +56,9 @@ struct ActQuantParams {
   uint8_t* lr;           // act + off_lr
   uint32_t* status;      // layer status word
   int32_t MT, KT, KC, RJ, r_tot, rc16, splits;
-  uint32_t stage_bytes, tmem_cols;
+  int32_t push;          // split partials are pushed to the owning CTA (else pulled)
+  int32_t rows_per;      // rows of a row tile each CTA of the cluster reduces
+  uint32_t stage_bytes, tmem_cols, rb_bytes;
   float g_a, c_a, inv_alpha;
   uint64_t timeout_ns;
 };
@@ -130,12 +132,19 @@ __global__ void __launch_bounds__(kThreads1, 2)
   const int nchunks = kc1 - kc0;
   constexpr bool lowrank = kLowRank;
 
-  uint8_t* ctrl = smem + kStages1 * p.stage_bytes;
-  const uint32_t ctrl_s = sbase + kStages1 * p.stage_bytes;
+  // [stages][receive buffer of pushed partials: splits x rows_per x r_tot floats][control]
+  const uint32_t rb_s = sbase + kStages1 * p.stage_bytes;
+  const float* rb = reinterpret_cast<const float*>(smem + kStages1 * p.stage_bytes);
+  uint8_t* ctrl = smem + kStages1 * p.stage_bytes + p.rb_bytes;
+  const uint32_t ctrl_s = sbase + kStages1 * p.stage_bytes + p.rb_bytes;
   const uint32_t FULL = ctrl_s, CONV = ctrl_s + 32u, EMPTY = ctrl_s + 64u;
   const uint32_t ACCF = ctrl_s + 96u, DRAIN = ctrl_s + 104u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 112);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 116);
+  const uint32_t RECV = ctrl_s + 120u;  // the pushed partials of this CTA's rows have landed
+  const int crank = kLowRank && p.splits > 1 ? int(cluster_ctarank()) : 0;
+  const int own0 = crank * p.rows_per;
+  const int own1 = own0 + p.rows_per < kBM ? own0 + p.rows_per : kBM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages1; ++s) {
@@ -145,7 +154,10 @@ __global__ void __launch_bounds__(kThreads1, 2)
     }
     mbar_init(ACCF, 1);
     mbar_init(DRAIN, 1);
+    mbar_init(RECV, 1);
     *abort_flag = 0u;
+    if (lowrank && p.push)  // every CTA of the cluster pushes its partial of these rows
+      mbar_expect_tx(RECV, uint32_t(p.splits * (own1 - own0) * p.r_tot * 4));
     fence_mbar_init();
   }
   if (warp == kMmaWarp1 && lowrank) {
@@ -156,6 +168,8 @@ __global__ void __launch_bounds__(kThreads1, 2)
   __syncthreads();
   if (lowrank) tc_fence_after();
   const uint32_t tmem = lowrank ? *tmem_slot : 0u;
+  // the receive barriers of the whole cluster are armed before anyone pushes
+  if (lowrank && p.push) cluster_arrive();
   // X may be the previous kernel's output and the activation buffer its input
   griddep_wait();
   griddep_launch_dependents();
@@ -262,7 +276,62 @@ __global__ void __launch_bounds__(kThreads1, 2)
   }
 
   // ------------------------------------------------- low-rank output lr'
-  if (lowrank) {
+  if (lowrank && p.push) {
+    // each thread of warps 0-3 holds one row's float partial; it goes to the
+    // CTA of the cluster that reduces that row, which adds the splits in order
+    if (warp < 4) {
+      bool ok = (*abort_flag == 0u) && mbar_wait(ACCF, 0u, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      cluster_wait();
+      if (ok) {
+        tc_fence_after();
+        const uint32_t t = threadIdx.x;
+        const uint32_t owner = t / uint32_t(p.rows_per), lrow = t % uint32_t(p.rows_per);
+        const uint32_t dst = mapa(rb_s + uint32_t(((crank * p.rows_per) + int(lrow)) * p.r_tot) * 4u, owner);
+        const uint32_t bar = mapa(RECV, owner);
+        const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+        for (int c = 0; c < p.r_tot; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(taddr + uint32_t(c), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_async_v4(dst + uint32_t(c + 4 * j) * 4u,
+                        make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                    __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])),
+                        bar);
+        }
+      } else if (*abort_flag == 0u) {
+        fail(0x8u);
+      }
+    }
+    if (warp < 8) {
+      bool ok = mbar_wait(RECV, 0u, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) {
+        if (lane == 0 && *abort_flag == 0u) fail(0x8u);
+      } else {
+        const int groups = p.r_tot / 4;
+        const int nrows = own1 - own0;
+        for (int item = int(threadIdx.x); item < nrows * groups; item += kConvThreads) {
+          const int lr = item / groups, c = (item % groups) * 4;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int q = 0; q < p.splits; ++q) {  // fixed order: deterministic sums
+            const float4 v = *reinterpret_cast<const float4*>(rb + size_t((q * p.rows_per + lr) * p.r_tot + c));
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+          }
+          uint2 w;
+          w.x = f32x2_to_bf16x2(__fmul_rn(acc.x, p.inv_alpha), __fmul_rn(acc.y, p.inv_alpha));
+          w.y = f32x2_to_bf16x2(__fmul_rn(acc.z, p.inv_alpha), __fmul_rn(acc.w, p.inv_alpha));
+          uint8_t* tile = p.lr + (size_t(mt) * p.RJ + size_t(c / kRChunk)) * kATileBytes;
+          *reinterpret_cast<uint2*>(tile + sw128(uint32_t(own0 + lr), uint32_t(c % kRChunk) * 2u)) = w;
+        }
+      }
+    }
+  } else if (lowrank) {
     const bool multi = p.splits > 1;
     float* part = reinterpret_cast<float*>(smem);  // stages are idle now: [128][r_tot + 4]
     const int pstride = p.r_tot + 4;
@@ -406,33 +475,81 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   p.inv_alpha = a.inv_alpha;
   p.timeout_ns = a.timeout_ns;
 
-  const size_t smem = size_t(kStages1) * p.stage_bytes + kCtrlBytes + 1024;
+  const bool lowrank = a.r_tot > 0;
+  auto kernel = lowrank ? act_quant_kernel<true> : act_quant_kernel<false>;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  auto set_smem = [&](auto k, int which, size_t bytes) -> cudaError_t {
+    // the attributes are per device and kernel: remember the largest size set on each
+    static std::atomic<size_t> smem_set[2][64];
+    std::atomic<size_t>& done = smem_set[which][dev & 63];
+    if (bytes <= done.load()) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    if (e == cudaSuccess)  // all of the unified L1 as shared memory: two CTAs per SM must fit
+      e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared));
+    if (e == cudaSuccess) done.store(bytes);
+    return e;
+  };
+  // Split count: enough CTAs to fill the GPU, then (low rank) the largest cluster
+  // size whose clusters of the row tiles are all resident at once.  Occupancy
+  // is asked of the rank-0 instance, which has the same resources but no
+  // tensor-memory allocation (for which the calculator assumes one CTA per SM,
+  // while clusters of this kernel run two per SM).
+  auto plan = [&](int sp, size_t* smem_out, int* push_out, int* rows_out, uint32_t* rb_out) {
+    const int rows = (kBM + sp - 1) / sp;
+    const size_t base = size_t(kStages1) * p.stage_bytes + kCtrlBytes + 1024;
+    const size_t rb = lowrank && sp > 1 ? size_t(round_up(int64_t(sp) * rows * a.r_tot * 4, 1024)) : 0;
+    const bool push = rb > 0 && (base + rb <= 113 * 1024 || (base > 113 * 1024 && base + rb <= 227 * 1024));
+    *push_out = push ? 1 : 0;
+    *rows_out = rows;
+    *rb_out = push ? uint32_t(rb) : 0u;
+    *smem_out = base + (push ? rb : 0);
+  };
+  size_t smem = 0;
+  int push = 0, rows_per = kBM;
+  uint32_t rb_bytes = 0;
+  plan(1, &smem, &push, &rows_per, &rb_bytes);
   const int per_sm = smem <= 113 * 1024 ? 2 : 1;
   int splits = int((int64_t(per_sm) * a.num_sms) / ag.MT);
-  const int max_splits = a.r_tot > 0 ? kMaxSplits : 64;  // the cluster reduction needs a portable cluster
+  const int max_splits = lowrank ? kMaxSplits : 64;  // the cluster reduction needs a portable cluster
   if (splits > max_splits) splits = max_splits;
   if (splits > p.KC) splits = p.KC;
   if (splits < 1) splits = 1;
-  p.splits = splits;
-
-  const bool lowrank = a.r_tot > 0;
-  auto kernel = lowrank ? act_quant_kernel<true> : act_quant_kernel<false>;
-  {
-    // the attributes are per device and kernel: remember the largest size set on each
-    static std::atomic<size_t> smem_set[2][64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    std::atomic<size_t>& done = smem_set[lowrank ? 1 : 0][dev & 63];
-    if (smem > done.load()) {
-      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-      if (e == cudaSuccess)  // all of the unified L1 as shared memory: two CTAs per SM must fit
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 int(cudaSharedmemCarveoutMaxShared));
+  if (lowrank) {
+    for (; splits > 1; --splits) {
+      plan(splits, &smem, &push, &rows_per, &rb_bytes);
+      cudaError_t e = set_smem(act_quant_kernel<false>, 0, smem);
       if (e != cudaSuccess) {
         *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
         return e;
       }
-      done.store(smem);
+      cudaLaunchConfig_t q{};
+      q.gridDim = dim3(unsigned(splits), unsigned(ag.MT), 1);
+      q.blockDim = dim3(kThreads1, 1, 1);
+      q.dynamicSmemBytes = smem;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = unsigned(splits);
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      q.attrs = at;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, act_quant_kernel<false>, &q) == cudaSuccess &&
+          int64_t(clusters) >= ag.MT)
+        break;
+    }
+  }
+  plan(splits, &smem, &push, &rows_per, &rb_bytes);
+  p.splits = splits;
+  p.push = push;
+  p.rows_per = rows_per;
+  p.rb_bytes = rb_bytes;
+  {
+    cudaError_t e = set_smem(kernel, lowrank ? 1 : 0, smem);
+    if (e != cudaSuccess) {
+      *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
+      return e;
     }
   }
   cudaLaunchConfig_t cfg{};
