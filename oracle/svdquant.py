@@ -153,10 +153,16 @@ def low_rank_factors(w_hat_t, rank):
 
 
 def residual(w_hat_t, l1, l2):
-    """R = W_hat^T - L1 L2, rank-one terms subtracted in order j = 0 .. r-1."""
+    """R = W_hat^T - L1 L2, rank-one terms subtracted in order j = 0 .. r-1.
+
+    (Done in blocks of rows so that no full-size temporary is made; every
+    element sees the same subtractions in the same order.)
+    """
     r = np.array(w_hat_t, dtype=np.float64, copy=True)
-    for j in range(l1.shape[1]):
-        r -= np.outer(l1[:, j], l2[j, :])
+    for k0 in range(0, r.shape[0], 512):
+        blk = r[k0:k0 + 512]
+        for j in range(l1.shape[1]):
+            blk -= np.outer(l1[k0:k0 + 512, j], l2[j, :])
     return r
 
 
@@ -219,13 +225,21 @@ def act_global_scale(act_amax, inv_lam):
     return global_scale(np.max(xh) if xh.size else 0.0)
 
 
-def prepare(W, act_amax, rank, bias=None, factors=None):
+def prepare(W, act_amax, rank, bias=None, factors=None, out_rows=None):
     """Offline preparation of one layer.
 
     W: [N, K] bfloat16 values (any float dtype holding them).
     act_amax: float32 [K], max|X_:,j| over calibration rows.
     factors: optional (L1 [K, r], L2 [r, N]) bfloat16 values to use instead of
              this module's SVD (the weights of a checkpoint, say).
+    out_rows: optional subset of the N output features to keep (for shapes too
+             large to prepare whole here).  lambda comes from the whole weight
+             and R's kept columns from the rank-one order above; g_w =
+             max|R| / 2688 takes the maximum of W_hat^T - L1 L2 evaluated
+             with one matrix product (it can differ from the rank-one order
+             only in the last bits, and enters a test only through Y, which
+             is compared within its tolerance).  Only the kept rows of R^T are
+             quantized, and L2, the bias and N are restricted to them.
     """
     W = np.asarray(W, dtype=np.float64)
     n, k = W.shape
@@ -243,13 +257,19 @@ def prepare(W, act_amax, rank, bias=None, factors=None):
         l1b = np.asarray(factors[0], dtype=np.float64)
         l2b = np.asarray(factors[1], dtype=np.float64)
         assert l1b.shape == (k, rank) and l2b.shape == (rank, n)
-    r = residual(w_hat_t, l1b, l2b)
-    r32 = r.astype(np.float32)
-    g_w = global_scale(np.max(np.abs(r32)) if r32.size else 0.0)
-    w_codes, w_scales = nvfp4_quantize(np.ascontiguousarray(r32.T), g_w)
+    cols = np.arange(n) if out_rows is None else np.asarray(out_rows)
+    if out_rows is None:
+        r = residual(w_hat_t, l1b, l2b)
+        amax_r = np.max(np.abs(r)) if r.size else 0.0
+    else:
+        r = residual(w_hat_t[:, cols], l1b, l2b[:, cols])
+        amax_r = np.max(np.abs(w_hat_t - l1b @ l2b)) if w_hat_t.size else 0.0
+    del w_hat_t
+    g_w = global_scale(np.float32(amax_r))  # max commutes with the (monotone) f32 rounding
+    w_codes, w_scales = nvfp4_quantize(np.ascontiguousarray(r.T.astype(np.float32)), g_w)
     g_a = act_global_scale(act_amax, inv_lam)
-    b = None if bias is None else np.asarray(bias, dtype=np.float64)
-    return Layer(k, n, rank, lam, inv_lam, l1b, l2b, r, w_codes, w_scales, g_w, g_a, b, sigma)
+    b = None if bias is None else np.asarray(bias, dtype=np.float64)[cols]
+    return Layer(k, len(cols), rank, lam, inv_lam, l1b, l2b[:, cols], r, w_codes, w_scales, g_w, g_a, b, sigma)
 
 
 def attach_lora(layer, A, B, scale=1.0):

@@ -214,3 +214,43 @@ def test_clone_on_another_buffer_gives_identical_output():
     torch.cuda.synchronize()
     assert torch.equal(Y0.view(torch.int16), Y1.view(torch.int16))
     twin.poll_status()
+
+
+def test_largest_sweep_point_on_sampled_outputs():
+    """M = 16384 tokens, K = N = 12288, rank 64: the largest sweep point, run whole on
+    the GPU and checked on 128 sampled rows x 64 sampled output features.
+
+    The low-rank factors are seeded N(0, 0.05) bf16 values given to both sides
+    (a LAPACK SVD of this size does not fit the test's time); the oracle
+    prepares only the sampled output features (lambda and g_w still come from
+    the whole weight).  Codes and scales of the sampled rows are compared bit
+    for bit, Y within the layer tolerance."""
+    from oracle import formats as F
+    from gpu_cases import LR_TOL, Y_TOL
+
+    spec = WL.sweep_spec(16384, 12288, 64)
+    X, W = spec.x(), spec.w()
+    X32 = X.astype(np.float32)
+    amax = np.max(np.abs(X32), axis=0)
+    g = np.random.default_rng([spec.seed, WL.STREAM_SAMPLE, 2])
+    l1 = S.bf16_from_f64(g.normal(0.0, 0.05, (spec.K, spec.rank)))
+    l2 = S.bf16_from_f64(g.normal(0.0, 0.05, (spec.rank, spec.N)))
+    cols = np.sort(np.concatenate([[0, spec.N - 1], g.choice(spec.N, size=62, replace=False)]))
+    rows = _rows(spec.M, n=126, seed=6)
+    ref = S.prepare(W.astype(np.float32), amax, spec.rank, factors=(l1, l2), out_rows=cols)
+    layer = svdq.Layer(W, amax, spec.rank, factors=(F.bf16_bits(l1.astype(np.float32)),
+                                                     F.bf16_bits(l2.astype(np.float32))), device="cuda")
+    Xd = torch.from_numpy(X.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    act = layer.quantize_act(Xd)
+    Y = layer.linear(act, spec.M)
+    torch.cuda.synchronize()
+    layer.poll_status()
+    codes, scales, lr = layer.act_unpack(act.cpu().numpy(), spec.M)
+    ref_act = S.quantize_act(ref, X32[rows])
+    np.testing.assert_array_equal(codes[rows], F.pack_e2m1(ref_act.codes))
+    np.testing.assert_array_equal(scales[rows], ref_act.scales)
+    lr_gpu = F.bf16_from_bits(lr[rows]).astype(np.float64) * ref.alpha
+    assert np.max(np.abs(lr_gpu - ref_act.lr)) <= LR_TOL * np.max(np.abs(ref_act.lr))
+    y = Y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
+    err = S.max_rel_err(y, S.linear(ref, ref_act))
+    assert err <= Y_TOL, err

@@ -317,3 +317,22 @@ def test_planted_mistake_is_caught(monkeypatch, name, target, mutant):
     monkeypatch.setattr(S, target, mutant)
     with pytest.raises(AssertionError):
         check_layer_against_bruteforce(3, 32, 5, 2, seed=35, bias=True, gelu=False)
+
+
+def test_prepare_on_sampled_outputs_matches_the_whole_layer():
+    """The restriction to some output features gives exactly those features of the whole layer."""
+    g = np.random.default_rng([11, 1])
+    K, N, r = 128, 96, 16
+    W = F.bf16(g.normal(0, 0.02, (N, K)).astype(np.float32)).astype(np.float64)
+    X = F.bf16(g.normal(0, 1, (8, K)).astype(np.float32))
+    amax = np.max(np.abs(X.astype(np.float32)), 0)
+    b = F.bf16(g.normal(0, 0.01, N).astype(np.float32)).astype(np.float64)
+    whole = S.prepare(W, amax, r, bias=b)
+    cols = np.array([0, 5, 17, 64, 95])
+    part = S.prepare(W, amax, r, bias=b, factors=(whole.L1, whole.L2), out_rows=cols)
+    assert part.N == len(cols) and part.g_w == whole.g_w
+    np.testing.assert_array_equal(part.w_codes, whole.w_codes[cols])
+    np.testing.assert_array_equal(part.w_scales, whole.w_scales[cols])
+    np.testing.assert_array_equal(part.L2, whole.L2[:, cols])
+    y_whole = S.forward(whole, X)
+    np.testing.assert_array_equal(S.forward(part, X), y_whole[:, cols])
