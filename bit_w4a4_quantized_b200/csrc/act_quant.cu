@@ -43,7 +43,8 @@ constexpr int kStages1 = 4;
 constexpr int kThreads1 = 320;  // warps 0-7 convert, 8 produce, 9 issue MMAs
 constexpr int kConvThreads = 256;
 constexpr int kProducerWarp1 = 8, kMmaWarp1 = 9;
-constexpr int kMaxSplits = 8;
+constexpr int kMaxSplits = 8;       // pulled partials: a portable cluster
+constexpr int kMaxPushSplits = 16;  // pushed partials: up to the non-portable cluster size
 constexpr uint32_t kXBytes = kBM * 128;  // 16 KB: 128 rows x 64 bf16
 constexpr uint32_t kInvSlot = 1024;      // 64 floats of 1/lambda (256 B), padded for alignment
 constexpr uint32_t kCtrlBytes = 128;
@@ -511,13 +512,24 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   plan(1, &smem, &push, &rows_per, &rb_bytes);
   const int per_sm = smem <= 113 * 1024 ? 2 : 1;
   int splits = int((int64_t(per_sm) * a.num_sms) / ag.MT);
-  const int max_splits = lowrank ? kMaxSplits : 64;  // the cluster reduction needs a portable cluster
+  const int max_splits = lowrank ? kMaxPushSplits : 64;
   if (splits > max_splits) splits = max_splits;
   if (splits > p.KC) splits = p.KC;
   if (splits < 1) splits = 1;
   if (lowrank) {
+    static std::atomic<int> nonportable[64];
+    if (nonportable[dev & 63].load() == 0) {
+      // clusters of up to 16 CTAs for the pushed partials (small M, long K)
+      cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(act_quant_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      nonportable[dev & 63].store(e == cudaSuccess ? 1 : -1);
+    }
+    const int cap = nonportable[dev & 63].load() > 0 ? kMaxPushSplits : kMaxSplits;
+    if (splits > cap) splits = cap;
     for (; splits > 1; --splits) {
       plan(splits, &smem, &push, &rows_per, &rb_bytes);
+      if (!push && splits > kMaxSplits) continue;  // pulled partials: at most a portable cluster
       cudaError_t e = set_smem(act_quant_kernel<false>, 0, smem);
       if (e != cudaSuccess) {
         *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
