@@ -108,6 +108,19 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   return 0.5f * x * (1.0f + tanh_approx(u));
 }
 
+// Tile t -> (row-tile pair mp, weight tile nt).  Tiles run in groups of
+// kGroupMP row-tile pairs swept across all weight tiles, so the tiles in flight
+// at any time touch at most kGroupMP pairs' activations and a few weight tiles:
+// both stay in L2 even when the whole operands do not.
+constexpr int kGroupMP = 8;
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& mp, int& nt) {
+  const int per_group = kGroupMP * p.NT;
+  const int grp = tile / per_group, in = tile % per_group;
+  const int gsize = (p.MP - grp * kGroupMP) < kGroupMP ? (p.MP - grp * kGroupMP) : kGroupMP;
+  mp = grp * kGroupMP + in % gsize;
+  nt = in / gsize;
+}
+
 // 32 accumulator columns of one row -> alpha, bias, act -> 16 words of bf16 pairs.
 // `bias` points at the 32 bias values of these columns in shared memory (or null).
 __device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t* v, const float* bias, uint32_t* out) {
@@ -187,7 +200,9 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       uint32_t it = 0;
       bool stop = false;
       for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
-        const int mt = 2 * (tile % p.MP) + int(rank), nt = tile / p.MP;
+        int mp, nt;
+        tile_coords(p, tile, mp, nt);
+        const int mt = 2 * mp + int(rank);
         for (int kt = 0; kt < p.KT; ++kt) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
@@ -345,7 +360,9 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colq * 64);
     for (int tile = pair; tile < ntiles; tile += npairs) {
-      const int mt = 2 * (tile % p.MP) + int(rank), nt = tile / p.MP;
+      int mp, nt;
+      tile_coords(p, tile, mp, nt);
+      const int mt = 2 * mp + int(rank);
       // stage this warp's 64 bias values (warp-private, double buffered)
       float* bias_w = bias_s + (size_t(warp) * 2 + (tc & 1u)) * 64;
       if (p.bias) {
