@@ -23,6 +23,15 @@
  *   - Streams are cudaStream_t values passed as void*; NULL is the legacy
  *     default stream.  Launching entry points are asynchronous and stream
  *     ordered unless stated otherwise.
+ *   - svdq_quantize_act and svdq_w4a4_linear launch with programmatic
+ *     dependent launch: their prologue may overlap the previous kernel in the
+ *     stream, but they touch no global memory before that kernel has completed
+ *     (griddepcontrol.wait), so ordinary stream order holds for the caller.
+ *     They also let the next kernel in the stream start early; only a kernel
+ *     that was itself launched with programmatic stream serialization can, and
+ *     it must wait in the same way before reading their outputs.
+ *   - One activation buffer serves one call at a time: two launches that use
+ *     the same buffer must be ordered (same stream or events).
  *   - bf16 arrays are passed as raw 16-bit patterns (uint16_t / void*).
  *   - Inputs must be finite; NaN/Inf inputs give unspecified (but memory-safe)
  *     results.
