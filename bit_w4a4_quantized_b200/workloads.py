@@ -30,6 +30,8 @@ STREAM_LORA_B = 6
 STREAM_W2 = 7
 STREAM_W2_OUTLIER = 8
 STREAM_SAMPLE = 9
+STREAM_NORM_Q = 10
+STREAM_NORM_K = 11
 
 
 def rng(seed, stream):
@@ -75,6 +77,23 @@ def make_lora(K, N, r_e, seed, std=0.01):
     a = rng(seed, STREAM_LORA_A).standard_normal((K, r_e), dtype=np.float32) * np.float32(std)
     b = rng(seed, STREAM_LORA_B).standard_normal((r_e, N), dtype=np.float32) * np.float32(std)
     return to_bf16(a), to_bf16(b)
+
+
+def make_norm_weights(head_dim, seed, std=0.1):
+    """RMSNorm weights of Q and K: bf16 [head_dim] each, 1 + N(0, std)."""
+    q = 1.0 + rng(seed, STREAM_NORM_Q).standard_normal(head_dim) * std
+    k = 1.0 + rng(seed, STREAM_NORM_K).standard_normal(head_dim) * std
+    return to_bf16(q), to_bf16(k)
+
+
+def make_rope(M, head_dim, base=10000.0):
+    """Rotary angle table float32 [M, head_dim / 2, 2] = (cos, sin) of
+    m * base^(-2 i / head_dim) for token m and pair i: one position per row,
+    the usual frequency ladder.  A fixed table, no random draws."""
+    m = np.arange(M, dtype=np.float64)[:, None]
+    freq = base ** (-2.0 * np.arange(head_dim // 2, dtype=np.float64) / head_dim)
+    ang = m * freq[None, :]
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32)
 
 
 @dataclass(frozen=True)

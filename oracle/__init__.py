@@ -17,7 +17,9 @@ Sources (the SVDQuant summary page, hoonably.github.io/blog/svdquant):
     the quantizer, the up projection is added into the 4-bit GEMM output.
 The abstract record of arXiv 2411.05007 adds: LoRA adapters attach to the
 low-rank branch without re-quantizing R.  The Diffusers/Nunchaku page adds:
-NVFP4 (Blackwell), compute dtype bfloat16, QKV fusion along the output dim.
+NVFP4 (Blackwell), compute dtype bfloat16, QKV fusion along the output dim,
+and (fused-QKV section) one fused operator for the QKV projection, the Q/K
+normalization and the rotary embedding: ``qkv`` restates that operator.
 
 Every reading the pages leave open (NVFP4 two-level scales, rounding, sign of
 zero, static activation scale, ...) is stated in the

@@ -135,3 +135,24 @@ def layer_forward(W, X, act_amax, L1, L2, bias=None, gelu=False):
         Y.append(row)
     return dict(lam=lam, inv=inv, g_w=g_w, g_a=g_a, w_codes=wc, w_scales=ws, a_codes=ac,
                 a_scales=as_, x_hat=xh, lr=lr, Y=Y)
+
+
+def qkv_norm_rope(Y, norm_q, norm_k, rope, eps, head_dim):
+    """Q/K head RMSNorm then pair rotation, V untouched, with plain loops.
+
+    Y: list of rows of 3 C values; rope[m][i] = (cos, sin) for pair i.
+    """
+    out = [list(row) for row in Y]
+    C = len(Y[0]) // 3
+    for m, row in enumerate(Y):
+        for part, w in ((0, norm_q), (1, norm_k)):
+            for h0 in range(part * C, (part + 1) * C, head_dim):
+                head = row[h0:h0 + head_dim]
+                ms = math.fsum(v * v for v in head) / head_dim
+                inv = 1.0 / math.sqrt(ms + eps)
+                z = [head[d] * inv * w[d] for d in range(head_dim)]
+                for i in range(head_dim // 2):
+                    c, s = rope[m][i]
+                    out[m][h0 + 2 * i] = z[2 * i] * c - z[2 * i + 1] * s
+                    out[m][h0 + 2 * i + 1] = z[2 * i + 1] * c + z[2 * i] * s
+    return out
