@@ -56,6 +56,11 @@ def workload_spec(name):
     raise SystemExit(f"unknown workload {name}")
 
 
+def qkv_shape(N, head_dim=128):
+    """True when N splits into Q | K | V of whole heads (the fused QKV epilogue applies)."""
+    return N % 3 == 0 and (N // 3) % head_dim == 0
+
+
 def layer_flops(spec, r_tot):
     """(FP4 GEMM flops, bf16 low-rank flops) of one forward of the layer."""
     fp4 = 2 * spec.M * spec.N * spec.K
@@ -560,6 +565,20 @@ def sweep_point(spec, device, steps, factors_cache):
                       stream)
         t1 = _graph_seconds(k1, nsets, steps, stream, device)
         t2 = _graph_seconds(k2, nsets, steps, stream, device)
+        if tag != "plain" and spec.name.startswith("qkv") and qkv_shape(N):
+            # the fused QKV epilogue (per-head Q/K RMSNorm + rotary turn) on the same layers
+            nq, nk = (to_dev(w) for w in WL.make_norm_weights(128, spec.seed))
+            rope = torch.from_numpy(WL.make_rope(M, 128)).to(device)
+            packed = svdq.rope_pack(rope, stream=stream)
+            k3 = _capture([lambda i=i: layers[i].linear_qkv_norm_rope(acts[i], M, nq, nk, packed, out=Ys[i])
+                           for i in range(nsets)], stream)
+            t3 = _graph_seconds(k3, nsets, steps, stream, device)
+            kp = _capture([lambda: svdq.rope_pack(rope, out=packed)], stream)
+            tp = _graph_seconds(kp, 1, steps, stream, device)
+            out["qkv_norm_rope_gemm_us"] = round(t3 * 1e6, 3)
+            out["qkv_norm_rope_overhead_gemm"] = round(t3 / t2 - 1, 4)
+            out["rope_pack_us"] = round(tp * 1e6, 3)
+            del k3, kp
         for L in layers:
             L.poll_status()
         out[f"{tag}_act_us"] = round(t1 * 1e6, 3)

@@ -176,8 +176,10 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   return SVDQ_OK;
 }
 
-svdq_status svdq_w4a4_linear(const svdq_layer* L, const void* act_buf, size_t act_buf_bytes, int64_t M, void* Y,
-                             int epilogue, void* stream) {
+namespace {
+
+svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_buf_bytes, int64_t M, void* Y,
+                          int epilogue, const svdq::GemmLaunch* qkv, void* stream) {
   svdq_status st = check_uploaded(L);
   if (st != SVDQ_OK) return st;
   if (!act_buf || !Y) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf and Y are required");
@@ -191,7 +193,7 @@ svdq_status svdq_w4a4_linear(const svdq_layer* L, const void* act_buf, size_t ac
   if (M * L->g.N > (int64_t(1) << 31) * 2 || M > (int64_t(1) << 31) - 1)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M too large");
   if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
-  svdq::GemmLaunch a{};
+  svdq::GemmLaunch a = qkv ? *qkv : svdq::GemmLaunch{};
   a.act = static_cast<const uint8_t*>(act_buf);
   a.layer = static_cast<const uint8_t*>(L->dev_buf);
   a.Y = Y;
@@ -207,6 +209,64 @@ svdq_status svdq_w4a4_linear(const svdq_layer* L, const void* act_buf, size_t ac
   cudaError_t e = svdq::launch_gemm(a, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
   return SVDQ_OK;
+}
+
+}  // namespace
+
+svdq_status svdq_w4a4_linear(const svdq_layer* L, const void* act_buf, size_t act_buf_bytes, int64_t M, void* Y,
+                             int epilogue, void* stream) {
+  return linear_launch(L, act_buf, act_buf_bytes, M, Y, epilogue, nullptr, stream);
+}
+
+svdq_status svdq_rope_packed_bytes(int64_t M, int32_t head_dim, size_t* bytes) {
+  if (!bytes) return fail(SVDQ_ERR_INVALID_ARGUMENT, "bytes is required");
+  if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
+  if (head_dim != svdq::kRopeHeadDim) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
+  *bytes = svdq::rope_packed_bytes(M);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_rope_pack(const void* rope, int64_t M, int32_t head_dim, void* packed, size_t packed_bytes,
+                           void* stream) {
+  size_t need = 0;
+  svdq_status st = svdq_rope_packed_bytes(M, head_dim, &need);
+  if (st != SVDQ_OK) return st;
+  if (!rope || !packed) return fail(SVDQ_ERR_INVALID_ARGUMENT, "rope and packed are required");
+  if (!aligned(rope, 16) || !aligned(packed, 16))
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "rope and packed must be 16-byte aligned");
+  if (packed_bytes < need)
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "packed needs " + std::to_string(need) + " bytes");
+  if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
+  cudaError_t e = svdq::launch_rope_pack(static_cast<const float*>(rope), M, static_cast<float*>(packed),
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "launch of the rotary table pack kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_w4a4_linear_qkv_norm_rope(const svdq_layer* L, const void* act_buf, size_t act_buf_bytes,
+                                           int64_t M, void* Y, const void* norm_q, const void* norm_k,
+                                           const void* rope_packed, size_t rope_packed_bytes, int32_t head_dim,
+                                           float eps, void* stream) {
+  svdq_status st = check_uploaded(L);
+  if (st != SVDQ_OK) return st;
+  if (head_dim != svdq::kRopeHeadDim) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
+  if (L->g.N % 3 || (L->g.N / 3) % head_dim)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N must be 3 x a multiple of head_dim (Q | K | V)");
+  if (!norm_q || !norm_k || !rope_packed)
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "norm_q, norm_k and rope_packed are required");
+  if (!aligned(norm_q, 16) || !aligned(norm_k, 16) || !aligned(rope_packed, 16))
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "norm_q, norm_k and rope_packed must be 16-byte aligned");
+  if (M >= 1 && rope_packed_bytes < svdq::rope_packed_bytes(M))
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL,
+                "rope_packed needs " + std::to_string(svdq::rope_packed_bytes(M)) + " bytes (svdq_rope_pack)");
+  if (!std::isfinite(eps) || eps < 0.0f) return fail(SVDQ_ERR_INVALID_ARGUMENT, "eps must be finite and >= 0");
+  svdq::GemmLaunch q{};
+  q.qkv_cols = int32_t(L->g.N / 3);
+  q.norm_q = static_cast<const uint16_t*>(norm_q);
+  q.norm_k = static_cast<const uint16_t*>(norm_k);
+  q.rope = static_cast<const float*>(rope_packed);
+  q.eps = eps;
+  return linear_launch(L, act_buf, act_buf_bytes, M, Y, SVDQ_EPI_NONE, &q, stream);
 }
 
 svdq_status svdq_lora_swap(svdq_layer* L, const void* A, const void* B, int32_t r_e, float scale, void* stream) {

@@ -18,24 +18,31 @@
 //     memory.  Sharing B across the pair cuts the operand bytes every SM
 //     streams per FLOP by 30 % against a 128 x 256 one-SM tile; the freed
 //     shared memory buys a fifth pipeline stage.
-//   * warp 8 of each CTA fills a 5-stage ring with tensor loads (one per
+//   * warp 20 of each CTA fills a 5-stage ring with tensor loads (one per
 //     operand, 2 KB rows) of the pre-tiled, pre-swizzled operands: A 16 KB and
 //     the B half 16 KB counted on the leader CTA's full barrier (armed by the
 //     leader with both CTAs' bytes), A scales 2 KB and all 256 rows of B scales
 //     4 KB counted on the CTA's own scale barrier.  After the K loop of a tile
 //     the same ring carries the lr' and L2^T chunks.
-//   * warps 10-13 of each CTA (one per tensor-memory lane quarter) move each
+//   * warps 16-19 of each CTA (one per tensor-memory lane quarter) move each
 //     stage's block scales from shared memory into their CTA's tensor memory
 //     with tcgen05.st, in the replicated layout the block-scaled MMA reads,
 //     then arrive on the leader's full barrier.  Scale staging therefore
 //     never occupies the tensor pipe, which issues nothing but MMAs.
-//   * warp 9 of the leader issues 4 block-scaled MMAs per 256-wide k-tile,
+//   * warp 21 of the leader issues 4 block-scaled MMAs per 256-wide k-tile,
 //     then the bf16 MMAs of the fold, and commits every stage back to both
 //     CTAs' empty barriers with a multicast commit.
-//   * warps 0-7 of each CTA: epilogue, one output row x 128 columns per
-//     thread: tensor memory -> registers, release the accumulator to the
-//     leader, then alpha, bias, GELU -> bf16 -> global while the next tile's K
-//     loop runs.
+//   * warps 0-15 of each CTA: epilogue, one output row x 64 columns per
+//     thread (warp w: lane quarter w % 4, columns 64 (w / 4) .. +63): tensor
+//     memory -> registers, release the accumulator to the leader, then alpha,
+//     bias, GELU -> bf16 -> global while the next tile's K loop runs.
+//   * The QKV instance (kQkv) finishes a fused Q|K|V projection instead
+//     (Diffusers/Nunchaku page, fused-QKV section: projection, Q/K norm and
+//     rotary embedding in one operator): each row's bf16 outputs of a Q or K
+//     head of 128 columns are RMS-normalized over the head (the two warps
+//     holding its halves swap their sums of squares through shared memory
+//     under an mbarrier), scaled by norm_q / norm_k, turned pair by pair by
+//     the row's rotary angles, and rounded to bf16 once more.  V passes.
 //   * Tensor memory (per CTA): accumulator columns [0, 256), scale factors of
 //     stage s at 256 + 16 s (A) and 336 + 32 s (B).
 //   * Every wait is bounded (status word + clean exit on timeout); the pair
@@ -69,6 +76,8 @@ constexpr uint32_t kStage2 = kOffSFB + kSFBTileBytes;    // 38912 bytes
 constexpr uint32_t kFoldBytes = 2 * kHalf * kRowBytes;   // lr' 16 KB + L2^T half 16 KB
 constexpr uint32_t kCtrl2 = 256;
 constexpr uint32_t kBiasBytes = kEpiWarps * 2 * 64 * 4;  // per epilogue warp: 2 tiles x 64 floats
+constexpr uint32_t kXchBytes = 8 * 2 * 64 * 4;  // QKV: [head warp pair][parity][2 halves x 32 rows] floats
+constexpr uint32_t kNormBytes = kEpiWarps * 64 * 4;  // QKV: per epilogue warp, its 64 norm_q and 64 norm_k weights
 constexpr uint32_t kTmemCols2 = 512;
 constexpr uint32_t kColSFA = 256, kColSFB = kColSFA + 16 * kStages2;
 constexpr uint16_t kPairMask = 0x3;
@@ -100,6 +109,12 @@ struct GemmParams {
   int32_t M, N, MP, NT, KT, RJ, r_tot, epilogue;
   float alpha;
   uint64_t timeout_ns;
+  // QKV instance only
+  const uint16_t* norm_q;  // bf16 [128]
+  const uint16_t* norm_k;  // bf16 [128]
+  const float* rope;       // packed rotary table: [row tile][32 chunks][128 rows] x 16 bytes
+  float eps;
+  int32_t qkv_cols;  // N / 3
 };
 
 __device__ __forceinline__ float gelu_tanh(float x) {
@@ -123,13 +138,14 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
 
 // 32 accumulator columns of one row -> alpha, bias, act -> 16 words of bf16 pairs.
 // `bias` points at the 32 bias values of these columns in shared memory (or null).
+template <bool kMayGelu = true>
 __device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t* v, const float* bias, uint32_t* out) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const float b0 = bias ? bias[2 * e] : 0.0f, b1 = bias ? bias[2 * e + 1] : 0.0f;
     float y0 = fmaf(p.alpha, __uint_as_float(v[2 * e]), b0);
     float y1 = fmaf(p.alpha, __uint_as_float(v[2 * e + 1]), b1);
-    if (p.epilogue == SVDQ_EPI_GELU_TANH) {
+    if (kMayGelu && p.epilogue == SVDQ_EPI_GELU_TANH) {
       y0 = gelu_tanh(y0);
       y1 = gelu_tanh(y1);
     }
@@ -137,6 +153,38 @@ __device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t
   }
 }
 
+// kRopeBatch chunks (2 pairs each) of one Q or K head row: the bf16 values in
+// out[2 kRopeBatch] are RMS-normalized with `inv`, scaled by the weights (bf16
+// pairs in wsm) and turned by the (cos, sin, cos, sin) chunks in t.
+#ifndef SVDQ_ROPE_BATCH
+#define SVDQ_ROPE_BATCH 4
+#endif
+constexpr int kRopeBatch = SVDQ_ROPE_BATCH;
+__device__ __forceinline__ void norm_rope_chunks(uint32_t* out, float inv, const uint32_t* wsm, const float4* t) {
+#pragma unroll
+  for (int e2 = 0; e2 < kRopeBatch; ++e2) {
+    const uint2 w = *reinterpret_cast<const uint2*>(wsm + 2 * e2);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t y = out[2 * e2 + j], ww = j ? w.y : w.x;
+      const float c = j ? t[e2].z : t[e2].x, sn = j ? t[e2].w : t[e2].y;
+      const float z0 = bf16lo(y) * inv * bf16lo(ww);
+      const float z1 = bf16hi(y) * inv * bf16hi(ww);
+      out[2 * e2 + j] = f32x2_to_bf16x2(z0 * c - z1 * sn, z1 * c + z0 * sn);
+    }
+  }
+}
+
+__global__ void rope_pack_kernel(const float4* rope, int64_t M, float4* packed, int64_t total) {
+  for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t i = idx % kBM, c = (idx / kBM) % kRopeChunks, t = idx / (int64_t(kBM) * kRopeChunks);
+    const int64_t row = t * kBM + i;
+    packed[idx] = row < M ? rope[row * kRopeChunks + c] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+template <bool kQkv>
 __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -157,6 +205,9 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 108);
   const uint32_t SFULL = ctrl_s + 112u;  // 5 barriers: this CTA's scales of a stage have landed
   float* bias_s = reinterpret_cast<float*>(ctrl + kCtrl2);  // [warp][tile parity][64] floats
+  const uint32_t XCH = ctrl_s + 152u;  // QKV: 8 barriers, one per warp pair sharing a head
+  float* xch = reinterpret_cast<float*>(ctrl + kCtrl2 + kBiasBytes);
+  uint32_t* norm_s = reinterpret_cast<uint32_t*>(ctrl + kCtrl2 + kBiasBytes + kXchBytes);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
@@ -167,6 +218,8 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     mbar_init(ACCF, 1);   // both: one multicast commit per tile
     mbar_init(ACCE, 2 * kEpiWarps);  // leader: one arrival per epilogue warp of both CTAs
     mbar_init(DRAIN, 1);
+    if (kQkv)
+      for (int h = 0; h < 8; ++h) mbar_init(XCH + 8u * h, 64);  // every thread of both warps
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -355,8 +408,15 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     // 64 (w / 4) .. +63: its share of the tile goes to registers, the
     // accumulator is released to the leader, then the rows are finished and
     // stored while the next tile's K loop runs.
-    uint32_t tc = 0;
+    uint32_t tc = 0, xc = 0;
     const int quarter = warp & 3, colq = warp >> 2;
+    uint32_t* norm_w = norm_s + warp * 64;  // QKV: [Q, K][32 bf16 pairs] of this warp's columns
+    if (kQkv) {
+      const int half = colq & 1;
+      norm_w[lane] = *reinterpret_cast<const uint32_t*>(p.norm_q + half * 64 + 2 * lane);
+      norm_w[32 + lane] = *reinterpret_cast<const uint32_t*>(p.norm_k + half * 64 + 2 * lane);
+      __syncwarp();
+    }
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colq * 64);
     for (int tile = pair; tile < ntiles; tile += npairs) {
@@ -385,7 +445,62 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
       const int64_t row = int64_t(mt) * kBM + row_in_tile;
-      if (row < p.M) {
+      if constexpr (kQkv) {
+        // the two warps of a head (colq 2h, 2h + 1) agree on every branch
+        // below: the head's columns are all below N or all above (N % 128 == 0)
+        const int n0 = nt * kBN + colq * 64;
+        if (n0 < p.N) {
+          uint32_t out[32];
+          finish_chunk<false>(p, v, p.bias ? bias_w : nullptr, out);
+          finish_chunk<false>(p, v + 32, p.bias ? bias_w + 32 : nullptr, out + 16);
+          const int part = n0 / p.qkv_cols;  // 0 Q, 1 K, 2 V
+          if (part < 2) {
+            float ss = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              uint32_t o = out[e];
+              asm volatile("" : "+r"(o));  // keep the packed words, not their unpacked floats, across the wait
+              const float y0 = bf16lo(o), y1 = bf16hi(o);
+              ss = fmaf(y0, y0, ss);
+              ss = fmaf(y1, y1, ss);
+            }
+            const int hp = quarter + 4 * (colq >> 1), half = colq & 1;
+            // this row's (cos, sin) chunks: coalesced across the warp's rows;
+            // the first batch is in flight while the two warps meet
+            const float4* cs = reinterpret_cast<const float4*>(p.rope) +
+                               (size_t(mt) * kRopeChunks + size_t(half) * 16) * kBM + size_t(row_in_tile);
+            float4 t[kRopeBatch];
+#pragma unroll
+            for (int j = 0; j < kRopeBatch; ++j) t[j] = __ldg(cs + j * kBM);
+            float* xb = xch + (hp * 2 + int(xc & 1u)) * 64;
+            xb[half * 32 + lane] = ss;
+            mbar_arrive(XCH + 8u * hp);
+            bool okx = mbar_wait(XCH + 8u * hp, xc & 1u, abort_flag, p.timeout_ns);
+            okx = __all_sync(0xFFFFFFFFu, okx);
+            if (!okx) {
+              if (*abort_flag == 0u) fail(0x80u);
+              break;
+            }
+            ++xc;
+            const float tot = xb[lane] + xb[32 + lane];  // the same order in both warps
+            const float inv = rsqrtf(fmaf(tot, 1.0f / 128.0f, p.eps));
+            const uint32_t* wsm = norm_w + part * 32;
+#pragma unroll
+            for (int b = 0; b < 16 / kRopeBatch; ++b) {
+              if (b) {
+#pragma unroll
+                for (int j = 0; j < kRopeBatch; ++j) t[j] = __ldg(cs + (b * kRopeBatch + j) * kBM);
+              }
+              norm_rope_chunks(out + 2 * kRopeBatch * b, inv, wsm + 2 * kRopeBatch * b, t);
+            }
+          }
+          if (row < p.M) {
+            uint16_t* dst = p.Y + row * p.N + n0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) st_global_v8(dst + 16 * j, out + 8 * j);
+          }
+        }
+      } else if (row < p.M) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int n0 = nt * kBN + colq * 64 + q * 32;
@@ -474,20 +589,28 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   p.epilogue = a.epilogue;
   p.alpha = a.alpha;
   p.timeout_ns = a.timeout_ns;
+  const bool qkv = a.qkv_cols > 0;
+  p.norm_q = a.norm_q;
+  p.norm_k = a.norm_k;
+  p.rope = a.rope;
+  p.eps = a.eps;
+  p.qkv_cols = a.qkv_cols;
+  auto kernel = qkv ? gemm_kernel<true> : gemm_kernel<false>;
 
   const int64_t ntiles = int64_t(p.MP) * lg.NT;
   if (ntiles > (int64_t(1) << 30)) {
     *why = "problem too large for one launch";
     return cudaErrorInvalidValue;
   }
-  const size_t smem = size_t(kStages2) * kStage2 + kCtrl2 + kBiasBytes + 1024;
-  static std::atomic<int> max_pairs[64];
+  const size_t smem = size_t(kStages2) * kStage2 + kCtrl2 + kBiasBytes + (qkv ? kXchBytes + kNormBytes : 0) + 1024;
+  static std::atomic<int> max_pairs_of[2][64];
   int dev = 0;
   cudaGetDevice(&dev);
+  std::atomic<int>* max_pairs = max_pairs_of[qkv ? 1 : 0];
   if (max_pairs[dev & 63].load() == 0) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+      e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                int(cudaSharedmemCarveoutMaxShared));
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
@@ -505,7 +628,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
     q.attrs = at;
     q.numAttrs = 1;
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel, &q);
+    e = cudaOccupancyMaxActiveClusters(&clusters, kernel, &q);
     if (e != cudaSuccess || clusters < 1) {
       *why = "no CTA pair of the GEMM fits on this device";
       return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
@@ -528,9 +651,18 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel, maps, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, maps, p);
   if (e != cudaSuccess) *why = "launch of the GEMM kernel failed";
   return e;
+}
+
+cudaError_t launch_rope_pack(const float* rope, int64_t M, float* packed, cudaStream_t s) {
+  const int64_t total = int64_t(rope_packed_bytes(M) / 16);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  rope_pack_kernel<<<unsigned(blocks), 256, 0, s>>>(reinterpret_cast<const float4*>(rope), M,
+                                                    reinterpret_cast<float4*>(packed), total);
+  return cudaGetLastError();
 }
 
 }  // namespace svdq

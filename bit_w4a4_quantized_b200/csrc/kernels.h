@@ -36,8 +36,18 @@ struct GemmLaunch {
   float alpha;
   int num_sms;
   uint64_t timeout_ns;
+  // fused QKV epilogue (qkv_cols = N / 3 > 0): per-head RMSNorm of Q and K,
+  // rotary turn of their pairs; V unchanged.  head_dim 128.
+  int32_t qkv_cols;
+  const uint16_t* norm_q;  // device bf16 [128]
+  const uint16_t* norm_k;  // device bf16 [128]
+  const float* rope;       // device packed rotary table (rope_packed_bytes(M) bytes)
+  float eps;
 };
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why);
+
+// [M][64][2] float (cos, sin) -> the packed layout of rope_packed_bytes(M).
+cudaError_t launch_rope_pack(const float* rope, int64_t M, float* packed, cudaStream_t s);
 
 // LoRA attach/detach: rewrite ranks [rank, rank_capacity) of L1^T and L2^T.
 struct LoraLaunch {

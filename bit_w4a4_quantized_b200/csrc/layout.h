@@ -42,6 +42,17 @@ SVDQ_HD int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 SVDQ_HD int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 SVDQ_HD size_t align256(size_t a) { return (a + 255) & ~size_t(255); }
 
+// Rotary table of the fused QKV epilogue (head_dim 128), packed so that the
+// epilogue's lanes (one output row each) read consecutive 16 bytes:
+//   [row tile t (an even count, like the GEMM's)][chunk c][row i of the tile]
+// of 16 bytes = (cos, sin) of pairs 2c and 2c + 1 of row 128 t + i (zeros
+// past the last row).
+constexpr int kRopeHeadDim = 128;
+constexpr int kRopeChunks = kRopeHeadDim / 4;  // 32 chunks of 2 pairs
+SVDQ_HD size_t rope_packed_bytes(int64_t M) {
+  return size_t(round_up(ceil_div(M, kBM), 2)) * kRopeChunks * kBM * 16;
+}
+
 // Byte offset, inside a tile of 128-byte rows, of byte `b` (0..127) of row
 // `row` under the 128-byte swizzle: the 16-byte chunk index is XORed with row % 8.
 SVDQ_HD uint32_t sw128(uint32_t row, uint32_t b) {

@@ -46,7 +46,8 @@ EXPORTED_SYMBOLS = (
     "svdq_prepare_host", "svdq_layer_upload", "svdq_prepare_weights", "svdq_act_buffer_bytes",
     "svdq_quantize_act", "svdq_w4a4_linear", "svdq_lora_swap", "svdq_layer_export", "svdq_act_unpack",
     "svdq_get_layer_info", "svdq_poll_status", "svdq_layer_destroy", "svdq_test_override_device_arch",
-    "svdq_test_bounded_wait", "svdq_layer_clone",
+    "svdq_test_bounded_wait", "svdq_layer_clone", "svdq_w4a4_linear_qkv_norm_rope",
+    "svdq_rope_packed_bytes", "svdq_rope_pack",
 )
 
 
@@ -102,6 +103,9 @@ def lib():
         "svdq_act_buffer_bytes": ([vp, i64, ctypes.POINTER(sz)], st),
         "svdq_quantize_act": ([vp, vp, i64, vp, sz, vp], st),
         "svdq_w4a4_linear": ([vp, vp, sz, i64, vp, ctypes.c_int, vp], st),
+        "svdq_w4a4_linear_qkv_norm_rope": ([vp, vp, sz, i64, vp, vp, vp, vp, sz, i32, ctypes.c_float, vp], st),
+        "svdq_rope_packed_bytes": ([i64, i32, ctypes.POINTER(sz)], st),
+        "svdq_rope_pack": ([vp, i64, i32, vp, sz, vp], st),
         "svdq_lora_swap": ([vp, vp, vp, i32, ctypes.c_float, vp], st),
         "svdq_layer_export": ([vp, ctypes.c_int, vp, sz], st),
         "svdq_act_unpack": ([vp, i64, vp, sz, vp, vp, vp], st),
@@ -127,6 +131,30 @@ def last_error():
 def check(status):
     if status != OK:
         raise SvdqError(status, last_error())
+
+
+def rope_packed_bytes(M, head_dim=128):
+    n = ctypes.c_size_t()
+    check(lib().svdq_rope_packed_bytes(int(M), int(head_dim), ctypes.byref(n)))
+    return n.value
+
+
+def rope_pack(rope, head_dim=128, out=None, stream=None):
+    """Device float32 [M, head_dim / 2, 2] (cos, sin) -> the packed table the
+    fused QKV epilogue reads (a uint8 device tensor)."""
+    import torch
+
+    M = rope.shape[0]
+    if not rope.is_contiguous() or rope.dtype != torch.float32:
+        raise ValueError("rope must be a contiguous float32 tensor")
+    if out is None:
+        out = torch.empty(rope_packed_bytes(M, head_dim), dtype=torch.uint8, device=rope.device)
+    check(lib().svdq_rope_pack(rope.data_ptr(), M, int(head_dim), out.data_ptr(), _nbytes(out), _stream(stream)))
+    return out
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
 
 
 def _ptr(a):
@@ -260,6 +288,21 @@ class Layer:
             out = torch.empty((M, self.N), dtype=torch.bfloat16, device=act.device)
         check(lib().svdq_w4a4_linear(self._h, act.data_ptr(), act.numel(), M, out.data_ptr(), epilogue,
                                      _stream(stream)))
+        return out
+
+    def linear_qkv_norm_rope(self, act, M, norm_q, norm_k, rope_packed, eps=1e-6, head_dim=128, out=None,
+                             stream=None):
+        """Kernel 2 on a fused Q | K | V layer with per-head RMSNorm of Q and K
+        and their rotary turn (norm_q, norm_k: device bf16 [head_dim];
+        rope_packed: from ``rope_pack``); returns bf16 [M, N]."""
+        import torch
+
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=act.device)
+        check(lib().svdq_w4a4_linear_qkv_norm_rope(self._h, act.data_ptr(), act.numel(), M, out.data_ptr(),
+                                                   _ptr(norm_q), _ptr(norm_k), _ptr(rope_packed),
+                                                   0 if rope_packed is None else _nbytes(rope_packed),
+                                                   int(head_dim), float(eps), _stream(stream)))
         return out
 
     def forward(self, X, out=None, epilogue=EPI_NONE, act=None, stream=None):

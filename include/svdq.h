@@ -23,7 +23,7 @@
  *   - Streams are cudaStream_t values passed as void*; NULL is the legacy
  *     default stream.  Launching entry points are asynchronous and stream
  *     ordered unless stated otherwise.
- *   - svdq_quantize_act and svdq_w4a4_linear launch with programmatic
+ *   - svdq_quantize_act and svdq_w4a4_linear(_qkv_norm_rope) launch with programmatic
  *     dependent launch: their prologue may overlap the previous kernel in the
  *     stream, but they touch no global memory before that kernel has completed
  *     (griddepcontrol.wait), so ordinary stream order holds for the caller.
@@ -179,6 +179,49 @@ SVDQ_API svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, i
  */
 SVDQ_API svdq_status svdq_w4a4_linear(const svdq_layer* layer, const void* act_buf, size_t act_buf_bytes,
                              int64_t M, void* Y, int epilogue, void* stream);
+
+/*
+ * Kernel 2 for a fused Q | K | V projection (Diffusers/Nunchaku page,
+ * fused-QKV section: to_q, to_k, to_v concatenated along the output dimension
+ * in that order, and the projection, the Q/K normalization and the rotary
+ * embedding handed to one fused operator).  The layer's output
+ * y = bf16(g_a g_w (Q(X_hat) Q(R) + lr' L2) + b), as svdq_w4a4_linear with
+ * SVDQ_EPI_NONE returns it, is split along N into Q, K and V of N / 3 columns,
+ * and those into heads of head_dim columns.  For every Q and K head of a row:
+ *   z = y / sqrt(mean(y^2) + eps) * w      (w = norm_q for Q, norm_k for K)
+ *   (z[2i], z[2i+1]) -> (z[2i] c - z[2i+1] s, z[2i+1] c + z[2i] s)
+ * with (c, s) the rotary angle of pair i of the row, in float32, rounded to
+ * bf16 once at the end.  V is written as y.  The page names the operator but
+ * not its arithmetic: the norm and the rotation above are the plain RMSNorm
+ * and rotary embedding.
+ * head_dim: 128 (SVDQ_ERR_UNSUPPORTED_SHAPE otherwise; N / 3 must be a
+ *   multiple of it).
+ * norm_q, norm_k: device bf16 [head_dim], 16-byte aligned.
+ * rope_packed: device, >= svdq_rope_packed_bytes(M) bytes, 16-byte aligned,
+ *   written by svdq_rope_pack from the [M][head_dim / 2][2] table; row m of Y
+ *   uses row m of the table.  One packed table serves every layer and call
+ *   with the same rows.
+ * eps: finite, >= 0 (FLUX uses 1e-6).
+ * act_buf, M, Y, stream: as svdq_w4a4_linear.
+ */
+SVDQ_API svdq_status svdq_w4a4_linear_qkv_norm_rope(const svdq_layer* layer, const void* act_buf,
+                                           size_t act_buf_bytes, int64_t M, void* Y, const void* norm_q,
+                                           const void* norm_k, const void* rope_packed,
+                                           size_t rope_packed_bytes, int32_t head_dim, float eps,
+                                           void* stream);
+
+/* Bytes of the packed rotary table for M rows (head_dim 128).  Host only. */
+SVDQ_API svdq_status svdq_rope_packed_bytes(int64_t M, int32_t head_dim, size_t* bytes);
+
+/*
+ * Pack a rotary table for svdq_w4a4_linear_qkv_norm_rope: rope is device float
+ * [M][head_dim / 2][2] = (cos, sin) of each row's pairs (16-byte aligned); the
+ * packed copy puts the same values in the order the epilogue's threads (one
+ * output row each) read them: row tiles of 128, then chunks of 2 pairs, then
+ * rows.  Stream ordered.  SVDQ_ERR_BUFFER_TOO_SMALL if packed_bytes is short.
+ */
+SVDQ_API svdq_status svdq_rope_pack(const void* rope, int64_t M, int32_t head_dim, void* packed,
+                                    size_t packed_bytes, void* stream);
 
 /*
  * Attach a LoRA adapter to the low-rank branch without touching R (abstract of

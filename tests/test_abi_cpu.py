@@ -94,6 +94,16 @@ def test_host_only_layer_cannot_launch():
         layer.export(svdq.EXPORT_R)  # not kept
 
 
+def test_rope_packed_bytes_follow_the_row_tiles():
+    n = ctypes.c_size_t()
+    L = svdq.lib()
+    assert L.svdq_rope_packed_bytes(1, 128, ctypes.byref(n)) == svdq.OK and n.value == 2 * 32 * 128 * 16
+    assert svdq.rope_packed_bytes(256) == 2 * 65536 and svdq.rope_packed_bytes(257) == 4 * 65536
+    assert L.svdq_rope_packed_bytes(0, 128, ctypes.byref(n)) == svdq.ERR_INVALID_ARGUMENT
+    assert L.svdq_rope_packed_bytes(16, 64, ctypes.byref(n)) == svdq.ERR_UNSUPPORTED_SHAPE
+    assert L.svdq_rope_pack(None, 16, 128, None, 0, None) == svdq.ERR_INVALID_ARGUMENT
+
+
 def test_calibrate_amax_is_running_max():
     x1 = WL.make_x(17, 64, seed=1)
     x2 = WL.make_x(9, 64, seed=2)
