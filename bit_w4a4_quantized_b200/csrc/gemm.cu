@@ -35,7 +35,11 @@
 //   * warps 0-15 of each CTA: epilogue, one output row x 64 columns per
 //     thread (warp w: lane quarter w % 4, columns 64 (w / 4) .. +63): tensor
 //     memory -> registers, release the accumulator to the leader, then alpha,
-//     bias, GELU -> bf16 -> global while the next tile's K loop runs.
+//     bias, GELU -> bf16 while the next tile's K loop runs.  Each warp writes
+//     32 rows x 16 columns at a time into its own 1 KB shared-memory buffer,
+//     and one lane hands the buffer to a TMA tensor store: Y leaves in whole
+//     sectors through the bulk-copy engine, not as row-strided stores that
+//     would contend with the operand feed.
 //   * The QKV instance (kQkv) finishes a fused Q|K|V projection instead
 //     (Diffusers/Nunchaku page, fused-QKV section: projection, Q/K norm and
 //     rotary embedding in one operator): each row's bf16 outputs of a Q or K
@@ -75,9 +79,25 @@ constexpr uint32_t kOffSFB = kOffSFA + kSFATileBytes;    // 4 KB
 constexpr uint32_t kStage2 = kOffSFB + kSFBTileBytes;    // 38912 bytes
 constexpr uint32_t kFoldBytes = 2 * kHalf * kRowBytes;   // lr' 16 KB + L2^T half 16 KB
 constexpr uint32_t kCtrl2 = 256;
-constexpr uint32_t kBiasBytes = kEpiWarps * 2 * 64 * 4;  // per epilogue warp: 2 tiles x 64 floats
+constexpr uint32_t kBiasBytes = kEpiWarps * 64 * 2;  // per epilogue warp: its 64 bias values (bf16)
 constexpr uint32_t kXchBytes = 8 * 2 * 64 * 4;  // QKV: [head warp pair][parity][2 halves x 32 rows] floats
 constexpr uint32_t kNormBytes = kEpiWarps * 64 * 4;  // QKV: per epilogue warp, its 64 norm_q and 64 norm_k weights
+// Output staging: each epilogue warp writes 32 rows x 16 columns of Y (1 KB,
+// 32-byte swizzle) to shared memory and one TMA store moves them to Y, so the
+// output leaves through the bulk-copy engine in whole sectors instead of 32
+// row-strided stores per instruction.  Two buffers per warp (one in the QKV
+// instance, whose exchange and weights take the room).
+constexpr uint32_t kYRows = 32, kYCols = 16, kYBufBytes = kYRows * kYCols * 2;
+template <bool kQkv>
+struct EpiSmem {
+  static constexpr int kYBufs = kQkv ? 1 : 2;
+  static constexpr uint32_t kXch = kStages2 * kStage2 + kCtrl2 + kBiasBytes;  // QKV only
+  static constexpr uint32_t kNorm = kXch + (kQkv ? kXchBytes : 0);
+  static constexpr uint32_t kY = (kNorm + (kQkv ? kNormBytes : 0) + 1023u) & ~1023u;
+  static constexpr uint32_t kEnd = kY + kEpiWarps * kYBufs * kYBufBytes;
+};
+static_assert(EpiSmem<false>::kEnd + 1024 <= 227 * 1024, "shared memory budget (plain)");
+static_assert(EpiSmem<true>::kEnd + 1024 <= 227 * 1024, "shared memory budget (QKV)");
 constexpr uint32_t kTmemCols2 = 512;
 constexpr uint32_t kColSFA = 256, kColSFB = kColSFA + 16 * kStages2;
 constexpr uint16_t kPairMask = 0x3;
@@ -94,6 +114,7 @@ constexpr int kRowsSFA = kSFATileBytes / kMapRow;           // 1
 constexpr int kRowsSFB = kSFBTileBytes / kMapRow;           // 2
 
 struct alignas(64) GemmMaps {
+  CUtensorMap y;    // Y bf16 [M, N], box = 32 rows x 16 columns, 32-byte swizzle
   CUtensorMap a;    // act codes, box = 128 rows of one tile (16 KB)
   CUtensorMap asf;  // act scales, box = one k-tile (2 KB)
   CUtensorMap lr;   // lr' tiles, box = 16 KB
@@ -137,12 +158,14 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
 }
 
 // 32 accumulator columns of one row -> alpha, bias, act -> 16 words of bf16 pairs.
-// `bias` points at the 32 bias values of these columns in shared memory (or null).
+// `bias` points at the 16 bf16 pairs of these columns' bias in shared memory (or null).
 template <bool kMayGelu = true>
-__device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t* v, const float* bias, uint32_t* out) {
+__device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t* v, const uint32_t* bias,
+                                             uint32_t* out) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    const float b0 = bias ? bias[2 * e] : 0.0f, b1 = bias ? bias[2 * e + 1] : 0.0f;
+    const uint32_t bw = bias ? bias[e] : 0u;
+    const float b0 = bf16lo(bw), b1 = bf16hi(bw);
     float y0 = fmaf(p.alpha, __uint_as_float(v[2 * e]), b0);
     float y1 = fmaf(p.alpha, __uint_as_float(v[2 * e + 1]), b1);
     if (kMayGelu && p.epilogue == SVDQ_EPI_GELU_TANH) {
@@ -151,6 +174,30 @@ __device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t
     }
     out[e] = f32x2_to_bf16x2(y0, y1);
   }
+}
+
+// 16 columns of this thread's row (8 words of bf16 pairs) -> the warp's staging
+// buffer `slot` (row = lane, two 16-byte chunks swizzled by bit 2 of the row)
+// -> one TMA store of the warp's 32 rows x 16 columns at (x, y).  Lane 0 owns
+// the warp's bulk groups; a buffer is rewritten only after its last store has
+// read it.
+template <int kBufs>
+__device__ __forceinline__ void store_y16(const CUtensorMap* map, uint8_t* ybuf, uint32_t ybuf_s, int lane,
+                                          const uint32_t* w, int32_t x, int32_t y, int32_t M, uint32_t& slot) {
+  if (y >= M) return;  // all 32 rows are padding (the same for the whole warp)
+  if (lane == 0) bulk_wait_read<kBufs - 1>();
+  __syncwarp();
+  uint8_t* b = ybuf + slot * kYBufBytes + uint32_t(lane) * 32u;
+  const uint32_t sw = (uint32_t(lane) >> 2) & 1u;
+  *reinterpret_cast<uint4*>(b + 16u * sw) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(b + 16u * (sw ^ 1u)) = make_uint4(w[4], w[5], w[6], w[7]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, ybuf_s + slot * kYBufBytes, x, y);
+    bulk_commit();
+  }
+  slot = slot + 1 == uint32_t(kBufs) ? 0u : slot + 1;
 }
 
 // kRopeBatch chunks (2 pairs each) of one Q or K head row: the bf16 values in
@@ -204,10 +251,11 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 104);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 108);
   const uint32_t SFULL = ctrl_s + 112u;  // 5 barriers: this CTA's scales of a stage have landed
-  float* bias_s = reinterpret_cast<float*>(ctrl + kCtrl2);  // [warp][tile parity][64] floats
+  uint32_t* bias_s = reinterpret_cast<uint32_t*>(ctrl + kCtrl2);  // [warp][32 bf16 pairs]
   const uint32_t XCH = ctrl_s + 152u;  // QKV: 8 barriers, one per warp pair sharing a head
-  float* xch = reinterpret_cast<float*>(ctrl + kCtrl2 + kBiasBytes);
-  uint32_t* norm_s = reinterpret_cast<uint32_t*>(ctrl + kCtrl2 + kBiasBytes + kXchBytes);
+  using ES = EpiSmem<kQkv>;
+  float* xch = reinterpret_cast<float*>(smem + ES::kXch);
+  uint32_t* norm_s = reinterpret_cast<uint32_t*>(smem + ES::kNorm);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
@@ -408,8 +456,10 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     // 64 (w / 4) .. +63: its share of the tile goes to registers, the
     // accumulator is released to the leader, then the rows are finished and
     // stored while the next tile's K loop runs.
-    uint32_t tc = 0, xc = 0;
+    uint32_t tc = 0, xc = 0, yslot = 0;
     const int quarter = warp & 3, colq = warp >> 2;
+    uint8_t* ybuf = smem + ES::kY + uint32_t(warp) * ES::kYBufs * kYBufBytes;
+    const uint32_t ybuf_s = sbase + ES::kY + uint32_t(warp) * ES::kYBufs * kYBufBytes;
     uint32_t* norm_w = norm_s + warp * 64;  // QKV: [Q, K][32 bf16 pairs] of this warp's columns
     if (kQkv) {
       const int half = colq & 1;
@@ -423,12 +473,10 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       int mp, nt;
       tile_coords(p, tile, mp, nt);
       const int mt = 2 * mp + int(rank);
-      // stage this warp's 64 bias values (warp-private, double buffered)
-      float* bias_w = bias_s + (size_t(warp) * 2 + (tc & 1u)) * 64;
-      if (p.bias) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(p.bias + size_t(nt) * kBN + colq * 64 + lane * 2);
-        *reinterpret_cast<float2*>(bias_w + lane * 2) = make_float2(bf16lo(w), bf16hi(w));
-      }
+      // stage this warp's 64 bias values (warp-private; the previous tile's reads are done)
+      uint32_t* bias_w = bias_s + warp * 32;
+      __syncwarp();
+      if (p.bias) bias_w[lane] = *reinterpret_cast<const uint32_t*>(p.bias + size_t(nt) * kBN + colq * 64 + lane * 2);
       __syncwarp();
       bool ok = mbar_wait(ACCF, tc & 1u, abort_flag, p.timeout_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);
@@ -445,6 +493,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
       const int64_t row = int64_t(mt) * kBM + row_in_tile;
+      const int32_t y0 = mt * kBM + quarter * 32;  // first row of this warp's share
       if constexpr (kQkv) {
         // the two warps of a head (colq 2h, 2h + 1) agree on every branch
         // below: the head's columns are all below N or all above (N % 128 == 0)
@@ -452,7 +501,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         if (n0 < p.N) {
           uint32_t out[32];
           finish_chunk<false>(p, v, p.bias ? bias_w : nullptr, out);
-          finish_chunk<false>(p, v + 32, p.bias ? bias_w + 32 : nullptr, out + 16);
+          finish_chunk<false>(p, v + 32, p.bias ? bias_w + 16 : nullptr, out + 16);
           const int part = n0 / p.qkv_cols;  // 0 Q, 1 K, 2 V
           if (part < 2) {
             float ss = 0.0f;
@@ -494,28 +543,26 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
               norm_rope_chunks(out + 2 * kRopeBatch * b, inv, wsm + 2 * kRopeBatch * b, t);
             }
           }
-          if (row < p.M) {
-            uint16_t* dst = p.Y + row * p.N + n0;
+          // rows past M are clipped by the tensor store
 #pragma unroll
-            for (int j = 0; j < 4; ++j) st_global_v8(dst + 16 * j, out + 8 * j);
-          }
+          for (int j = 0; j < 4; ++j) store_y16<ES::kYBufs>(&maps.y, ybuf, ybuf_s, lane, out + 8 * j, n0 + 16 * j, y0, p.M, yslot);
         }
-      } else if (row < p.M) {
+      } else {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int n0 = nt * kBN + colq * 64 + q * 32;
-          if (n0 < p.N) {
+          if (n0 < p.N) {  // N % 64 == 0: the warp's 64 columns are all in or all out
             uint32_t out[16];
-            finish_chunk(p, v + 32 * q, p.bias ? bias_w + q * 32 : nullptr, out);
-            // 64 bytes at a 32-byte aligned address (n0 % 32 == 0, N % 64 == 0, Y 32-byte aligned)
-            uint16_t* dst = p.Y + row * p.N + n0;
-            st_global_v8(dst, out);
-            st_global_v8(dst + 16, out + 8);
+            finish_chunk(p, v + 32 * q, p.bias ? bias_w + q * 16 : nullptr, out);
+            store_y16<ES::kYBufs>(&maps.y, ybuf, ybuf_s, lane, out, n0, y0, p.M, yslot);
+            store_y16<ES::kYBufs>(&maps.y, ybuf, ybuf_s, lane, out + 8, n0 + 16, y0, p.M, yslot);
           }
         }
       }
       ++tc;
     }
+    if (lane == 0) bulk_wait_read<0>();  // the staging buffers are read before the CTA may exit
+    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown
@@ -552,6 +599,19 @@ bool encode_rows(CUtensorMap* m, const void* base, uint64_t bytes, uint32_t box)
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Y bf16 [M, N] row-major for the epilogue's tensor stores: box 32 rows x 16 columns.
+bool encode_y(CUtensorMap* m, void* Y, int64_t M, int64_t N) {
+  auto enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(M)};
+  const cuuint64_t strides[1] = {cuuint64_t(N) * 2u};
+  const cuuint32_t boxd[2] = {kYCols, kYRows};
+  const cuuint32_t es[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Y, dims, strides, boxd, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
@@ -563,7 +623,8 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   bool ok = encode_rows(&maps.a, act + ag.off_codes, uint64_t(ag.MT) * ag.KT * kATileBytes, kRowsA) &&
             encode_rows(&maps.asf, act + ag.off_sf, uint64_t(ag.MT) * ag.KT * kSFATileBytes, kRowsSFA) &&
             encode_rows(&maps.b, lay + lg.off_bcodes, uint64_t(lg.NT) * lg.KT * kBTileBytes, kRowsA) &&
-            encode_rows(&maps.bsf, lay + lg.off_sfb, uint64_t(lg.NT) * lg.KT * kSFBTileBytes, kRowsSFB);
+            encode_rows(&maps.bsf, lay + lg.off_sfb, uint64_t(lg.NT) * lg.KT * kSFBTileBytes, kRowsSFB) &&
+            encode_y(&maps.y, a.Y, a.M, lg.N);
   if (ok && lg.RJ > 0) {
     ok = encode_rows(&maps.lr, act + ag.off_lr, uint64_t(ag.MT) * ag.RJ * kATileBytes, kRowsA) &&
          encode_rows(&maps.l2, lay + lg.off_l2t, uint64_t(lg.NT) * lg.RJ * kBTileBytes, kRowsA);
@@ -602,7 +663,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
     *why = "problem too large for one launch";
     return cudaErrorInvalidValue;
   }
-  const size_t smem = size_t(kStages2) * kStage2 + kCtrl2 + kBiasBytes + (qkv ? kXchBytes + kNormBytes : 0) + 1024;
+  const size_t smem = size_t(qkv ? EpiSmem<true>::kEnd : EpiSmem<false>::kEnd) + 1024;
   static std::atomic<int> max_pairs_of[2][64];
   int dev = 0;
   cudaGetDevice(&dev);
