@@ -97,6 +97,7 @@ struct EpiSmem {
   static constexpr uint32_t kEnd = kY + kEpiWarps * kYBufs * kYBufBytes;
 };
 static_assert(EpiSmem<false>::kEnd + 1024 <= 227 * 1024, "shared memory budget (plain)");
+static_assert(kEpiWarps * 4 * kYBufBytes <= kStages2 * kStage2, "last-tile staging fits in the stage ring");
 static_assert(EpiSmem<true>::kEnd + 1024 <= 227 * 1024, "shared memory budget (QKV)");
 constexpr uint32_t kTmemCols2 = 512;
 constexpr uint32_t kColSFA = 256, kColSFB = kColSFA + 16 * kStages2;
@@ -176,28 +177,34 @@ __device__ __forceinline__ void finish_chunk(const GemmParams& p, const uint32_t
   }
 }
 
-// 16 columns of this thread's row (8 words of bf16 pairs) -> the warp's staging
-// buffer `slot` (row = lane, two 16-byte chunks swizzled by bit 2 of the row)
-// -> one TMA store of the warp's 32 rows x 16 columns at (x, y).  Lane 0 owns
-// the warp's bulk groups; a buffer is rewritten only after its last store has
-// read it.
+// 16 columns of this thread's row (8 words of bf16 pairs) -> buffer `slot` of
+// the warp's staging area (row = lane, two 16-byte chunks swizzled by bit 2 of
+// the row) -> one TMA store of the warp's 32 rows x 16 columns at (x, y).
+// Lane 0 owns the warp's bulk groups; a buffer is rewritten only after its
+// last store has read it (kBufs buffers normally, 4 on the CTA's last tile).
 template <int kBufs>
-__device__ __forceinline__ void store_y16(const CUtensorMap* map, uint8_t* ybuf, uint32_t ybuf_s, int lane,
+__device__ __forceinline__ void store_y16(const CUtensorMap* map, uint8_t* buf, uint32_t buf_s, bool last, int lane,
                                           const uint32_t* w, int32_t x, int32_t y, int32_t M, uint32_t& slot) {
   if (y >= M) return;  // all 32 rows are padding (the same for the whole warp)
-  if (lane == 0) bulk_wait_read<kBufs - 1>();
+  if (lane == 0) {
+    if (last)
+      bulk_wait_read<3>();
+    else
+      bulk_wait_read<kBufs - 1>();
+  }
   __syncwarp();
-  uint8_t* b = ybuf + slot * kYBufBytes + uint32_t(lane) * 32u;
+  uint8_t* b = buf + slot * kYBufBytes + uint32_t(lane) * 32u;
   const uint32_t sw = (uint32_t(lane) >> 2) & 1u;
   *reinterpret_cast<uint4*>(b + 16u * sw) = make_uint4(w[0], w[1], w[2], w[3]);
   *reinterpret_cast<uint4*>(b + 16u * (sw ^ 1u)) = make_uint4(w[4], w[5], w[6], w[7]);
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(map, ybuf_s + slot * kYBufBytes, x, y);
+    tma_store_2d(map, buf_s + slot * kYBufBytes, x, y);
     bulk_commit();
   }
-  slot = slot + 1 == uint32_t(kBufs) ? 0u : slot + 1;
+  const uint32_t n = last ? 4u : uint32_t(kBufs);
+  slot = slot + 1 == n ? 0u : slot + 1;
 }
 
 // kRopeBatch chunks (2 pairs each) of one Q or K head row: the bf16 values in
@@ -494,6 +501,16 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
       const int64_t row = int64_t(mt) * kBM + row_in_tile;
       const int32_t y0 = mt * kBM + quarter * 32;  // first row of this warp's share
+      // On its last tile the CTA's stage ring is idle (every MMA that read it
+      // has completed): each warp stages its 4 stores there, 4 KB apart, and
+      // never waits for a buffer.
+      const bool last = tile + npairs >= ntiles;
+      if (last) yslot = 0;
+      uint8_t* const sbuf = last ? smem + uint32_t(warp) * 4u * kYBufBytes : ybuf;
+      const uint32_t sbuf_s = last ? sbase + uint32_t(warp) * 4u * kYBufBytes : ybuf_s;
+      auto put16 = [&](const uint32_t* w, int32_t x) {
+        store_y16<ES::kYBufs>(&maps.y, sbuf, sbuf_s, last, lane, w, x, y0, p.M, yslot);
+      };
       if constexpr (kQkv) {
         // the two warps of a head (colq 2h, 2h + 1) agree on every branch
         // below: the head's columns are all below N or all above (N % 128 == 0)
@@ -545,7 +562,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           }
           // rows past M are clipped by the tensor store
 #pragma unroll
-          for (int j = 0; j < 4; ++j) store_y16<ES::kYBufs>(&maps.y, ybuf, ybuf_s, lane, out + 8 * j, n0 + 16 * j, y0, p.M, yslot);
+          for (int j = 0; j < 4; ++j) put16(out + 8 * j, n0 + 16 * j);
         }
       } else {
 #pragma unroll
@@ -554,8 +571,8 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           if (n0 < p.N) {  // N % 64 == 0: the warp's 64 columns are all in or all out
             uint32_t out[16];
             finish_chunk(p, v + 32 * q, p.bias ? bias_w + q * 16 : nullptr, out);
-            store_y16<ES::kYBufs>(&maps.y, ybuf, ybuf_s, lane, out, n0, y0, p.M, yslot);
-            store_y16<ES::kYBufs>(&maps.y, ybuf, ybuf_s, lane, out + 8, n0 + 16, y0, p.M, yslot);
+            put16(out, n0);
+            put16(out + 8, n0 + 16);
           }
         }
       }
