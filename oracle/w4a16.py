@@ -1,0 +1,69 @@
+"""W4A16 linear layer: 4-bit weights, 16-bit activations.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).  Plain NumPy, float64
+except where a step is defined in float32.
+
+Sources: the Diffusers/Nunchaku page names a second kernel family next to the
+W4A4 one, awq_w4a16: 4-bit weights with 16-bit activations, for the adaptive
+norm and modulation projections (FLUX adanorm_single / adanorm_zero), which
+are memory bound and precision sensitive.  The SVDQuant summary page, section
+2 "AWQ", describes AWQ as activation-aware weight quantization that protects
+the weights that matter by shifting scale onto the activations; its section 3
+notes that W4A16 upcasts the weights, so the gain is memory, not arithmetic.
+
+Readings of what the pages leave open:
+  * The 4-bit weights use the NVFP4 encoding of the W4A4 layer's residual:
+    E2M1 codes, one E4M3 scale per 16 consecutive weights along K, a float32
+    tensor scale g = amax / 2688 (1 when amax is 0).
+  * The activation-aware scale is one positive float32 s_j per input channel
+    (1 when absent): the quantized weight is W' = f32(W diag(s)), and the
+    activations are divided by s at run time, x~_j = f32(x_j * f32(1 / s_j)),
+    so X W^T = X~ W'^T before quantization.  The pages give no rule for
+    choosing s (AWQ searches for it offline), so s is an input of the layer.
+  * Y = g * sum_j x~_j deq(W')_nj + b, act = identity, rounded to bf16 once.
+"""
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import svdquant as S
+
+
+@dataclass
+class W4A16:
+    codes: np.ndarray   # uint8 [N, K], one E2M1 code per weight (sign in bit 3)
+    scales: np.ndarray  # uint8 [N, K / 16], E4M3
+    g: np.float32       # tensor scale
+    inv_s: np.ndarray   # float32 [K]
+    bias: np.ndarray    # float64 [N] or None
+    deq: np.ndarray     # float64 [N, K] = e2m1 * e4m3 (without g)
+
+
+def prepare(W, s=None, bias=None):
+    """Quantize W [N, K] (float32 values of bf16 weights) as W' = f32(W diag(s))."""
+    W = np.asarray(W, np.float32)
+    N, K = W.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    s32 = np.ones(K, np.float32) if s is None else np.asarray(s, np.float32)
+    if np.any(~(s32 > 0)) or not np.all(np.isfinite(s32)):
+        raise ValueError("s must be positive and finite")
+    Wp = (W * s32[None, :]).astype(np.float32)
+    g = S.global_scale(np.max(np.abs(Wp)) if Wp.size else np.float32(0))
+    codes, scales = S.nvfp4_quantize(Wp, g)
+    inv_s = (np.float32(1.0) / s32).astype(np.float32)
+    b = None if bias is None else np.asarray(bias, np.float64)
+    return W4A16(codes, scales, np.float32(g), inv_s, b, S.nvfp4_dequantize(codes, scales))
+
+
+def linear(layer, X, rows=None):
+    """Y = g * (X~ @ deq^T) + b in float64, X~ = f32(X * inv_s)."""
+    X = np.asarray(X, np.float32)
+    if rows is not None:
+        X = X[rows]
+    Xt = (X * layer.inv_s[None, :]).astype(np.float32).astype(np.float64)
+    y = np.float64(layer.g) * (Xt @ layer.deq.T)
+    if layer.bias is not None:
+        y = y + layer.bias[None, :]
+    return y

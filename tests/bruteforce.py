@@ -156,3 +156,24 @@ def qkv_norm_rope(Y, norm_q, norm_k, rope, eps, head_dim):
                     out[m][h0 + 2 * i] = z[2 * i] * c - z[2 * i + 1] * s
                     out[m][h0 + 2 * i + 1] = z[2 * i + 1] * c + z[2 * i] * s
     return out
+
+
+def w4a16_forward(W, X, s, bias=None):
+    """W4A16 layer on nested lists: W [N][K], X [M][K], s [K] (per input channel)."""
+    N, K = len(W), len(W[0])
+    Wp = [[f32r(W[n][j] * s[j]) for j in range(K)] for n in range(N)]
+    g = global_scale(max(abs(v) for row in Wp for v in row))
+    codes, scales = quantize_rows(Wp, g)
+    dw = deq(codes, scales)
+    inv = [f32r(1.0 / s[j]) for j in range(K)]
+    Y = []
+    for x in X:
+        xt = [f32r(x[j] * inv[j]) for j in range(K)]
+        row = []
+        for n in range(N):
+            y = g * math.fsum(xt[j] * dw[n][j] for j in range(K))
+            if bias is not None:
+                y += bias[n]
+            row.append(y)
+        Y.append(row)
+    return dict(codes=codes, scales=scales, g=g, Y=Y)
