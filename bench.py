@@ -616,6 +616,56 @@ def sweep_point(spec, device, steps, factors_cache):
     return out
 
 
+def w4a16_point(spec, device, steps):
+    """The W4A16 layer on one modulation shape: kernel time over rotating weight copies (more than L2),
+    the weight stream's GB/s against the measured HBM peak, and bf16 cuBLAS on the same shape."""
+    import torch
+
+    from bit_w4a4_quantized_b200 import svdq
+
+    M, K, N = spec.M, spec.K, spec.N
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.uint16).astype(np.int16)).view(
+        torch.bfloat16).to(device)
+    W, s, b = spec.w(), spec.s(), spec.b()
+    base = svdq.W4A16Layer(W, s=s, bias=b)
+    wbytes = N * K // 2 + N * K // 16
+    nsets = int(min(8, max(2, math.ceil(3 * L2_BYTES / wbytes))))
+    layers = []
+    for _ in range(nsets):
+        L = svdq.W4A16Layer(W, s=s, bias=b)
+        L.upload(device)
+        layers.append(L)
+    Xd = to_dev(spec.x())
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(nsets):
+            layers[i].linear(Xd, out=Ys[i], stream=stream)
+        stream.synchronize()
+    gr = _capture([lambda i=i: layers[i].linear(Xd, out=Ys[i], stream=stream) for i in range(nsets)], stream)
+    t = _graph_seconds(gr, nsets, steps, stream, device)
+    algo = wbytes + 4 * K + 2 * N + 2 * M * K + 2 * M * N  # weights, 1/s, bias, X, Y
+    _, peak, peak_kind = measured_peaks()
+    Wd = [to_dev(W) for _ in range(nsets)]
+    Yc = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+    mm = [lambda i=i: torch.matmul(Xd, Wd[i].t(), out=Yc[i]) for i in range(nsets)]
+    with torch.cuda.stream(stream):
+        for f in mm:
+            f()
+        stream.synchronize()
+    gc = _capture(mm, stream)
+    tc = _graph_seconds(gc, nsets, steps, stream, device)
+    out = {"workload": spec.name, "layer": "w4a16", "M": M, "K": K, "N": N, "w4a16_us": round(t * 1e6, 3),
+           "bytes": algo, "GBps": round(algo / t / 1e9, 1), "hbm_peak_GBps": peak, "peak_kind": peak_kind,
+           "frac_of_hbm": round(algo / t / 1e9 / peak, 3),
+           "cublas_bf16_us": round(tc * 1e6, 3), "speedup_vs_cublas_bf16": round(tc / t, 3)}
+    del gr, gc
+    base.close()
+    for L in layers:
+        L.close()
+    return out
+
+
 def run_sweep(args):
     import torch
 
@@ -630,13 +680,18 @@ def run_sweep(args):
             specs += [WL.CFG2, WL.CFG3_FC1, WL.CFG3_FC2, WL.CFG4] + WL.sweep()
         elif n == "sweep":
             specs += WL.sweep()
+        elif n == "w4a16":
+            specs += [WL.w4a16_spec(m, N=nn) for nn in (18432, 9216) for m in (1, 2, 4)]
         else:
             specs.append(workload_spec(n))
     cache = {}
     props = torch.cuda.get_device_properties(device)
     for spec in specs:
         with ClockSampler(getattr(props, "uuid", None)) as clk:
-            row = sweep_point(spec, device, args.sweep_steps, cache)
+            if isinstance(spec, WL.W4A16Spec):
+                row = w4a16_point(spec, device, args.sweep_steps)
+            else:
+                row = sweep_point(spec, device, args.sweep_steps, cache)
         row["clocks"] = clk.summary()
         print(json.dumps(row), flush=True)
         torch.cuda.empty_cache()
@@ -677,7 +732,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", default=None,
-                    help="per-shape report instead of the bench line: 'all', 'sweep' or workload names, comma separated")
+                    help="per-shape report instead of the bench line: 'all', 'sweep', 'w4a16' or workload names, "
+                         "comma separated")
     ap.add_argument("--sweep-steps", type=int, default=50)
     args = ap.parse_args(argv)
     if args.sweep:

@@ -13,6 +13,7 @@
 
 #include "kernels.h"
 #include "layer.h"
+#include "w4a16.h"
 
 namespace {
 
@@ -371,5 +372,93 @@ svdq_status svdq_test_bounded_wait(uint64_t timeout_ns, uint32_t* status_out, vo
   if (e != cudaSuccess) return cuda_fail(e, "bounded-wait test kernel");
   return SVDQ_OK;
 }
+
+
+// ------------------------------------------------------------------ W4A16
+size_t svdq_w4a16_device_bytes(const svdq_w4a16_desc* d) {
+  if (!d || d->K < 64 || d->K % 64 || d->K > 12288 || d->N < 1 || d->N > (int64_t(1) << 24)) {
+    g_last_error = "bad W4A16 descriptor";
+    return 0;
+  }
+  return svdq::make_w4a16_geom(d->K, d->N).total;
+}
+
+svdq_status svdq_w4a16_prepare_host(const svdq_w4a16_desc* d, svdq_w4a16** out) {
+  if (!out) return fail(SVDQ_ERR_INVALID_ARGUMENT, "out is NULL");
+  std::string err;
+  auto* L = new (std::nothrow) svdq_w4a16();
+  if (!L) return fail(SVDQ_ERR_INTERNAL, "out of host memory");
+  svdq_status st = svdq::w4a16_quantize(d, &L->image, &L->gscale, &err);
+  if (st != SVDQ_OK) {
+    delete L;
+    return fail(st, err);
+  }
+  L->g = svdq::make_w4a16_geom(d->K, d->N);
+  L->has_bias = d->bias != nullptr;
+  *out = L;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_w4a16_upload(svdq_w4a16* L, void* dev_buf, size_t dev_buf_bytes, void* stream) {
+  if (!L || !dev_buf) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and dev_buf are required");
+  if (!aligned(dev_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "dev_buf must be 256-byte aligned");
+  if (dev_buf_bytes < L->g.total)
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "dev_buf needs " + std::to_string(L->g.total) + " bytes");
+  int dev = 0, sms = 0;
+  svdq_status st = check_device(&dev, &sms);
+  if (st != SVDQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(dev_buf, L->image.data(), L->g.total, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(W4A16 image)");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  L->dev_buf = dev_buf;
+  L->device = dev;
+  L->num_sms = sms;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_w4a16_linear(const svdq_w4a16* L, const void* X, int64_t M, void* Y, void* stream) {
+  if (!L) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is NULL");
+  if (!L->dev_buf) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is not uploaded to a device");
+  if (!X || !Y) return fail(SVDQ_ERR_INVALID_ARGUMENT, "X and Y are required");
+  if (M < 1 || M > (int64_t(1) << 31) / L->g.N) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M out of range");
+  if (!aligned(X, 16)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "X must be 16-byte aligned");
+  if (!aligned(Y, 2)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "Y must be 2-byte aligned");
+  svdq_status st = check_device(nullptr, nullptr);
+  if (st != SVDQ_OK) return st;
+  svdq::W4A16Launch a{};
+  a.layer = static_cast<const uint8_t*>(L->dev_buf);
+  a.g = L->g;
+  a.X = static_cast<const uint16_t*>(X);
+  a.M = M;
+  a.Y = static_cast<uint16_t*>(Y);
+  a.gscale = L->gscale;
+  a.has_bias = L->has_bias ? 1 : 0;
+  a.num_sms = L->num_sms;
+  const char* why = "";
+  cudaError_t e = svdq::launch_w4a16(a, static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_w4a16_export(const svdq_w4a16* L, int what, void* host_dst, size_t bytes) {
+  if (!L || !host_dst) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and host_dst are required");
+  const auto& g = L->g;
+  const uint8_t* img = L->image.data();
+  const void* src = nullptr;
+  size_t n = 0;
+  switch (what) {
+    case SVDQ_EXPORT_W_CODES: src = img + g.off_codes; n = size_t(g.N) * size_t(g.K / 2); break;
+    case SVDQ_EXPORT_W_SCALES: src = img + g.off_scales; n = size_t(g.N) * size_t(g.K / 16); break;
+    case SVDQ_EXPORT_INV_LAMBDA: src = img + g.off_inv_s; n = size_t(g.K) * 4; break;
+    case SVDQ_EXPORT_SCALARS: src = &L->gscale; n = 4; break;
+    default: return fail(SVDQ_ERR_INVALID_ARGUMENT, "unknown export for a W4A16 layer");
+  }
+  if (bytes < n) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "export needs " + std::to_string(n) + " bytes");
+  std::memcpy(host_dst, src, n);
+  return SVDQ_OK;
+}
+
+void svdq_w4a16_destroy(svdq_w4a16* L) { delete L; }
 
 }  // extern "C"

@@ -20,6 +20,7 @@
 
 #include "layer.h"
 #include "svd.h"
+#include "w4a16.h"
 
 namespace svdq {
 
@@ -327,6 +328,55 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
 }
 
 // ---------------------------------------------------------------- exports
+
+// W4A16: W' = f32(W diag(s)) quantized row by row with the same NVFP4 quantizer
+// as the W4A4 residual, under the tensor scale g = max|W'| / 2688.
+svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image, float* g_out, std::string* err) {
+  if (!d || !d->W) {
+    *err = "descriptor and W are required";
+    return SVDQ_ERR_INVALID_ARGUMENT;
+  }
+  const int64_t K = d->K, N = d->N;
+  if (K < 64 || K % 64 || K > 12288 || N < 1 || N > (int64_t(1) << 24)) {
+    *err = "K must be a multiple of 64 in [64, 12288] and N in [1, 2^24]";
+    return SVDQ_ERR_UNSUPPORTED_SHAPE;
+  }
+  std::vector<float> s(size_t(K), 1.0f);
+  if (d->s)
+    for (int64_t k = 0; k < K; ++k) {
+      s[size_t(k)] = d->s[k];
+      if (!(s[size_t(k)] > 0.0f) || !std::isfinite(s[size_t(k)])) {
+        *err = "s must be positive and finite";
+        return SVDQ_ERR_INVALID_ARGUMENT;
+      }
+    }
+  const uint16_t* W = static_cast<const uint16_t*>(d->W);
+  std::vector<float> wp(size_t(N) * size_t(K));
+  float amax = 0.0f;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      const float v = bf16_bits_to_f32(W[size_t(n) * K + k]) * s[size_t(k)];
+      wp[size_t(n) * K + k] = v;
+      amax = std::max(amax, std::fabs(v));
+    }
+  const float g = global_scale(amax);
+  const float c = 1.0f / (6.0f * g);
+  const W4A16Geom geo = make_w4a16_geom(K, N);
+  image->assign(geo.total, 0);
+  uint8_t* img = image->data();
+  float* inv = reinterpret_cast<float*>(img + geo.off_inv_s);
+  for (int64_t k = 0; k < K; ++k) inv[k] = 1.0f / s[size_t(k)];
+  if (d->bias) std::memcpy(img + geo.off_bias, d->bias, sizeof(uint16_t) * size_t(N));
+  const int threads = int(std::max(1u, std::min(16u, std::thread::hardware_concurrency())));
+  parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
+    for (int64_t n = n0; n < n1; ++n)
+      quantize_row(&wp[size_t(n) * K], K, g, c,
+                   [&](int64_t k, uint8_t byte) { img[geo.off_codes + size_t(n) * size_t(K / 2) + size_t(k / 2)] = byte; },
+                   [&](int64_t sb, uint8_t code) { img[geo.off_scales + size_t(n) * size_t(K / 16) + size_t(sb)] = code; });
+  });
+  *g_out = g;
+  return SVDQ_OK;
+}
 
 svdq_status export_array(const svdq_layer* L, int what, void* dst, size_t bytes, std::string* err) {
   const LayerGeom& g = L->g;

@@ -47,7 +47,8 @@ EXPORTED_SYMBOLS = (
     "svdq_quantize_act", "svdq_w4a4_linear", "svdq_lora_swap", "svdq_layer_export", "svdq_act_unpack",
     "svdq_get_layer_info", "svdq_poll_status", "svdq_layer_destroy", "svdq_test_override_device_arch",
     "svdq_test_bounded_wait", "svdq_layer_clone", "svdq_w4a4_linear_qkv_norm_rope",
-    "svdq_rope_packed_bytes", "svdq_rope_pack",
+    "svdq_rope_packed_bytes", "svdq_rope_pack", "svdq_w4a16_device_bytes", "svdq_w4a16_prepare_host",
+    "svdq_w4a16_upload", "svdq_w4a16_linear", "svdq_w4a16_export", "svdq_w4a16_destroy",
 )
 
 
@@ -65,6 +66,13 @@ class PrepareDesc(ctypes.Structure):
         ("W", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("act_amax", ctypes.c_void_p),
         ("L1", ctypes.c_void_p), ("L2", ctypes.c_void_p),
         ("svd_seed", ctypes.c_uint64), ("svd_power_iters", ctypes.c_int32), ("svd_oversample", ctypes.c_int32),
+    ]
+
+
+class W4A16Desc(ctypes.Structure):
+    _fields_ = [
+        ("K", ctypes.c_int64), ("N", ctypes.c_int64), ("W", ctypes.c_void_p), ("s", ctypes.c_void_p),
+        ("bias", ctypes.c_void_p),
     ]
 
 
@@ -113,6 +121,12 @@ def lib():
         "svdq_poll_status": ([vp, vp], st),
         "svdq_layer_destroy": ([vp], None),
         "svdq_layer_clone": ([vp, ctypes.POINTER(vp)], st),
+        "svdq_w4a16_device_bytes": ([ctypes.POINTER(W4A16Desc)], sz),
+        "svdq_w4a16_prepare_host": ([ctypes.POINTER(W4A16Desc), ctypes.POINTER(vp)], st),
+        "svdq_w4a16_upload": ([vp, vp, sz, vp], st),
+        "svdq_w4a16_linear": ([vp, vp, i64, vp, vp], st),
+        "svdq_w4a16_export": ([vp, ctypes.c_int, vp, sz], st),
+        "svdq_w4a16_destroy": ([vp], None),
         "svdq_test_override_device_arch": ([ctypes.c_int], None),
         "svdq_test_bounded_wait": ([ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32), vp], st),
     }
@@ -351,6 +365,67 @@ class Layer:
     def close(self):
         if self._h is not None and _lib is not None:
             _lib.svdq_layer_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class W4A16Layer:
+    """A W4A16 layer: 4-bit NVFP4 weights of W diag(s), bf16 activations divided by s."""
+
+    def __init__(self, W, s=None, bias=None, *, device=None, stream=None):
+        self._h = None
+        w = _bf16_bits(W)
+        self.N, self.K = w.shape
+        sv = None if s is None else np.ascontiguousarray(np.asarray(s, dtype=np.float32))
+        b = _bf16_bits(bias)
+        d = W4A16Desc()
+        d.K, d.N, d.W, d.s, d.bias = self.K, self.N, _ptr(w), _ptr(sv), _ptr(b)
+        self.device_bytes = lib().svdq_w4a16_device_bytes(ctypes.byref(d))
+        if self.device_bytes == 0:
+            raise SvdqError(ERR_UNSUPPORTED_SHAPE, last_error())
+        h = ctypes.c_void_p()
+        check(lib().svdq_w4a16_prepare_host(ctypes.byref(d), ctypes.byref(h)))
+        self._h = h
+        self.dev_buf = None
+        if device is not None:
+            self.upload(device, stream)
+
+    def upload(self, device="cuda", stream=None):
+        import torch
+
+        self.dev_buf = torch.empty(self.device_bytes, dtype=torch.uint8, device=device)
+        with torch.cuda.device(self.dev_buf.device):
+            check(lib().svdq_w4a16_upload(self._h, self.dev_buf.data_ptr(), self.device_bytes, _stream(stream)))
+
+    def linear(self, X, out=None, stream=None):
+        """Y bf16 [M, N] from a device bf16 [M, K] tensor."""
+        import torch
+
+        if not X.is_contiguous():
+            raise ValueError("X must be contiguous")
+        M = X.shape[0]
+        if out is None:
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=X.device)
+        check(lib().svdq_w4a16_linear(self._h, X.data_ptr(), M, out.data_ptr(), _stream(stream)))
+        return out
+
+    def export(self, what):
+        K, N = self.K, self.N
+        shapes = {EXPORT_W_CODES: ((N, K // 2), np.uint8), EXPORT_W_SCALES: ((N, K // 16), np.uint8),
+                  EXPORT_INV_LAMBDA: ((K,), np.float32), EXPORT_SCALARS: ((1,), np.float32)}
+        shape, dt = shapes.get(what, ((1,), np.uint8))  # anything else: the library reports the error
+        out = np.empty(shape, dtype=dt)
+        check(lib().svdq_w4a16_export(self._h, what, out.ctypes.data, out.nbytes))
+        return out
+
+    def close(self):
+        if self._h is not None and _lib is not None:
+            _lib.svdq_w4a16_destroy(self._h)
         self._h = None
 
     def __del__(self):

@@ -32,6 +32,7 @@ STREAM_W2_OUTLIER = 8
 STREAM_SAMPLE = 9
 STREAM_NORM_Q = 10
 STREAM_NORM_K = 11
+STREAM_AWQ_S = 12
 
 
 def rng(seed, stream):
@@ -94,6 +95,39 @@ def make_rope(M, head_dim, base=10000.0):
     freq = base ** (-2.0 * np.arange(head_dim // 2, dtype=np.float64) / head_dim)
     ang = m * freq[None, :]
     return np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32)
+
+
+def make_awq_scales(K, seed, spread=0.5):
+    """Positive per-input-channel scales exp(U(-spread, spread)) for the W4A16 layer (float32)."""
+    return np.exp(rng(seed, STREAM_AWQ_S).uniform(-spread, spread, K)).astype(np.float32)
+
+
+@dataclass(frozen=True)
+class W4A16Spec:
+    """A W4A16 modulation projection: M conditioning rows, K -> N."""
+
+    name: str
+    M: int
+    K: int
+    N: int
+    seed: int
+
+    def x(self):
+        return make_x(self.M, self.K, self.seed, n_outlier=0)
+
+    def w(self):
+        return make_w(self.N, self.K, self.seed)
+
+    def s(self):
+        return make_awq_scales(self.K, self.seed)
+
+    def b(self):
+        return make_bias(self.N, self.seed)
+
+
+def w4a16_spec(M, N=18432, K=3072):
+    """FLUX-like modulation projection: 3072 -> 6 x 3072 (double blocks) or 3 x 3072 (single blocks)."""
+    return W4A16Spec(f"w4a16_mod_M{M}_K{K}_N{N}", M, K, N, seed=5)
 
 
 @dataclass(frozen=True)

@@ -295,6 +295,58 @@ SVDQ_API void svdq_layer_destroy(svdq_layer* layer);
 SVDQ_API svdq_status svdq_layer_clone(const svdq_layer* layer, svdq_layer** out);
 
 /*
+ * The W4A16 layer (Diffusers/Nunchaku page: the awq_w4a16 kernel family, 4-bit
+ * weights with 16-bit activations, for the memory-bound adaptive-norm and
+ * modulation projections; SVDQuant summary page, section 2 "AWQ": protect the
+ * weights by shifting scale onto the activations):
+ *
+ *     Y = g (X diag(s)^-1) deq(Q(W diag(s)))^T + b
+ *
+ * Q is the NVFP4 quantizer of the W4A4 layer (E2M1 codes, an E4M3 scale per 16
+ * weights along K, tensor scale g = max|W diag(s)| / 2688); s is one positive
+ * activation-aware scale per input channel (the pages give no rule for it:
+ * it is an input, 1 when NULL).  Activations stay bf16 and are divided by s
+ * in float32; the sums are float32; Y is bf16.  The path is built for the
+ * small batches of the modulation layers (M rows of X, a few at a time).
+ */
+typedef struct svdq_w4a16 svdq_w4a16;
+
+typedef struct svdq_w4a16_desc {
+  int64_t K;          /* input features, multiple of 64, <= 12288 */
+  int64_t N;          /* output features, >= 1 */
+  const void* W;      /* host bf16 [N, K] (nn.Linear layout) */
+  const float* s;     /* host float [K] activation-aware scales (> 0), or NULL */
+  const void* bias;   /* host bf16 [N], or NULL */
+} svdq_w4a16_desc;
+
+/* Bytes of the device image (the caller allocates it, 256-byte aligned). 0 on a bad descriptor. */
+SVDQ_API size_t svdq_w4a16_device_bytes(const svdq_w4a16_desc* d);
+
+/* Host half: quantize W diag(s) into a new handle (no CUDA call). */
+SVDQ_API svdq_status svdq_w4a16_prepare_host(const svdq_w4a16_desc* d, svdq_w4a16** out);
+
+/* Device half: copy the image into dev_buf on `stream` and synchronize it. */
+SVDQ_API svdq_status svdq_w4a16_upload(svdq_w4a16* layer, void* dev_buf, size_t dev_buf_bytes, void* stream);
+
+/*
+ * Y = g (X diag(s)^-1) deq^T + b.  X: device bf16 [M, K] row-major, 16-byte
+ * aligned; Y: device bf16 [M, N] row-major, 2-byte aligned; any M >= 1 (rows
+ * go 4 at a time, one launch each, stream ordered).  No bounded waits: the
+ * kernel never waits on another CTA.
+ */
+SVDQ_API svdq_status svdq_w4a16_linear(const svdq_w4a16* layer, const void* X, int64_t M, void* Y, void* stream);
+
+/*
+ * Copy from the handle's host image: SVDQ_EXPORT_W_CODES uint8 [N, K/2] (E2M1,
+ * element 2i in the low nibble), SVDQ_EXPORT_W_SCALES uint8 [N, K/16] (E4M3),
+ * SVDQ_EXPORT_INV_LAMBDA float [K] (1/s), SVDQ_EXPORT_SCALARS float [1] (g).
+ */
+SVDQ_API svdq_status svdq_w4a16_export(const svdq_w4a16* layer, int what, void* host_dst, size_t bytes);
+
+/* Free the handle's host memory (the caller frees dev_buf). NULL is a no-op. */
+SVDQ_API void svdq_w4a16_destroy(svdq_w4a16* layer);
+
+/*
  * Test hooks.
  * svdq_test_override_device_arch: pretend the device reports this sm version
  * (e.g. 90) in the capability checks; 0 restores the real query.

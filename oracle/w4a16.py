@@ -40,8 +40,12 @@ class W4A16:
     deq: np.ndarray     # float64 [N, K] = e2m1 * e4m3 (without g)
 
 
-def prepare(W, s=None, bias=None):
-    """Quantize W [N, K] (float32 values of bf16 weights) as W' = f32(W diag(s))."""
+def prepare(W, s=None, bias=None, rows=None):
+    """Quantize W [N, K] (float32 values of bf16 weights) as W' = f32(W diag(s)).
+
+    ``rows`` keeps only those output rows (g still comes from all of W'), for
+    large layers checked on sampled outputs.
+    """
     W = np.asarray(W, np.float32)
     N, K = W.shape
     if K % 16:
@@ -49,11 +53,16 @@ def prepare(W, s=None, bias=None):
     s32 = np.ones(K, np.float32) if s is None else np.asarray(s, np.float32)
     if np.any(~(s32 > 0)) or not np.all(np.isfinite(s32)):
         raise ValueError("s must be positive and finite")
-    Wp = (W * s32[None, :]).astype(np.float32)
-    g = S.global_scale(np.max(np.abs(Wp)) if Wp.size else np.float32(0))
+    amax = np.float32(0)
+    for r0 in range(0, N, 4096):  # max |W'| in blocks of rows
+        blk = (W[r0:r0 + 4096] * s32[None, :]).astype(np.float32)
+        amax = max(amax, np.max(np.abs(blk)))
+    g = S.global_scale(amax)
+    sel = slice(None) if rows is None else rows
+    Wp = (W[sel] * s32[None, :]).astype(np.float32)
     codes, scales = S.nvfp4_quantize(Wp, g)
     inv_s = (np.float32(1.0) / s32).astype(np.float32)
-    b = None if bias is None else np.asarray(bias, np.float64)
+    b = None if bias is None else np.asarray(bias, np.float64)[sel]
     return W4A16(codes, scales, np.float32(g), inv_s, b, S.nvfp4_dequantize(codes, scales))
 
 
