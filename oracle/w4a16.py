@@ -17,9 +17,14 @@ Readings of what the pages leave open:
     tensor scale g = amax / 2688 (1 when amax is 0).
   * The activation-aware scale is one positive float32 s_j per input channel
     (1 when absent): the quantized weight is W' = f32(W diag(s)), and the
-    activations are divided by s at run time, x~_j = f32(x_j * f32(1 / s_j)),
-    so X W^T = X~ W'^T before quantization.  The pages give no rule for
-    choosing s (AWQ searches for it offline), so s is an input of the layer.
+    activations are divided by s at run time, so X W^T = X~ W'^T before
+    quantization.  The pages give no rule for choosing s (AWQ searches for it
+    offline), so s is an input of the layer.
+  * The divided activation is rounded once to a 16-bit operand, as X_hat is in
+    the W4A4 layer: x~_j = f16(f32(x_j * f32(1 / s_j))), to nearest, saturating
+    at +-65504.  f16 rather than bf16: the dequantized weights (E2M1 times
+    E4M3) are exact in f16, the two tensor-core operands share one type, and
+    f16 keeps 3 more bits of x~; its range covers the modulation inputs.
   * Y = g * sum_j x~_j deq(W')_nj + b, act = identity, rounded to bf16 once.
 """
 
@@ -66,12 +71,19 @@ def prepare(W, s=None, bias=None, rows=None):
     return W4A16(codes, scales, np.float32(g), inv_s, b, S.nvfp4_dequantize(codes, scales))
 
 
+def act_operand(X, inv_s):
+    """x~ = f16(f32(x * inv_s)), round to nearest even, saturating at the f16 maximum."""
+    t = (np.asarray(X, np.float32) * np.asarray(inv_s, np.float32)[None, :]).astype(np.float32)
+    t = np.clip(t, np.float32(-65504.0), np.float32(65504.0))
+    return t.astype(np.float16)
+
+
 def linear(layer, X, rows=None):
-    """Y = g * (X~ @ deq^T) + b in float64, X~ = f32(X * inv_s)."""
+    """Y = g * (X~ @ deq^T) + b in float64, X~ = act_operand(X, 1/s)."""
     X = np.asarray(X, np.float32)
     if rows is not None:
         X = X[rows]
-    Xt = (X * layer.inv_s[None, :]).astype(np.float32).astype(np.float64)
+    Xt = act_operand(X, layer.inv_s).astype(np.float64)
     y = np.float64(layer.g) * (Xt @ layer.deq.T)
     if layer.bias is not None:
         y = y + layer.bias[None, :]

@@ -16,6 +16,18 @@ def f32r(x):
     return struct.unpack("<f", struct.pack("<f", x))[0]
 
 
+def f16r(x):
+    """Round to the nearest IEEE half (ties to even, subnormals kept), saturating at 65504."""
+    if x == 0.0:
+        return x
+    a = min(abs(x), 65504.0)
+    m, e = math.frexp(a)              # a = m 2^e, m in [0.5, 1)
+    q = 2.0 ** max(e - 11, -24)       # 11 significant bits; subnormal quantum 2^-24
+    r = round(a / q) * q              # Python round: ties to even
+    r = min(r, 65504.0)
+    return math.copysign(r, x)
+
+
 def bf16r(x):
     """Round to 8 significant bits, ties to even (normal range)."""
     if x == 0.0:
@@ -168,7 +180,7 @@ def w4a16_forward(W, X, s, bias=None):
     inv = [f32r(1.0 / s[j]) for j in range(K)]
     Y = []
     for x in X:
-        xt = [f32r(x[j] * inv[j]) for j in range(K)]
+        xt = [f16r(f32r(x[j] * inv[j])) for j in range(K)]
         row = []
         for n in range(N):
             y = g * math.fsum(xt[j] * dw[n][j] for j in range(K))

@@ -22,9 +22,16 @@ def _grid_weights(N, K, seed, scale_pow=0):
     return (W * 448.0 * 2.0 ** scale_pow).astype(np.float32)
 
 
+def _f16_exact_x(M, K, seed):
+    # values exactly representable in f16 (and bf16): 8 significant bits, no tiny magnitudes
+    X = np.random.default_rng(seed).standard_normal((M, K)).astype(np.float32)
+    X = np.where(np.abs(X) < 1e-2, np.float32(0.0), X).astype(np.float16).astype(np.float32)
+    return (np.round(X * 64.0) / 64.0).astype(np.float32)
+
+
 def test_exact_weights_give_the_exact_product():
     W = _grid_weights(24, 64, seed=1, scale_pow=-12)
-    X = np.random.default_rng(2).standard_normal((5, 64)).astype(np.float32)
+    X = _f16_exact_x(5, 64, seed=2)
     L = W4.prepare(W)
     assert L.g == np.float32(2.0 ** -12)
     assert np.all(L.scales == F.e4m3_encode(np.float32(448.0)))
@@ -40,7 +47,7 @@ def test_power_of_two_channel_scales_cancel():
     s = (2.0 ** np.random.default_rng(3).integers(-3, 4, K)).astype(np.float32)
     Wp = _grid_weights(16, K, seed=4, scale_pow=-10)
     W = (Wp / s[None, :]).astype(np.float32)
-    X = np.random.default_rng(5).standard_normal((3, K)).astype(np.float32)
+    X = _f16_exact_x(3, K, seed=5)
     L = W4.prepare(W, s=s)
     np.testing.assert_array_equal(np.float64(L.g) * L.deq, Wp.astype(np.float64))
     np.testing.assert_allclose(W4.linear(L, X), X.astype(np.float64) @ W.T.astype(np.float64), rtol=1e-12,
@@ -76,6 +83,15 @@ def test_matches_brute_force(seed, with_s, with_bias):
     np.testing.assert_allclose(W4.linear(L, X), np.array(want["Y"]), rtol=1e-12, atol=1e-12)
 
 
+def test_activation_operand_rounds_to_f16_and_saturates():
+    x = np.array([[1.0, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 7e4, -1e6, 2.0 ** -25, 3 * 2.0 ** -25]],
+                 np.float32)
+    got = W4.act_operand(x, np.ones(x.shape[1], np.float32)).astype(np.float64)[0]
+    np.testing.assert_array_equal(got, [1.0, 1.0, 1.0 + 2.0 ** -9, 65504.0, -65504.0, 0.0, 2.0 ** -23])
+    for v in x[0]:  # the brute force's rounding agrees
+        assert BF.f16r(float(v)) == float(W4.act_operand(np.array([[v]], np.float32), np.ones(1, np.float32))[0, 0])
+
+
 def test_rejects_bad_scales_and_shapes():
     with pytest.raises(ValueError):
         W4.prepare(np.zeros((4, 20), np.float32))
@@ -98,17 +114,17 @@ def _pins_fail():
 
 
 def _linear_times_s(layer, X, rows=None):  # multiplies by s instead of dividing
-    Xt = (np.asarray(X, np.float32) / layer.inv_s[None, :]).astype(np.float32).astype(np.float64)
+    Xt = W4.act_operand(X, 1.0 / layer.inv_s).astype(np.float64)
     return np.float64(layer.g) * (Xt @ layer.deq.T) + (0 if layer.bias is None else layer.bias[None, :])
 
 
 def _linear_no_g(layer, X, rows=None):
-    Xt = (np.asarray(X, np.float32) * layer.inv_s[None, :]).astype(np.float32).astype(np.float64)
+    Xt = W4.act_operand(X, layer.inv_s).astype(np.float64)
     return Xt @ layer.deq.T + (0 if layer.bias is None else layer.bias[None, :])
 
 
 def _linear_no_bias(layer, X, rows=None):
-    Xt = (np.asarray(X, np.float32) * layer.inv_s[None, :]).astype(np.float32).astype(np.float64)
+    Xt = W4.act_operand(X, layer.inv_s).astype(np.float64)
     return np.float64(layer.g) * (Xt @ layer.deq.T)
 
 
