@@ -388,7 +388,7 @@ svdq_status svdq_w4a16_prepare_host(const svdq_w4a16_desc* d, svdq_w4a16** out) 
   std::string err;
   auto* L = new (std::nothrow) svdq_w4a16();
   if (!L) return fail(SVDQ_ERR_INTERNAL, "out of host memory");
-  svdq_status st = svdq::w4a16_quantize(d, &L->image, &L->gscale, &err);
+  svdq_status st = svdq::w4a16_quantize(d, &L->image, &L->codes, &L->scales, &L->gscale, &err);
   if (st != SVDQ_OK) {
     delete L;
     return fail(st, err);
@@ -448,8 +448,8 @@ svdq_status svdq_w4a16_export(const svdq_w4a16* L, int what, void* host_dst, siz
   const void* src = nullptr;
   size_t n = 0;
   switch (what) {
-    case SVDQ_EXPORT_W_CODES: src = img + g.off_codes; n = size_t(g.N) * size_t(g.K / 2); break;
-    case SVDQ_EXPORT_W_SCALES: src = img + g.off_scales; n = size_t(g.N) * size_t(g.K / 16); break;
+    case SVDQ_EXPORT_W_CODES: src = L->codes.data(); n = L->codes.size(); break;
+    case SVDQ_EXPORT_W_SCALES: src = L->scales.data(); n = L->scales.size(); break;
     case SVDQ_EXPORT_INV_LAMBDA: src = img + g.off_inv_s; n = size_t(g.K) * 4; break;
     case SVDQ_EXPORT_SCALARS: src = &L->gscale; n = 4; break;
     default: return fail(SVDQ_ERR_INVALID_ARGUMENT, "unknown export for a W4A16 layer");

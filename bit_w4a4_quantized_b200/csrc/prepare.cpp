@@ -331,7 +331,8 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
 
 // W4A16: W' = f32(W diag(s)) quantized row by row with the same NVFP4 quantizer
 // as the W4A4 residual, under the tensor scale g = max|W'| / 2688.
-svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image, float* g_out, std::string* err) {
+svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image, std::vector<uint8_t>* codes,
+                           std::vector<uint8_t>* scales, float* g_out, std::string* err) {
   if (!d || !d->W) {
     *err = "descriptor and W are required";
     return SVDQ_ERR_INVALID_ARGUMENT;
@@ -361,19 +362,42 @@ svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image
     }
   const float g = global_scale(amax);
   const float c = 1.0f / (6.0f * g);
+  codes->assign(size_t(N) * size_t(K / 2), 0);
+  scales->assign(size_t(N) * size_t(K / 16), 0);
+  uint8_t* cr = codes->data();
+  uint8_t* sr = scales->data();
+  const int threads = int(std::max(1u, std::min(16u, std::thread::hardware_concurrency())));
+  parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
+    for (int64_t n = n0; n < n1; ++n)
+      quantize_row(&wp[size_t(n) * K], K, g, c,
+                   [&](int64_t k, uint8_t byte) { cr[size_t(n) * size_t(K / 2) + size_t(k / 2)] = byte; },
+                   [&](int64_t sb, uint8_t code) { sr[size_t(n) * size_t(K / 16) + size_t(sb)] = code; });
+  });
+  // the device image: tiles of 16 rows x 64 inputs in fragment order
   const W4A16Geom geo = make_w4a16_geom(K, N);
   image->assign(geo.total, 0);
   uint8_t* img = image->data();
   float* inv = reinterpret_cast<float*>(img + geo.off_inv_s);
   for (int64_t k = 0; k < K; ++k) inv[k] = 1.0f / s[size_t(k)];
   if (d->bias) std::memcpy(img + geo.off_bias, d->bias, sizeof(uint16_t) * size_t(N));
-  const int threads = int(std::max(1u, std::min(16u, std::thread::hardware_concurrency())));
-  parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
-    for (int64_t n = n0; n < n1; ++n)
-      quantize_row(&wp[size_t(n) * K], K, g, c,
-                   [&](int64_t k, uint8_t byte) { img[geo.off_codes + size_t(n) * size_t(K / 2) + size_t(k / 2)] = byte; },
-                   [&](int64_t sb, uint8_t code) { img[geo.off_scales + size_t(n) * size_t(K / 16) + size_t(sb)] = code; });
-  });
+  for (int64_t nt = 0; nt < geo.N16 / 16; ++nt)
+    for (int64_t kt = 0; kt < geo.KT; ++kt) {
+      uint8_t* ct = img + geo.off_codes + size_t(nt * geo.KT + kt) * 512;
+      uint8_t* st = img + geo.off_scales + size_t(nt * geo.KT + kt) * 64;
+      for (int t = 0; t < 32; ++t)
+        for (int j = 0; j < 4; ++j)
+          for (int q = 0; q < 4; ++q) {
+            const int64_t row = nt * 16 + (t >> 2) + 8 * (q & 1);
+            const int64_t k = kt * 64 + 16 * j + 2 * (t & 3) + 8 * (q >> 1);
+            ct[t * 16 + j * 4 + q] = row < N ? cr[size_t(row) * size_t(K / 2) + size_t(k / 2)] : 0;
+          }
+      for (int gi = 0; gi < 8; ++gi)
+        for (int h = 0; h < 2; ++h)
+          for (int j = 0; j < 4; ++j) {
+            const int64_t row = nt * 16 + gi + 8 * h;
+            st[gi * 8 + h * 4 + j] = row < N ? sr[size_t(row) * size_t(K / 16) + size_t(kt * 4 + j)] : 0;
+          }
+    }
   *g_out = g;
   return SVDQ_OK;
 }

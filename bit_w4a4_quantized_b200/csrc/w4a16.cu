@@ -1,20 +1,22 @@
-// w4a16.cu -- the W4A16 layer's kernel: Y = g (X diag(s)^-1) deq(W')^T + b with
-// 4-bit NVFP4 weights and bf16 activations, for the small batches of the
+// w4a16.cu -- the W4A16 layer's kernel: Y = g x~ deq(W')^T + b with 4-bit NVFP4
+// weights W' = W diag(s) and x~ = f16(x / s), for the small batches of the
 // modulation projections (Diffusers/Nunchaku page: awq_w4a16, memory bound).
 //
-// Design (sm_100a): the kernel streams the weights once, so its roofline is
-// HBM bandwidth.  A warp streams 4 weight rows at a time (2 when X has 3 or 4
-// rows) and issues all of their loads for a 1024-weight step before any
-// arithmetic: per step a lane reads 16 bytes of codes (32 weights) and their 2
-// block scales of each row, so a warp reads 512 contiguous bytes per row.
-// Every CTA keeps x~ = f32(x / s) for its rows of X in shared memory (16-byte
-// chunks swizzled so the lanes' reads hit distinct banks); each x~ value a lane
-// reads serves all the rows in flight, which keeps shared-memory traffic below
-// the weight stream.  The E2M1 codes and
-// E4M3 scales are decoded with the hardware f16x2 conversions (exact: every
-// code times scale is an f16 value); the sums are float32, even and odd
-// weights apart, one partial per 16-weight block, multiplied by the block
-// scale.
+// Design (sm_100a): the kernel streams the 4-bit weights once, so its roofline
+// is HBM bandwidth; the arithmetic only has to stay out of the way.  It runs on
+// the tensor cores with the warp-level m16n8k16 MMA (f16 operands, float32
+// accumulators): A = 16 weight rows x 16 inputs, dequantized in registers (the
+// hardware E2M1 -> f16x2 conversion, times the E4M3 block scale: exact in f16),
+// B = 16 inputs x 8 rows of X (x~ in shared memory; rows past M are zero
+// operands in registers).  The
+// prepared image stores each 16 x 64 weight tile in fragment order, so one
+// 16-byte load per lane brings the A operands of four MMAs.  A CTA of 8 warps
+// takes a 16-row tile of the output; its warps split K (tile kt goes to warp
+// kt % 8), issue all their weight loads before any arithmetic, and add their
+// partial sums through shared memory in a fixed order.  With one row of X the
+// MMA would be 7/8 padding, so that launch does the same tiles on the CUDA
+// cores instead: mixed-precision fused multiply-adds (f16 operands, float32
+// accumulator) straight from the f16 weights, no conversion to float32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -29,250 +31,302 @@ W4A16Geom make_w4a16_geom(int64_t K, int64_t N) {
   W4A16Geom g{};
   g.K = K;
   g.N = N;
+  g.N16 = (N + 15) / 16 * 16;
+  g.KT = K / 64;
   size_t o = kStatusBytes;
   g.off_inv_s = o;
   o = align256(o + size_t(K) * 4);
   g.off_bias = o;
   o = align256(o + size_t(N) * 2);
   g.off_codes = o;
-  o = align256(o + size_t(N) * size_t(K / 2));
+  o = align256(o + size_t(g.N16) * size_t(K / 2));
   g.off_scales = o;
-  o = align256(o + size_t(N) * size_t(K / 16));
+  o = align256(o + size_t(g.N16) * size_t(K / 16));
   g.total = o;
   return g;
 }
 
 namespace {
 
-constexpr int kThreadsW = 256;  // 8 warps (128 measured slower)
-constexpr int kMaxMW = 4;       // rows of X per launch
+constexpr int kThreadsW = 256;  // 8 warps
+constexpr int kWarpsW = kThreadsW / 32;
+constexpr int kMaxMW = 8;  // rows of X per launch: the MMA's N
+constexpr int kTilesPerWarp = 6;  // weight tiles whose loads a warp issues together (K = 3072: all of them)
 
 struct W4A16Params {
-  const uint8_t* codes;
-  const uint8_t* scales;
+  const uint4* codes;   // [N16 / 16][KT][32 lanes] x 16 bytes
+  const uint2* scales;  // [N16 / 16][KT][8 groups] x 8 bytes
   const float* inv_s;
   const uint16_t* bias;  // or null
   const uint16_t* X;
   uint16_t* Y;
-  int64_t K, N, M;
+  int64_t K, N, M, NT, KT;
   float g;
 };
 
-// Physical 16-byte chunk of logical chunk c of an x~ row: the 3 low bits are
-// XORed with bits 3..5, so the 8 lanes of a quarter-warp, whose chunks are 8
-// apart, read 8 different bank groups.
-__device__ __forceinline__ uint32_t xswz(uint32_t c) { return c ^ ((c >> 3) & 7u); }
-
-__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& h0, uint32_t& h1, uint32_t& h2, uint32_t& h3) {
+// Four code bytes (8 E2M1 codes, each byte's first in its low nibble) -> four
+// f16x2, byte i in h[i], its first code in the low half.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t* h) {
   asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n"
       " cvt.rn.f16x2.e2m1x2 %0, b0;\n cvt.rn.f16x2.e2m1x2 %1, b1;\n"
       " cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
       : "r"(w));
 }
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t s) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(s));
-  return h;
+// Four E4M3 scales (one word) -> two f16x2: {s0, s1} and {s2, s3}.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n cvt.rn.f16x2.e4m3x2 %1, h;\n}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
-__device__ __forceinline__ float2 f16x2_to_f32(uint32_t h) {
-  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+// The low (j = 0) or high (j = 1) half of an f16x2, in both halves.
+__device__ __forceinline__ uint32_t dup_half(uint32_t v, int j) { return __byte_perm(v, 0u, j ? 0x3232u : 0x1010u); }
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
-// The even and odd weights of a pair accumulate separately: (a.x b.x + c.x, a.y b.y + c.y).
-// (The packed f32x2 fused multiply-add measured the same time as two scalar ones.)
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+// D = A B + D, m16n8k16, f16 operands, float32 accumulators.
+__device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Weight rows a warp streams at once: every x~ value read from shared memory
-// serves all of them, so the shared-memory traffic per weight is 4 kM / kR bytes.
+// One 16 x 64 weight tile against x~: 4 MMAs.  cw: this lane's 16 code bytes;
+// sw: the 8 scale bytes of its rows g (x) and g + 8 (y); xrow: x~ row g as
+// f16 pairs, at the tile's first input, or null when row g of X is past M.
+__device__ __forceinline__ void tile_mma(float* acc, uint4 cw, uint2 sw, const uint32_t* xrow, int c) {
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+  uint32_t sg[2], sg8[2];  // scales of rows g and g + 8: steps {0, 1}, {2, 3}
+  e4m3x4_to_f16x2(sw.x, sg[0], sg[1]);
+  e4m3x4_to_f16x2(sw.y, sg8[0], sg8[1]);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t h[4];
+    e2m1x8_to_f16x2(words[j], h);
+    const uint32_t s0 = dup_half(sg[j >> 1], j & 1);   // row g
+    const uint32_t s1 = dup_half(sg8[j >> 1], j & 1);  // row g + 8
+    const uint32_t a0 = hmul2(h[0], s0);
+    const uint32_t a1 = hmul2(h[1], s1);
+    const uint32_t a2 = hmul2(h[2], s0);
+    const uint32_t a3 = hmul2(h[3], s1);
+    const uint32_t b0 = xrow ? xrow[8 * j + c] : 0u;      // inputs 16 j + 2 c, + 1
+    const uint32_t b1 = xrow ? xrow[8 * j + c + 4] : 0u;  // inputs 16 j + 2 c + 8, + 9
+    mma_16816(acc, a0, a1, a2, a3, b0, b1);
+  }
+}
+
+// acc + x.lo w.lo + x.hi w.hi with f16 operands and a float32 accumulator
+// (exact products, float32 sums).
+__device__ __forceinline__ float fma2_f16_f32(uint32_t x2, uint32_t w2, float acc) {
+  asm("{\n .reg .f16 xl, xh, wl, wh;\n mov.b32 {xl, xh}, %1;\n mov.b32 {wl, wh}, %2;\n"
+      " fma.rn.f32.f16 %0, xl, wl, %0;\n fma.rn.f32.f16 %0, xh, wh, %0;\n}"
+      : "+f"(acc)
+      : "r"(x2), "r"(w2));
+  return acc;
+}
+
+// The same 16 x 64 tile on the CUDA cores, for kM <= 2 rows of X (the MMA's 8
+// columns would be mostly padding): lane (g, c) adds its 16 weights of rows g
+// (acc[0][m]) and g + 8 (acc[1][m]) times x~; xs: x~ rows as f16 pairs, at the
+// tile's first input.
 template <int kM>
-__host__ __device__ constexpr int rows_in_flight() {
-  return kM <= 2 ? 4 : 2;
-}
-
-// 1024-weight steps per lane whose loads are issued together.  More (3 cover
-// K = 3072) was measured slower: the registers cost more occupancy than the
-// extra loads in flight bought.
-constexpr int kJ = 1;
-
-// One 32-weight step of every row in flight: x~[m][c0 * 4 .. + 31] against
-// the 16 code bytes cw[r] and 2 block scales sw[r] of row r; each x~ chunk read
-// from shared memory serves all kR rows.
-template <int kM, int kR>
-__device__ __forceinline__ void step32(const float4* xs4, uint32_t KC, uint32_t c0, const uint4* cw,
-                                       const uint16_t* sw, float2 (*acc)[kM]) {
+__device__ __forceinline__ void tile_dot(float (*acc)[kM], uint4 cw, uint2 sw, const uint32_t* xs, uint32_t RW,
+                                         int c) {
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+  uint32_t sg[2], sg8[2];  // scales of rows g and g + 8: steps {0, 1}, {2, 3}
+  e4m3x4_to_f16x2(sw.x, sg[0], sg[1]);
+  e4m3x4_to_f16x2(sw.y, sg8[0], sg8[1]);
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {  // two 16-weight blocks
-    float2 part[kR][kM];
+  for (int j = 0; j < 4; ++j) {
+    uint32_t h[4];
+    e2m1x8_to_f16x2(words[j], h);
+    const uint32_t s0 = dup_half(sg[j >> 1], j & 1);   // row g
+    const uint32_t s1 = dup_half(sg8[j >> 1], j & 1);  // row g + 8
+    const uint32_t a0 = hmul2(h[0], s0);  // row g, inputs 16 j + 2 c, + 1
+    const uint32_t a1 = hmul2(h[1], s1);  // row g + 8, the same inputs
+    const uint32_t a2 = hmul2(h[2], s0);  // row g, inputs 16 j + 2 c + 8, + 9
+    const uint32_t a3 = hmul2(h[3], s1);  // row g + 8, the same inputs
 #pragma unroll
-    for (int r = 0; r < kR; ++r)
-#pragma unroll
-      for (int m = 0; m < kM; ++m) part[r][m] = make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int wi = 0; wi < 2; ++wi) {  // 8 weights per code word
-      const uint32_t c = c0 + uint32_t(4 * half + 2 * wi);
-      float4 xa[kM], xb[kM];
-#pragma unroll
-      for (int m = 0; m < kM; ++m) {
-        xa[m] = xs4[m * KC + xswz(c)];
-        xb[m] = xs4[m * KC + xswz(c + 1)];
-      }
-#pragma unroll
-      for (int r = 0; r < kR; ++r) {
-        const uint32_t word = half ? (wi ? cw[r].w : cw[r].z) : (wi ? cw[r].y : cw[r].x);
-        uint32_t h[4];
-        e2m1x8_to_f16x2(word, h[0], h[1], h[2], h[3]);
-        const float2 w0 = f16x2_to_f32(h[0]), w1 = f16x2_to_f32(h[1]);
-        const float2 w2 = f16x2_to_f32(h[2]), w3 = f16x2_to_f32(h[3]);
-#pragma unroll
-        for (int m = 0; m < kM; ++m) {
-          part[r][m] = ffma2(make_float2(xa[m].x, xa[m].y), w0, part[r][m]);
-          part[r][m] = ffma2(make_float2(xa[m].z, xa[m].w), w1, part[r][m]);
-          part[r][m] = ffma2(make_float2(xb[m].x, xb[m].y), w2, part[r][m]);
-          part[r][m] = ffma2(make_float2(xb[m].z, xb[m].w), w3, part[r][m]);
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      const float2 sc = f16x2_to_f32(e4m3x2_to_f16x2(sw[r]));
-      const float sv = half ? sc.y : sc.x;
-#pragma unroll
-      for (int m = 0; m < kM; ++m) acc[r][m] = ffma2(part[r][m], make_float2(sv, sv), acc[r][m]);
+    for (int m = 0; m < kM; ++m) {
+      const uint32_t x0 = xs[m * RW + 8 * j + c], x1 = xs[m * RW + 8 * j + c + 4];
+      acc[0][m] = fma2_f16_f32(x1, a2, fma2_f16_f32(x0, a0, acc[0][m]));
+      acc[1][m] = fma2_f16_f32(x1, a3, fma2_f16_f32(x0, a1, acc[1][m]));
     }
   }
 }
 
-template <int kM>
+// kDot = 0: the MMA path (2 to 8 rows of X); kDot = 1: the CUDA-core path for one row.
+template <int kDot>
 __global__ void __launch_bounds__(kThreadsW) w4a16_kernel(const W4A16Params p) {
-  constexpr int kR = rows_in_flight<kM>();
-  extern __shared__ float4 xs4[];  // [kM][K / 4] chunks of x~, swizzled
+  extern __shared__ uint32_t smem_w[];
   const int64_t K = p.K;
-  const uint32_t KC = uint32_t(K / 4);
-  // x~ = f32(x * (1 / s)) for this launch's rows
-  for (uint32_t i = threadIdx.x; i < uint32_t(kM) * KC; i += kThreadsW) {
-    const uint32_t m = i / KC, c = i % KC;
-    const uint2 xb = *reinterpret_cast<const uint2*>(p.X + int64_t(m) * K + int64_t(c) * 4);
-    const float4 is = *reinterpret_cast<const float4*>(p.inv_s + int64_t(c) * 4);
-    float4 v;
-    v.x = __uint_as_float(xb.x << 16) * is.x;
-    v.y = __uint_as_float(xb.x & 0xFFFF0000u) * is.y;
-    v.z = __uint_as_float(xb.y << 16) * is.z;
-    v.w = __uint_as_float(xb.y & 0xFFFF0000u) * is.w;
-    xs4[m * KC + xswz(c)] = v;
+  const uint32_t RW = uint32_t(K / 2) + 4;  // x~ row stride in f16 pairs (+4: rows start on different banks)
+  const uint32_t MR = uint32_t(p.M);        // rows of x~ kept (B columns past M are zero in registers)
+  uint32_t* xs = smem_w;                    // [M][RW] f16 pairs
+  float* red = reinterpret_cast<float*>(smem_w + MR * RW);  // [8 warps][32 lanes][4]
+  const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
+  const int g = lane >> 2, c = lane & 3;
+
+  // the first tile's weight loads go out before x~ is staged
+  int64_t nt = blockIdx.x;
+  uint4 cw[kTilesPerWarp];
+  uint2 sw[kTilesPerWarp];
+  auto load = [&](int64_t tile, int64_t kt0) {
+#pragma unroll
+    for (int i = 0; i < kTilesPerWarp; ++i) {
+      const int64_t kt = kt0 + int64_t(i) * kWarpsW;
+      if (tile < p.NT && kt < p.KT) {
+        cw[i] = __ldg(p.codes + (tile * p.KT + kt) * 32 + lane);
+        sw[i] = __ldg(p.scales + (tile * p.KT + kt) * 8 + g);
+      } else {
+        cw[i] = make_uint4(0u, 0u, 0u, 0u);
+        sw[i] = make_uint2(0u, 0u);
+      }
+    }
+  };
+  load(nt, warp);
+
+  // x~ = f16(x / s), saturating
+  for (uint32_t i = threadIdx.x; i < MR * uint32_t(K / 2); i += kThreadsW) {
+    const uint32_t m = i / uint32_t(K / 2), w = i % uint32_t(K / 2);
+    const uint32_t xb = *reinterpret_cast<const uint32_t*>(p.X + int64_t(m) * K + 2 * int64_t(w));
+    const float2 is = *reinterpret_cast<const float2*>(p.inv_s + 2 * int64_t(w));
+    const float lo = fminf(fmaxf(__uint_as_float(xb << 16) * is.x, -65504.0f), 65504.0f);
+    const float hi = fminf(fmaxf(__uint_as_float(xb & 0xFFFF0000u) * is.y, -65504.0f), 65504.0f);
+    const __half2 h = __floats2half2_rn(lo, hi);
+    xs[m * RW + w] = *reinterpret_cast<const uint32_t*>(&h);
   }
   __syncthreads();
 
-  const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
-  const int64_t nwarps = int64_t(gridDim.x) * (kThreadsW / 32);
-  const int64_t row_bytes = K / 2, srow_bytes = K / 16;
-  for (int64_t n0 = int64_t(blockIdx.x) * (kThreadsW / 32) + warp; n0 < p.N; n0 += kR * nwarps) {
-    float2 acc[kR][kM];
+  for (; nt < p.NT; nt += gridDim.x) {
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float dacc[2][kDot > 0 ? kDot : 1] = {};
+    const uint32_t* xrow = uint32_t(g) < MR ? xs + uint32_t(g) * RW : nullptr;
+    for (int64_t kt0 = warp;; kt0 += int64_t(kTilesPerWarp) * kWarpsW) {
 #pragma unroll
-    for (int r = 0; r < kR; ++r)
-#pragma unroll
-      for (int m = 0; m < kM; ++m) acc[r][m] = make_float2(0.0f, 0.0f);
-    // lane l covers weights l * 32 .. + 31 of every 1024 along K; the loads of
-    // kJ such steps for all kR rows are in flight before the arithmetic
-    for (int64_t kb = 0; kb < K; kb += kJ * 1024) {
-      uint4 cw[kJ][kR];
-      uint16_t sw[kJ][kR];
-#pragma unroll
-      for (int j = 0; j < kJ; ++j)
-#pragma unroll
-        for (int r = 0; r < kR; ++r) {
-          const int64_t n = n0 + r * nwarps, k0 = kb + j * 1024 + lane * 32;
-          cw[j][r] = make_uint4(0u, 0u, 0u, 0u);
-          sw[j][r] = 0;
-          if (n < p.N && k0 < K) {
-            cw[j][r] = __ldg(reinterpret_cast<const uint4*>(p.codes + n * row_bytes + k0 / 2));
-            sw[j][r] = __ldg(reinterpret_cast<const uint16_t*>(p.scales + n * srow_bytes + k0 / 16));
-          }
+      for (int i = 0; i < kTilesPerWarp; ++i) {
+        const int64_t kt = kt0 + int64_t(i) * kWarpsW;
+        if (kt < p.KT) {
+          if constexpr (kDot > 0)
+            tile_dot<kDot>(dacc, cw[i], sw[i], xs + uint32_t(kt) * 32u, RW, c);
+          else
+            tile_mma(acc, cw[i], sw[i], xrow ? xrow + uint32_t(kt) * 32u : nullptr, c);
         }
-#pragma unroll
-      for (int j = 0; j < kJ; ++j) {
-        const int64_t k0 = kb + j * 1024 + lane * 32;
-        if (k0 < K) step32<kM, kR>(xs4, KC, uint32_t(k0 / 4), cw[j], sw[j], acc);
+      }
+      const int64_t next = kt0 + int64_t(kTilesPerWarp) * kWarpsW;
+      if (next < p.KT) {
+        load(nt, next);  // more of this row tile (K > 3072)
+      } else {
+        load(nt + gridDim.x, warp);  // the next row tile's first loads overlap the reduction
+        break;
       }
     }
+    if constexpr (kDot > 0) {
+      // the 4 lanes of a row group hold disjoint inputs: add them (lane c = 0 keeps the sums), then lay
+      // the result out as the MMA accumulator would hold it: lane (g, c) row g (x, y), row g + 8 (z, w),
+      // X rows 2 c, 2 c + 1
 #pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      const int64_t n = n0 + r * nwarps;
-      float y[kM];
+      for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int m = 0; m < kM; ++m) {
-        y[m] = acc[r][m].x + acc[r][m].y;
+        for (int m = 0; m < kDot; ++m) {
+          dacc[h][m] += __shfl_xor_sync(0xFFFFFFFFu, dacc[h][m], 1);
+          dacc[h][m] += __shfl_xor_sync(0xFFFFFFFFu, dacc[h][m], 2);
+        }
+      acc[0] = c == 0 ? dacc[0][0] : 0.0f;
+      acc[2] = c == 0 ? dacc[1][0] : 0.0f;
+      acc[1] = (c == 0 && kDot > 1) ? dacc[0][kDot > 1 ? 1 : 0] : 0.0f;
+      acc[3] = (c == 0 && kDot > 1) ? dacc[1][kDot > 1 ? 1 : 0] : 0.0f;
+    }
+    // the 8 warps' partial tiles, added in warp order
+    *reinterpret_cast<float4*>(red + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    if (warp == 0) {
+      float4 t = *reinterpret_cast<const float4*>(red + lane * 4);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) y[m] += __shfl_xor_sync(0xFFFFFFFFu, y[m], o);
+      for (int w = 1; w < kWarpsW; ++w) {
+        const float4 u = *reinterpret_cast<const float4*>(red + (w * 32 + lane) * 4);
+        t.x += u.x;
+        t.y += u.y;
+        t.z += u.z;
+        t.w += u.w;
       }
-      if (n < p.N && lane < kM) {
-        float a = y[0];
+      // lane (g, c): rows n = 16 nt + g (x, y) and + 8 (z, w); X rows m = 2 c (x, z) and 2 c + 1 (y, w)
+      const float v[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-        for (int m = 1; m < kM; ++m)
-          if (lane == m) a = y[m];
-        const float b = p.bias ? __uint_as_float(uint32_t(p.bias[n]) << 16) : 0.0f;
-        const __nv_bfloat16 out = __float2bfloat16_rn(fmaf(p.g, a, b));
-        p.Y[int64_t(lane) * p.N + n] = *reinterpret_cast<const uint16_t*>(&out);
+      for (int q = 0; q < 4; ++q) {
+        const int64_t n = nt * 16 + g + 8 * (q >> 1);
+        const int64_t m = 2 * c + (q & 1);
+        if (n < p.N && m < p.M) {
+          const float b = p.bias ? __uint_as_float(uint32_t(p.bias[n]) << 16) : 0.0f;
+          const __nv_bfloat16 y = __float2bfloat16_rn(fmaf(p.g, v[q], b));
+          p.Y[m * p.N + n] = *reinterpret_cast<const uint16_t*>(&y);
+        }
       }
     }
+    __syncthreads();  // red is rewritten by the next row tile
   }
 }
 
-// Blocks per SM for this instance, device and K, queried once (the attribute
-// and occupancy calls cost microseconds of host time; a launch should not).
-template <int kM>
-int blocks_per_sm(int64_t K, size_t smem) {
+// Blocks per SM for this device and shared-memory size, queried once (the
+// attribute and occupancy calls cost microseconds of host time; a launch
+// should not).  The carveout asks for all of the unified L1 as shared memory,
+// or the driver may size it for one CTA.
+template <int kDot>
+int blocks_per_sm(size_t smem) {
   static std::atomic<int64_t> cached_key[64];
   static std::atomic<int> cached_val[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  const int64_t key = K + 1;
+  const int64_t key = int64_t(smem) + 1;
   if (cached_key[dev & 63].load() == key) return cached_val[dev & 63].load();
-  if (cudaFuncSetAttribute(w4a16_kernel<kM>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+  if (cudaFuncSetAttribute(w4a16_kernel<kDot>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(w4a16_kernel<kDot>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
     return 0;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, w4a16_kernel<kM>, kThreadsW, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, w4a16_kernel<kDot>, kThreadsW, smem) != cudaSuccess)
     return 0;
   cached_val[dev & 63].store(per_sm);
   cached_key[dev & 63].store(key);
   return per_sm;
 }
 
-template <int kM>
-cudaError_t launch_m(const W4A16Params& p, int num_sms, cudaStream_t s) {
-  const size_t smem = size_t(kM) * size_t(p.K) * 4;
-  const int per_sm = blocks_per_sm<kM>(p.K, smem);
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  const int64_t rows_per_cta = (kThreadsW / 32) * rows_in_flight<kM>();
-  int64_t blocks = int64_t(per_sm) * num_sms;
-  const int64_t need = (p.N + rows_per_cta - 1) / rows_per_cta;
-  if (blocks > need) blocks = need;
-  w4a16_kernel<kM><<<unsigned(blocks), kThreadsW, smem, s>>>(p);
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 cudaError_t launch_w4a16(const W4A16Launch& a, cudaStream_t s, const char** why) {
   W4A16Params p{};
-  p.codes = a.layer + a.g.off_codes;
-  p.scales = a.layer + a.g.off_scales;
+  p.codes = reinterpret_cast<const uint4*>(a.layer + a.g.off_codes);
+  p.scales = reinterpret_cast<const uint2*>(a.layer + a.g.off_scales);
   p.inv_s = reinterpret_cast<const float*>(a.layer + a.g.off_inv_s);
   p.bias = a.has_bias ? reinterpret_cast<const uint16_t*>(a.layer + a.g.off_bias) : nullptr;
   p.K = a.g.K;
   p.N = a.g.N;
+  p.NT = a.g.N16 / 16;
+  p.KT = a.g.KT;
   p.g = a.gscale;
-  // rows of X in launches of at most kMaxMW, stream ordered
+  // rows of X in launches of at most 8 (the MMA's N), stream ordered
   for (int64_t m0 = 0; m0 < a.M; m0 += kMaxMW) {
-    const int64_t mc = a.M - m0 < kMaxMW ? a.M - m0 : kMaxMW;
     p.X = a.X + m0 * a.g.K;
     p.Y = a.Y + m0 * a.g.N;
-    p.M = mc;
-    cudaError_t e = mc == 1   ? launch_m<1>(p, a.num_sms, s)
-                    : mc == 2 ? launch_m<2>(p, a.num_sms, s)
-                    : mc == 3 ? launch_m<3>(p, a.num_sms, s)
-                              : launch_m<4>(p, a.num_sms, s);
+    p.M = a.M - m0 < kMaxMW ? a.M - m0 : kMaxMW;
+    const size_t smem = (size_t(p.M) * size_t(a.g.K / 2 + 4) + size_t(kThreadsW) * 4) * 4;
+    const int per_sm = p.M == 1 ? blocks_per_sm<1>(smem) : blocks_per_sm<0>(smem);
+    if (per_sm < 1) {
+      *why = "the W4A16 kernel does not fit on this device";
+      return cudaErrorInvalidConfiguration;
+    }
+    int64_t blocks = int64_t(per_sm) * a.num_sms;
+    if (blocks > p.NT) blocks = p.NT;
+    if (p.M == 1)  // one row of X: the CUDA cores (measured 15 us against 18 us for the MMA at M = 1..4)
+      w4a16_kernel<1><<<unsigned(blocks), kThreadsW, smem, s>>>(p);
+    else
+      w4a16_kernel<0><<<unsigned(blocks), kThreadsW, smem, s>>>(p);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       *why = "launch of the W4A16 kernel failed";
       return e;

@@ -15,10 +15,18 @@
 namespace svdq {
 
 // Device image of one W4A16 layer (one caller buffer, 256-byte aligned sections):
-//   status word | 1/s float [K] | bias bf16 [N] | codes [N][K/2] | scales [N][K/16]
-// Codes: E2M1, element 2i in the low nibble of byte i of its row.  Scales: E4M3.
+//   status word | 1/s float [K] | bias bf16 [N] | codes | scales
+// The weights are cut into tiles of 16 rows x 64 inputs, stored tile after tile
+// (row tile major), each in the order the tensor-core fragments want them:
+//   codes: 512 bytes per tile = 32 lanes x 16 bytes; lane t = 4 g + c holds,
+//     for the tile's four 16-input steps j, the 4 bytes (rows g, g + 8 at
+//     inputs 16 j + 2 c, then rows g, g + 8 at 16 j + 2 c + 8), two E2M1
+//     codes per byte, the lower input in the low nibble;
+//   scales: 64 bytes per tile = 8 groups g x 8 bytes: the E4M3 scales of rows
+//     g (steps 0..3), then g + 8 (steps 0..3).
+// Rows past N are zero.
 struct W4A16Geom {
-  int64_t K, N;
+  int64_t K, N, N16, KT;  // N16 = N rounded up to 16; KT = K / 64
   size_t off_inv_s, off_bias, off_codes, off_scales, total;
 };
 W4A16Geom make_w4a16_geom(int64_t K, int64_t N);
@@ -35,14 +43,18 @@ struct W4A16Launch {
 };
 cudaError_t launch_w4a16(const W4A16Launch& a, cudaStream_t s, const char** why);
 
-// Host quantization: fills `image` (host copy of the device image) and *g.
-svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image, float* g, std::string* err);
+// Host quantization: fills `image` (host copy of the device image), the
+// row-major codes [N][K/2] and scales [N][K/16] (for exports) and *g.
+svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image, std::vector<uint8_t>* codes,
+                           std::vector<uint8_t>* scales, float* g, std::string* err);
 
 }  // namespace svdq
 
 struct svdq_w4a16 {
   svdq::W4A16Geom g;
   std::vector<uint8_t> image;  // host copy of the device image
+  std::vector<uint8_t> codes;  // row-major [N][K/2], for exports
+  std::vector<uint8_t> scales;  // row-major [N][K/16], for exports
   float gscale = 1.0f;
   bool has_bias = false;
   void* dev_buf = nullptr;
