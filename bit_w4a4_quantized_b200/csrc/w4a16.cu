@@ -161,8 +161,11 @@ __device__ __forceinline__ void tile_dot(float (*acc)[kM], uint4 cw, uint2 sw, c
 }
 
 // kDot = 0: the MMA path (2 to 8 rows of X); kDot = 1: the CUDA-core path for one row.
+// The one-row instance fits 64 registers, so 4 CTAs share an SM (measured 15.2 -> 14.6 us at K = 3072,
+// N = 18432).  The MMA instance is faster with room for 106 registers and 2 CTAs per SM (M = 4:
+// 18.7 -> 17.3 us) than held to 80 registers and 3.
 template <int kDot>
-__global__ void __launch_bounds__(kThreadsW) w4a16_kernel(const W4A16Params p) {
+__global__ void __launch_bounds__(kThreadsW, kDot ? 4 : 1) w4a16_kernel(const W4A16Params p) {
   extern __shared__ uint32_t smem_w[];
   const int64_t K = p.K;
   const uint32_t RW = uint32_t(K / 2) + 4;  // x~ row stride in f16 pairs (+4: rows start on different banks)
