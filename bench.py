@@ -627,7 +627,6 @@ def w4a16_point(spec, device, steps):
     to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.uint16).astype(np.int16)).view(
         torch.bfloat16).to(device)
     W, s, b = spec.w(), spec.s(), spec.b()
-    base = svdq.W4A16Layer(W, s=s, bias=b)
     wbytes = N * K // 2 + N * K // 16
     nsets = int(min(8, max(2, math.ceil(3 * L2_BYTES / wbytes))))
     layers = []
@@ -660,7 +659,6 @@ def w4a16_point(spec, device, steps):
            "frac_of_hbm": round(algo / t / 1e9 / peak, 3),
            "cublas_bf16_us": round(tc * 1e6, 3), "speedup_vs_cublas_bf16": round(tc / t, 3)}
     del gr, gc
-    base.close()
     for L in layers:
         L.close()
     return out
