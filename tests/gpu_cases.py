@@ -14,7 +14,7 @@ from bit_w4a4_quantized_b200 import svdq
 from oracle import formats as F
 from oracle import svdquant as S
 
-Y_TOL = 1e-2       # max|Y - Y_ref| / max|Y_ref| (the layer tolerance of the benchmark spec)
+Y_TOL = 1e-2       # max|Y - Y_ref| / max|Y_ref| (the layer tolerance)
 LR_TOL = 2.0**-7   # lr' is rounded to bf16 once: relative error <= 2^-9, margin for fp32 sums
 
 
