@@ -254,3 +254,30 @@ def test_largest_sweep_point_on_sampled_outputs():
     y = Y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
     err = S.max_rel_err(y, S.linear(ref, ref_act))
     assert err <= Y_TOL, err
+
+
+@pytest.mark.parametrize("M,K,N,r", [(300, 1024, 512, 128), (200, 2048, 256, 256)])
+def test_large_ranks_up_to_the_capacity_limit(M, K, N, r):
+    # rank 256 is the capacity limit: kernel 1 reduces its float partials by
+    # pulling them from the cluster (the push buffer no longer fits beside the
+    # stages) and kernel 2 folds four 64-rank chunks
+    case = Case(WL.make_x(M, K, seed=r), WL.make_w(N, K, seed=r), r, bias=WL.make_bias(N, seed=r))
+    act, Y = case.run()
+    err = check_y(case, Y, check_act(case, act))
+    print(f"M{M} K{K} N{N} r{r}: max rel err {err:.3e}")
+    case.layer.poll_status()
+
+
+def test_lora_filling_the_rank_capacity():
+    # rank 240 + a 16-rank adapter = 256, the largest total the layer takes
+    M, K, N = 130, 512, 320
+    case = Case(WL.make_x(M, K, seed=33), WL.make_w(N, K, seed=33), 240, rank_capacity=256)
+    A, B = WL.make_lora(K, N, 16, seed=33)
+    Ad = torch.from_numpy(A.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    Bd = torch.from_numpy(B.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    case.layer.lora_swap(Ad, Bd)
+    S.attach_lora(case.ref, A.astype(np.float32), B.astype(np.float32))
+    act, Y = case.run()
+    check_y(case, Y, check_act(case, act))
+    assert case.layer.info().rank_total == 256
+    case.layer.poll_status()
