@@ -55,3 +55,23 @@ def test_host_only_layer_cannot_launch():
     assert "uploaded" in svdq.last_error()
     with pytest.raises(svdq.SvdqError):
         L.export(svdq.EXPORT_L1)
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(kt=st.integers(1, 4), n=st.integers(1, 40), seed=st.integers(0, 10_000), with_s=st.booleans(),
+       scale=st.sampled_from([1e-4, 0.02, 3.0, 200.0]))
+def test_host_quantization_matches_the_oracle_on_random_layers(kt, n, seed, with_s, scale):
+    # any K that is a multiple of 64, any N, weights over several orders of magnitude
+    K = 64 * kt
+    g = np.random.default_rng(seed)
+    W = WL.to_bf16(g.standard_normal((n, K)) * scale)
+    s = (np.exp(g.uniform(-2, 2, K))).astype(np.float32) if with_s else None
+    L = svdq.W4A16Layer(W, s=s)
+    ref = W4.prepare(W.astype(np.float32), s=s)
+    np.testing.assert_array_equal(L.export(svdq.EXPORT_W_CODES), F.pack_e2m1(ref.codes))
+    np.testing.assert_array_equal(L.export(svdq.EXPORT_W_SCALES), ref.scales)
+    assert L.export(svdq.EXPORT_SCALARS)[0] == ref.g
+    L.close()
