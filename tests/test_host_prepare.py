@@ -117,3 +117,41 @@ def test_library_svd_exact_rank():
     s = scipy.linalg.svd(A, compute_uv=False)
     assert r_f64 <= 1.01 * np.sqrt(np.sum(s[r:] ** 2))
     assert r_f64 < 1e-2 * np.linalg.norm(A)
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=20, deadline=None)
+@given(kt=st.integers(1, 3), nt=st.integers(1, 2), r=st.sampled_from([0, 16]), seed=st.integers(0, 10_000),
+       wscale=st.sampled_from([1e-6, 0.02, 50.0]), zero_cols=st.integers(0, 3))
+def test_prepare_is_bit_exact_on_random_layers(kt, nt, r, seed, wscale, zero_cols):
+    # zero activation channels and zero weight columns (lambda = 1 there), weights from
+    # E4M3-subnormal block scales to large ones, ranks 0 and 16
+    K, N = 64 * kt, 64 * nt
+    g = np.random.default_rng(seed)
+    W = WL.to_bf16(g.standard_normal((N, K)) * wscale)
+    amax = np.abs(g.standard_normal(K) * 3.0).astype(np.float32)
+    cols = g.choice(K, size=zero_cols, replace=False)
+    if zero_cols:
+        amax[cols[: (zero_cols + 1) // 2]] = 0.0
+        Wz = W.astype(np.float32)
+        Wz[:, cols[(zero_cols + 1) // 2:]] = 0.0
+        W = WL.to_bf16(Wz)
+    amax = WL.to_bf16(amax).astype(np.float32)  # calibration maxima of bf16 activations
+    Wf = W.astype(np.float32)
+    if r:
+        l1b, l2b, _ = _oracle_factors(Wf, amax, r)
+        factors = (l1b, l2b)
+        lib_factors = (F.bf16_bits(l1b.astype(np.float32)), F.bf16_bits(l2b.astype(np.float32)))
+    else:
+        factors, lib_factors = None, None
+    ref = S.prepare(Wf, amax, r, bias=None, factors=factors)
+    layer = svdq.Layer(W, amax, r, factors=lib_factors, keep_r=True, threads=2)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_LAMBDA), ref.lam)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_R), ref.R.astype(np.float32))
+    g_a, g_w, _, _ = layer.export(svdq.EXPORT_SCALARS)
+    assert g_w == ref.g_w and g_a == ref.g_a
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_CODES), F.pack_e2m1(ref.w_codes))
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_SCALES), ref.w_scales)
+    layer.close()
