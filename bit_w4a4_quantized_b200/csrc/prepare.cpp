@@ -12,6 +12,7 @@
 // Every decision that fixes a code is taken in float32 with correctly rounded
 // operations, so the codes equal those of any other exact implementation.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <memory>
@@ -351,27 +352,42 @@ svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image
         return SVDQ_ERR_INVALID_ARGUMENT;
       }
     }
+  // two passes over W' = f32(W diag(s)), one row at a time (no N x K copy): its maximum, then the codes
   const uint16_t* W = static_cast<const uint16_t*>(d->W);
-  std::vector<float> wp(size_t(N) * size_t(K));
+  const int threads = int(std::max(1u, std::min(16u, std::thread::hardware_concurrency())));
+  auto scaled_row = [&](int64_t n, float* out) {
+    for (int64_t k = 0; k < K; ++k) out[k] = bf16_bits_to_f32(W[size_t(n) * K + k]) * s[size_t(k)];
+  };
+  std::vector<float> part_max(size_t(threads), 0.0f);
+  {
+    std::atomic<int> next_slot{0};
+    parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
+      const int slot = next_slot.fetch_add(1);
+      std::vector<float> row(static_cast<size_t>(K));
+      float m = 0.0f;
+      for (int64_t n = n0; n < n1; ++n) {
+        scaled_row(n, row.data());
+        for (int64_t k = 0; k < K; ++k) m = std::max(m, std::fabs(row[size_t(k)]));
+      }
+      part_max[size_t(slot)] = m;
+    });
+  }
   float amax = 0.0f;
-  for (int64_t n = 0; n < N; ++n)
-    for (int64_t k = 0; k < K; ++k) {
-      const float v = bf16_bits_to_f32(W[size_t(n) * K + k]) * s[size_t(k)];
-      wp[size_t(n) * K + k] = v;
-      amax = std::max(amax, std::fabs(v));
-    }
+  for (float m : part_max) amax = std::max(amax, m);  // max is order-independent: exact
   const float g = global_scale(amax);
   const float c = 1.0f / (6.0f * g);
   codes->assign(size_t(N) * size_t(K / 2), 0);
   scales->assign(size_t(N) * size_t(K / 16), 0);
   uint8_t* cr = codes->data();
   uint8_t* sr = scales->data();
-  const int threads = int(std::max(1u, std::min(16u, std::thread::hardware_concurrency())));
   parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
-    for (int64_t n = n0; n < n1; ++n)
-      quantize_row(&wp[size_t(n) * K], K, g, c,
+    std::vector<float> row(static_cast<size_t>(K));
+    for (int64_t n = n0; n < n1; ++n) {
+      scaled_row(n, row.data());
+      quantize_row(row.data(), K, g, c,
                    [&](int64_t k, uint8_t byte) { cr[size_t(n) * size_t(K / 2) + size_t(k / 2)] = byte; },
                    [&](int64_t sb, uint8_t code) { sr[size_t(n) * size_t(K / 16) + size_t(sb)] = code; });
+    }
   });
   // the device image: tiles of 16 rows x 64 inputs in fragment order
   const W4A16Geom geo = make_w4a16_geom(K, N);
