@@ -300,14 +300,15 @@ SVDQ_API svdq_status svdq_layer_clone(const svdq_layer* layer, svdq_layer** out)
  * modulation projections; SVDQuant summary page, section 2 "AWQ": protect the
  * weights by shifting scale onto the activations):
  *
- *     Y = g (X diag(s)^-1) deq(Q(W diag(s)))^T + b
+ *     Y = g f16(X diag(s)^-1) deq(Q(W diag(s)))^T + b
  *
  * Q is the NVFP4 quantizer of the W4A4 layer (E2M1 codes, an E4M3 scale per 16
  * weights along K, tensor scale g = max|W diag(s)| / 2688); s is one positive
  * activation-aware scale per input channel (the pages give no rule for it:
- * it is an input, 1 when NULL).  Activations stay bf16 and are divided by s
- * in float32; the sums are float32; Y is bf16.  The path is built for the
- * small batches of the modulation layers (M rows of X, a few at a time).
+ * it is an input, 1 when NULL).  The activations are divided by s in float32
+ * and rounded once to f16 (saturating at +-65504), as X_hat is rounded to a
+ * 16-bit operand in the W4A4 layer; products are exact, sums float32, Y bf16.
+ * The path is built for the small batches of the modulation layers.
  */
 typedef struct svdq_w4a16 svdq_w4a16;
 
@@ -329,10 +330,10 @@ SVDQ_API svdq_status svdq_w4a16_prepare_host(const svdq_w4a16_desc* d, svdq_w4a1
 SVDQ_API svdq_status svdq_w4a16_upload(svdq_w4a16* layer, void* dev_buf, size_t dev_buf_bytes, void* stream);
 
 /*
- * Y = g (X diag(s)^-1) deq^T + b.  X: device bf16 [M, K] row-major, 16-byte
- * aligned; Y: device bf16 [M, N] row-major, 2-byte aligned; any M >= 1 (rows
- * go 4 at a time, one launch each, stream ordered).  No bounded waits: the
- * kernel never waits on another CTA.
+ * Y = g f16(X diag(s)^-1) deq^T + b.  X: device bf16 [M, K] row-major,
+ * 16-byte aligned; Y: device bf16 [M, N] row-major, 2-byte aligned; any M >= 1
+ * (rows go 8 at a time, one launch each, stream ordered).  No bounded waits:
+ * the kernel's CTAs never wait on one another.
  */
 SVDQ_API svdq_status svdq_w4a16_linear(const svdq_w4a16* layer, const void* X, int64_t M, void* Y, void* stream);
 
