@@ -375,7 +375,8 @@ class Layer:
 
 
 class W4A16Layer:
-    """A W4A16 layer: 4-bit NVFP4 weights of W diag(s), bf16 activations divided by s."""
+    """A W4A16 layer: 4-bit NVFP4 weights of W diag(s); bf16 activations divided by s and
+    rounded once to f16 in the kernel; float32 sums, bf16 output."""
 
     def __init__(self, W, s=None, bias=None, *, device=None, stream=None):
         self._h = None
