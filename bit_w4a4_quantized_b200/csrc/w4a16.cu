@@ -8,9 +8,9 @@
 // accumulators): A = 16 weight rows x 16 inputs, dequantized in registers (the
 // hardware E2M1 -> f16x2 conversion, times the E4M3 block scale: exact in f16),
 // B = 16 inputs x 8 rows of X (x~ in shared memory; rows past M are zero
-// operands in registers).  The
-// prepared image stores each 16 x 64 weight tile in fragment order, so one
-// 16-byte load per lane brings the A operands of four MMAs.  A CTA of 8 warps
+// operands in registers).  The prepared image stores each 16 x 64 weight tile
+// in fragment order, so one 16-byte load per lane brings the A operands of
+// four MMAs.  A CTA of 8 warps
 // takes a 16-row tile of the output; its warps split K (tile kt goes to warp
 // kt % 8), issue all their weight loads before any arithmetic, and add their
 // partial sums through shared memory in a fixed order.  With one row of X the
