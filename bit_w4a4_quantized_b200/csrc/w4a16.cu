@@ -10,13 +10,13 @@
 // B = 16 inputs x 8 rows of X (x~ in shared memory; rows past M are zero
 // operands in registers).  The prepared image stores each 16 x 64 weight tile
 // in fragment order, so one 16-byte load per lane brings the A operands of
-// four MMAs.  A CTA of 8 warps
-// takes a 16-row tile of the output; its warps split K (tile kt goes to warp
-// kt % 8), issue all their weight loads before any arithmetic, and add their
-// partial sums through shared memory in a fixed order.  With one row of X the
-// MMA would be 7/8 padding, so that launch does the same tiles on the CUDA
-// cores instead: mixed-precision fused multiply-adds (f16 operands, float32
-// accumulator) straight from the f16 weights, no conversion to float32.
+// four MMAs.  A CTA of 8 warps takes a 16-row tile of the output; its warps
+// split K (tile kt goes to warp kt % 8), issue all their weight loads before
+// any arithmetic, and add their partial sums through shared memory in a fixed
+// order.  With one row of X the MMA would be 7/8 padding, so that launch does
+// the same tiles on the CUDA cores instead: mixed-precision fused multiply-adds
+// (f16 operands, float32 accumulator) straight from the f16 weights, no
+// conversion to float32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
