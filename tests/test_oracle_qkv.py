@@ -178,3 +178,17 @@ def _norm_no_weight(y, w, eps):
 def test_planted_mistakes_are_caught(monkeypatch, name, fn):
     monkeypatch.setattr(Q, name, fn)
     assert _pins_fail() >= 1
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=30, deadline=None)
+@given(M=st.integers(1, 4), heads=st.integers(1, 3), half=st.sampled_from([1, 2, 4]), seed=st.integers(0, 10_000),
+       eps=st.sampled_from([0.0, 1e-6, 0.5]), scale=st.sampled_from([1e-3, 1.0, 300.0]))
+def test_matches_brute_force_on_random_heads(M, heads, half, seed, eps, scale):
+    D = 2 * half
+    y, wq, wk, rope, _ = _case(M=M, heads=heads, D=D, seed=seed, scale=scale)
+    want = BF.qkv_norm_rope(y.tolist(), wq.tolist(), wk.tolist(), rope.tolist(), eps, D)
+    got = Q.qkv_norm_rope(y, wq, wk, rope, eps=eps, head_dim=D)
+    np.testing.assert_allclose(got, np.array(want), rtol=1e-11, atol=1e-11)
