@@ -132,3 +132,23 @@ def _linear_no_bias(layer, X, rows=None):
 def test_planted_mistakes_are_caught(monkeypatch, fn):
     monkeypatch.setattr(W4, "linear", fn)
     assert _pins_fail() >= 1
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(N=st.integers(1, 5), kb=st.integers(1, 3), M=st.integers(1, 3), seed=st.integers(0, 10_000),
+       with_s=st.booleans(), with_bias=st.booleans(), wscale=st.sampled_from([1e-3, 0.05, 20.0]))
+def test_matches_brute_force_on_random_layers(N, kb, M, seed, with_s, with_bias, wscale):
+    K = 16 * kb
+    g = np.random.default_rng(seed)
+    W = (g.standard_normal((N, K)) * wscale).astype(np.float32)
+    X = g.standard_normal((M, K)).astype(np.float32)
+    s = (0.25 + 2 * g.random(K)).astype(np.float32) if with_s else np.ones(K, np.float32)
+    b = g.standard_normal(N) * 0.01 if with_bias else None
+    want = BF.w4a16_forward(W.tolist(), X.tolist(), s.tolist(), None if b is None else b.tolist())
+    L = W4.prepare(W, s=s if with_s else None, bias=b)
+    np.testing.assert_array_equal(L.codes, np.array(want["codes"]))
+    np.testing.assert_array_equal(L.scales, np.array(want["scales"]))
+    np.testing.assert_allclose(W4.linear(L, X), np.array(want["Y"]), rtol=1e-11, atol=1e-11)
