@@ -3,7 +3,7 @@ activation-aware scale s per input channel) against oracle.w4a16.
 
 Codes and scales are checked bit for bit on the host (tests/test_w4a16_host.py);
 here Y is compared with max|Y - Y_ref| / max|Y_ref| <= 1e-2 over several row
-counts (the kernel takes X 4 rows per launch), ragged N, the smallest K, bias
+counts (the kernel takes X 8 rows per launch), ragged N, the smallest K, bias
 and s, and the FLUX-like modulation shape on sampled output features."""
 
 import numpy as np
