@@ -159,16 +159,41 @@ def rope_pack(rope, head_dim=128, out=None, stream=None):
     import torch
 
     M = rope.shape[0]
-    if not rope.is_contiguous() or rope.dtype != torch.float32:
-        raise ValueError("rope must be a contiguous float32 tensor")
+    if not rope.is_cuda:
+        raise ValueError("rope must be a device tensor")
+    _need(rope, "rope", rope.device, torch.float32, min_numel=M * int(head_dim))
     if out is None:
         out = torch.empty(rope_packed_bytes(M, head_dim), dtype=torch.uint8, device=rope.device)
+    _need(out, "out", rope.device)
     check(lib().svdq_rope_pack(rope.data_ptr(), M, int(head_dim), out.data_ptr(), _nbytes(out), _stream(stream)))
     return out
 
 
 def _nbytes(t):
     return t.numel() * t.element_size()
+
+
+def _need(t, name, device, dtype=None, shape=None, min_numel=None):
+    """Refuse, before any library call, a tensor that the C ABI cannot check
+    itself (it sees only a pointer): one on another device or on the host, a
+    non-contiguous view, or one of the wrong dtype or shape.  None passes
+    through, so that the library reports a missing argument."""
+    import torch
+
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the layer on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, fewer than {min_numel}")
 
 
 def _ptr(a):
@@ -274,6 +299,11 @@ class Layer:
             check(lib().svdq_layer_upload(self._h, self.dev_buf.data_ptr(), self.device_bytes, _stream(stream)))
         return self
 
+    def _device(self):
+        if self.dev_buf is None:
+            raise SvdqError(ERR_INVALID_ARGUMENT, "layer has not been uploaded")
+        return self.dev_buf.device
+
     def act_buffer_bytes(self, M):
         n = ctypes.c_size_t()
         check(lib().svdq_act_buffer_bytes(self._h, M, ctypes.byref(n)))
@@ -282,26 +312,34 @@ class Layer:
     def new_act_buffer(self, M):
         import torch
 
-        return torch.empty(self.act_buffer_bytes(M), dtype=torch.uint8, device=self.dev_buf.device)
+        return torch.empty(self.act_buffer_bytes(M), dtype=torch.uint8, device=self._device())
 
     def quantize_act(self, X, act=None, stream=None):
         """Kernel 1 on a device bf16 [M, K] tensor; returns the activation buffer."""
+        import torch
+
+        dev = self._device()
+        if X is None or X.dim() != 2:
+            raise ValueError("X must be a 2-D tensor [M, K]")
         M = X.shape[0]
+        _need(X, "X", dev, torch.bfloat16, (M, self.K))
         if act is None:
             act = self.new_act_buffer(M)
-        if not X.is_contiguous():
-            raise ValueError("X must be contiguous")
-        check(lib().svdq_quantize_act(self._h, X.data_ptr(), M, act.data_ptr(), act.numel(), _stream(stream)))
+        _need(act, "act", dev)
+        check(lib().svdq_quantize_act(self._h, X.data_ptr(), M, act.data_ptr(), _nbytes(act), _stream(stream)))
         return act
 
     def linear(self, act, M, out=None, epilogue=EPI_NONE, stream=None):
         """Kernel 2; returns Y bf16 [M, N]."""
         import torch
 
+        dev = self._device()
+        _need(act, "act", dev)
         if out is None:
-            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=act.device)
-        check(lib().svdq_w4a4_linear(self._h, act.data_ptr(), act.numel(), M, out.data_ptr(), epilogue,
-                                     _stream(stream)))
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
+        _need(out, "out", dev, torch.bfloat16, (M, self.N))
+        check(lib().svdq_w4a4_linear(self._h, _ptr(act), 0 if act is None else _nbytes(act), M, out.data_ptr(),
+                                     epilogue, _stream(stream)))
         return out
 
     def linear_qkv_norm_rope(self, act, M, norm_q, norm_k, rope_packed, eps=1e-6, head_dim=128, out=None,
@@ -311,9 +349,16 @@ class Layer:
         rope_packed: from ``rope_pack``); returns bf16 [M, N]."""
         import torch
 
+        dev = self._device()
+        _need(act, "act", dev)
+        _need(norm_q, "norm_q", dev, torch.bfloat16, min_numel=int(head_dim))
+        _need(norm_k, "norm_k", dev, torch.bfloat16, min_numel=int(head_dim))
+        _need(rope_packed, "rope_packed", dev)
         if out is None:
-            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=act.device)
-        check(lib().svdq_w4a4_linear_qkv_norm_rope(self._h, act.data_ptr(), act.numel(), M, out.data_ptr(),
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
+        _need(out, "out", dev, torch.bfloat16, (M, self.N))
+        check(lib().svdq_w4a4_linear_qkv_norm_rope(self._h, _ptr(act), 0 if act is None else _nbytes(act), M,
+                                                   out.data_ptr(),
                                                    _ptr(norm_q), _ptr(norm_k), _ptr(rope_packed),
                                                    0 if rope_packed is None else _nbytes(rope_packed),
                                                    int(head_dim), float(eps), _stream(stream)))
@@ -325,7 +370,18 @@ class Layer:
 
     def lora_swap(self, A=None, B=None, scale=1.0, stream=None):
         """Attach a LoRA (device bf16 A [K, r_e], B [r_e, N]); A=None detaches."""
-        r_e = 0 if A is None else A.shape[1]
+        import torch
+
+        dev = self._device()
+        if A is None:
+            B = None
+            r_e = 0
+        else:
+            if A.dim() != 2 or B is None:
+                raise ValueError("A must be [K, r_e] and B [r_e, N]")
+            r_e = A.shape[1]
+            _need(A, "A", dev, torch.bfloat16, (self.K, r_e))
+            _need(B, "B", dev, torch.bfloat16, (r_e, self.N))
         check(lib().svdq_lora_swap(self._h, _ptr(A), _ptr(B), r_e, float(scale), _stream(stream)))
 
     def poll_status(self, stream=None):
@@ -407,11 +463,16 @@ class W4A16Layer:
         """Y bf16 [M, N] from a device bf16 [M, K] tensor."""
         import torch
 
-        if not X.is_contiguous():
-            raise ValueError("X must be contiguous")
+        if self.dev_buf is None:
+            raise SvdqError(ERR_INVALID_ARGUMENT, "layer has not been uploaded")
+        dev = self.dev_buf.device
+        if X is None or X.dim() != 2:
+            raise ValueError("X must be a 2-D tensor [M, K]")
         M = X.shape[0]
+        _need(X, "X", dev, torch.bfloat16, (M, self.K))
         if out is None:
-            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=X.device)
+            out = torch.empty((M, self.N), dtype=torch.bfloat16, device=dev)
+        _need(out, "out", dev, torch.bfloat16, (M, self.N))
         check(lib().svdq_w4a16_linear(self._h, X.data_ptr(), M, out.data_ptr(), _stream(stream)))
         return out
 

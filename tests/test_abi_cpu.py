@@ -142,3 +142,61 @@ def test_clone_copies_the_prepared_layer_and_outlives_it():
     # not bound to a device buffer: launching must be refused, not crash
     st = svdq.lib().svdq_quantize_act(twin._h, 1, 1, 1, 1, None)
     assert st == svdq.ERR_INVALID_ARGUMENT
+
+
+def test_binding_refuses_tensors_the_abi_cannot_check():
+    """The C ABI sees only pointers, so the binding refuses, before any library
+    call, a host tensor, another device, a wrong dtype or shape, a
+    non-contiguous view and a short norm weight.  A meta tensor stands in for
+    the layer's device buffer: nothing here touches a GPU."""
+    import torch
+
+    spec = WL.CFG1
+    K, N = spec.K, spec.N
+    layer = svdq.Layer(spec.w(), svdq.calibrate_amax(spec.x()), spec.rank)
+    with pytest.raises(svdq.SvdqError) as e:
+        layer.quantize_act(torch.zeros((4, K), dtype=torch.bfloat16))
+    assert e.value.status == svdq.ERR_INVALID_ARGUMENT and "uploaded" in str(e.value)
+    layer.dev_buf = torch.empty(0, dtype=torch.uint8, device="meta")
+
+    def meta(shape, dt=torch.bfloat16):
+        return torch.empty(shape, dtype=dt, device="meta")
+
+    act = meta((1 << 16,), torch.uint8)
+    refused = [
+        lambda: layer.quantize_act(torch.zeros((4, K), dtype=torch.bfloat16)),  # host memory
+        lambda: layer.quantize_act(meta((4, K), torch.float32)),
+        lambda: layer.quantize_act(meta((4, K + 64))),
+        lambda: layer.quantize_act(meta((K,))),
+        lambda: layer.quantize_act(meta((K, 4)).t()),  # a transposed view
+        lambda: layer.quantize_act(meta((4, K)), act=torch.zeros(1 << 16, dtype=torch.uint8)),
+        lambda: layer.linear(torch.zeros(1 << 16, dtype=torch.uint8), 4),
+        lambda: layer.linear(act, 4, out=meta((4, N + 1))),
+        lambda: layer.linear(act, 4, out=meta((4, N), torch.float16)),
+        lambda: layer.linear(act, 4, out=meta((N, 4)).t()),
+        lambda: layer.forward(meta((4, K), torch.float16)),
+        lambda: layer.lora_swap(meta((K, 16)), None),
+        lambda: layer.lora_swap(meta((K, 16)), meta((32, N))),
+        lambda: layer.lora_swap(meta((K + 64, 16)), meta((16, N))),
+        lambda: layer.lora_swap(torch.zeros((K, 16), dtype=torch.bfloat16), meta((16, N))),
+        lambda: layer.linear_qkv_norm_rope(act, 4, meta((64,)), meta((128,)), meta((64,), torch.uint8)),
+        lambda: layer.linear_qkv_norm_rope(act, 4, meta((128,)), meta((128,), torch.float32), meta((64,), torch.uint8)),
+        lambda: layer.linear_qkv_norm_rope(act, 4, meta((128,)), meta((128,)), torch.zeros(64, dtype=torch.uint8)),
+    ]
+    for i, f in enumerate(refused):
+        with pytest.raises((ValueError, TypeError)):
+            f()
+            pytest.fail(f"case {i} was not refused")
+
+    w = svdq.W4A16Layer(WL.make_w(16, 64, seed=3))
+    with pytest.raises(svdq.SvdqError):
+        w.linear(torch.zeros((1, 64), dtype=torch.bfloat16))
+    w.dev_buf = torch.empty(0, dtype=torch.uint8, device="meta")
+    for f in (lambda: w.linear(torch.zeros((1, 64), dtype=torch.bfloat16)),
+              lambda: w.linear(meta((1, 128))),
+              lambda: w.linear(meta((1, 64), torch.float32)),
+              lambda: w.linear(meta((1, 64)), out=meta((1, 17)))):
+        with pytest.raises((ValueError, TypeError)):
+            f()
+    with pytest.raises(ValueError):
+        svdq.rope_pack(torch.zeros((4, 64, 2), dtype=torch.float32))  # host memory
