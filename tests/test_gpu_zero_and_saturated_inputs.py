@@ -1,0 +1,107 @@
+"""GPU parity on the degenerate inputs of the method, through the C ABI.
+
+- Zero blocks: a 16-element block of X_hat whose maximum is 0 gets the E4M3
+  scale 0 and all codes 0 (reciprocal taken as 0), a zero channel gets
+  lambda = 1, and a zero row of X gives Y = b exactly, since every term of the
+  accumulator is 0 (SVDQuant summary page, section 3 "Quantization
+  preliminary": s = max|X| / q_max, here per block).
+- An all-zero calibration batch: the activation tensor scale falls back to 1.
+- Activations beyond the calibrated maximum: the activation tensor scale is
+  static, so larger runtime values saturate, the block scale at E4M3's 448 and
+  the elements at E2M1's +-6, on both sides.
+- An empty batch is refused before any launch.
+
+Codes and scales are compared bit for bit, Y within the layer tolerance."""
+
+import numpy as np
+import pytest
+import torch
+from ml_dtypes import bfloat16
+
+from bit_w4a4_quantized_b200 import svdq
+from bit_w4a4_quantized_b200 import workloads as WL
+from gpu_cases import Case, check_act, check_y, y_to_f64
+from oracle import formats as F
+from oracle import svdquant as S
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(X):
+    return torch.from_numpy(X.view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _zeroed_x(M, K, seed):
+    X = WL.make_x(M, K, seed=seed).astype(np.float32)
+    g = np.random.default_rng([seed, 99])
+    blocks = X.reshape(M, K // 16, 16)
+    blocks[g.random((M, K // 16)) < 0.1] = 0.0  # a tenth of the blocks
+    X[[0, M // 3, M - 1]] = 0.0  # whole rows
+    X[:, 32:48] = 0.0  # whole channels (lambda = 1)
+    return X.astype(bfloat16)
+
+
+@pytest.mark.parametrize("r", [0, 32])
+def test_zero_rows_channels_and_blocks(r):
+    M, K, N = 200, 512, 384
+    X = _zeroed_x(M, K, seed=61 + r)
+    bias = WL.make_bias(N, seed=61)
+    case = Case(X, WL.make_w(N, K, seed=61), r, bias=bias)
+    assert case.ref.lam[32] == 1.0
+    act, Y = case.run()
+    ref = check_act(case, act)
+    assert np.count_nonzero(ref.scales == 0) > M  # zero blocks were exercised
+    check_y(case, Y, ref)
+    Yb = Y.view(torch.int16).cpu().numpy().view(np.uint16)
+    want = np.asarray(bias).view(np.uint16)
+    for m in (0, M // 3, M - 1):
+        np.testing.assert_array_equal(Yb[m], want)
+
+
+def test_all_zero_calibration_batch_gives_the_bias():
+    M, K, N = 130, 256, 192
+    X = np.zeros((M, K), dtype=bfloat16)
+    bias = WL.make_bias(N, seed=62)
+    case = Case(X, WL.make_w(N, K, seed=62), 16, bias=bias)
+    assert case.ref.g_a == 1.0
+    act, Y = case.run()
+    ref = check_act(case, act)
+    assert not np.any(ref.codes) and not np.any(ref.scales)
+    np.testing.assert_array_equal(Y.view(torch.int16).cpu().numpy().view(np.uint16),
+                                  np.broadcast_to(np.asarray(bias).view(np.uint16), (M, N)))
+
+
+@pytest.mark.parametrize("factor", [8.0, 64.0])
+def test_activations_beyond_calibration_saturate(factor):
+    M, K, N, r = 160, 768, 256, 16
+    X = WL.make_x(M, K, seed=63)
+    case = Case(X, WL.make_w(N, K, seed=63), r)
+    Xs = (X.astype(np.float32) * np.float32(factor)).astype(bfloat16)  # a power of two: exact in bf16
+    act, Y = case.run(X=_dev(Xs))
+    codes, scales, lr = case.unpack(act, M)
+    ref = S.quantize_act(case.ref, Xs.astype(np.float32))
+    assert np.count_nonzero(ref.scales == 0x7E) > 0  # block scales saturated at 448
+    top = np.float64(6 * 448) * np.float64(case.ref.g_a)  # the largest value Q can represent
+    assert np.max(np.abs(ref.x_hat)) > 1.5 * top  # elements saturated at +-6
+    np.testing.assert_array_equal(codes, F.pack_e2m1(ref.codes))
+    np.testing.assert_array_equal(scales, ref.scales)
+    lr_gpu = F.bf16_from_bits(lr).astype(np.float64) * case.ref.alpha
+    assert np.max(np.abs(lr_gpu - ref.lr)) <= 2.0**-7 * np.max(np.abs(ref.lr))
+    err = S.max_rel_err(y_to_f64(Y), S.linear(case.ref, ref))
+    assert err <= 1e-2, err
+
+
+def test_empty_batch_is_refused():
+    case = Case(WL.make_x(64, 256, seed=64), WL.make_w(256, 256, seed=64), 16)
+    with pytest.raises(svdq.SvdqError) as e:
+        case.layer.quantize_act(case.Xd[:0])
+    assert e.value.status == svdq.ERR_INVALID_ARGUMENT
+    act = case.layer.quantize_act(case.Xd)
+    Y = torch.empty((64, 256), dtype=torch.bfloat16, device="cuda")
+    lib = svdq.lib()
+    assert lib.svdq_w4a4_linear(case.layer._h, act.data_ptr(), act.numel(), 0, Y.data_ptr(), 0, None) == \
+        svdq.ERR_INVALID_ARGUMENT
+    # the layer still runs
+    Y = case.layer.linear(act, 64)
+    torch.cuda.synchronize()
+    check_y(case, Y, check_act(case, act))

@@ -155,3 +155,22 @@ def test_prepare_is_bit_exact_on_random_layers(kt, nt, r, seed, wscale, zero_col
     np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_CODES), F.pack_e2m1(ref.w_codes))
     np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_SCALES), ref.w_scales)
     layer.close()
+
+
+def test_all_zero_calibration_batch():
+    """A layer calibrated on an all-zero batch: lambda = 1 on every channel
+    (either maximum 0) and the activation tensor scale falls back to 1, on both
+    sides, bit for bit."""
+    W = WL.make_w(192, 256, seed=62)
+    Wf = W.astype(np.float32)
+    amax = np.zeros(256, np.float32)
+    l1b, l2b, _ = _oracle_factors(Wf, amax, 16)
+    ref = S.prepare(Wf, amax, 16, factors=(l1b, l2b))
+    assert np.all(ref.lam == 1.0) and ref.g_a == 1.0
+    layer = svdq.Layer(W, amax, 16, factors=(F.bf16_bits(l1b.astype(np.float32)), F.bf16_bits(l2b.astype(np.float32))),
+                       threads=2)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_LAMBDA), ref.lam)
+    g_a, g_w, alpha, _ = layer.export(svdq.EXPORT_SCALARS)
+    assert g_a == 1.0 and g_w == ref.g_w and alpha == np.float32(ref.g_a * ref.g_w)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_CODES), F.pack_e2m1(ref.w_codes))
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_SCALES), ref.w_scales)
