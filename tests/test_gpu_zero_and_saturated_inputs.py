@@ -105,3 +105,52 @@ def test_empty_batch_is_refused():
     Y = case.layer.linear(act, 64)
     torch.cuda.synchronize()
     check_y(case, Y, check_act(case, act))
+
+
+def _w4a16_check(X, W, s=None, bias=None):
+    from oracle import w4a16 as W4
+
+    L = svdq.W4A16Layer(W, s=s, bias=bias, device="cuda")
+    Y = L.linear(_dev(X))
+    torch.cuda.synchronize()
+    ref = W4.prepare(W.astype(np.float32), s=s, bias=None if bias is None else bias.astype(np.float32))
+    want = W4.linear(ref, X.astype(np.float32))
+    err = S.max_rel_err(y_to_f64(Y), want)
+    assert err <= 1e-2, err
+    return Y, ref
+
+
+@pytest.mark.parametrize("M", [1, 5])
+def test_w4a16_zero_weight_rows_and_blocks_give_the_bias(M):
+    """W4A16: zero weight blocks get the scale 0; an all-zero output row gives
+    Y = b exactly; an all-zero W falls back to the tensor scale 1."""
+    K, N = 512, 96
+    W = WL.make_w(N, K, seed=65).astype(np.float32)
+    g = np.random.default_rng([65, 99])
+    W.reshape(N, K // 16, 16)[g.random((N, K // 16)) < 0.2] = 0.0
+    W[[3, 40, N - 1]] = 0.0
+    W = W.astype(bfloat16)
+    bias = WL.make_bias(N, seed=65)
+    X = WL.make_x(M, K, seed=65, n_outlier=0)
+    Y, ref = _w4a16_check(X, W, s=WL.make_awq_scales(K, seed=65), bias=bias)
+    assert np.count_nonzero(ref.scales == 0) > 3 * K // 16
+    Yb = Y.view(torch.int16).cpu().numpy().view(np.uint16)
+    for n in (3, 40, N - 1):
+        np.testing.assert_array_equal(Yb[:, n], np.asarray(bias).view(np.uint16)[n])
+    Z = np.zeros((N, K), dtype=bfloat16)
+    Y0, ref0 = _w4a16_check(X, Z, bias=bias)
+    assert ref0.g == 1.0
+    np.testing.assert_array_equal(Y0.view(torch.int16).cpu().numpy().view(np.uint16),
+                                  np.broadcast_to(np.asarray(bias).view(np.uint16), (M, N)))
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_w4a16_activations_beyond_f16_saturate(M):
+    """W4A16: x / s is rounded to f16 saturating at +-65504 on both sides."""
+    K, N = 256, 64
+    X = (WL.make_x(M, K, seed=66, n_outlier=0).astype(np.float32) * np.float32(2.0**17)).astype(bfloat16)
+    from oracle import w4a16 as W4
+
+    s = WL.make_awq_scales(K, seed=66)
+    assert np.count_nonzero(np.abs(W4.act_operand(X.astype(np.float32), np.float32(1.0) / s)) == 65504.0) > 0
+    _w4a16_check(X, WL.make_w(N, K, seed=66), s=s)
