@@ -201,7 +201,8 @@ SVDQ_API svdq_status svdq_w4a4_linear(const svdq_layer* layer, const void* act_b
  *   written by svdq_rope_pack from the [M][head_dim / 2][2] table; row m of Y
  *   uses row m of the table.  One packed table serves every layer and call
  *   with the same rows.
- * eps: finite, >= 0 (FLUX uses 1e-6).
+ * eps: finite, >= 0 (FLUX uses 1e-6).  With eps = 0 an all-zero Q or K head
+ *   is 0 / 0 and comes out NaN, as the formula gives.
  * act_buf, M, Y, stream: as svdq_w4a4_linear.
  */
 SVDQ_API svdq_status svdq_w4a4_linear_qkv_norm_rope(const svdq_layer* layer, const void* act_buf,

@@ -154,3 +154,20 @@ def test_w4a16_activations_beyond_f16_saturate(M):
     s = WL.make_awq_scales(K, seed=66)
     assert np.count_nonzero(np.abs(W4.act_operand(X.astype(np.float32), np.float32(1.0) / s)) == 65504.0) > 0
     _w4a16_check(X, WL.make_w(N, K, seed=66), s=s)
+
+
+def test_qkv_norm_rope_on_zero_heads():
+    """The fused Q/K RMSNorm + rotary epilogue on zero rows (no bias): every
+    head's sum of squares is 0, eps keeps the norm finite, and the row stays
+    0; other rows carry zero blocks and channels."""
+    from test_gpu_qkv import _check, _inputs, _run, _v_passes_through
+
+    M, K, C = 200, 512, 256
+    X = _zeroed_x(M, K, seed=67)
+    case = Case(X, WL.make_w(3 * C, K, seed=67), 16)
+    host, dev = _inputs(M, seed=67)
+    act, Yf, Yp = _run(case, dev, M)
+    _check(case, Yf, check_act(case, act), host)
+    _v_passes_through(Yf, Yp)
+    for m in (0, M // 3, M - 1):
+        assert not torch.any(Yf[m].float() != 0).item()
