@@ -11,6 +11,8 @@ import numpy as np
 import pytest
 import scipy.linalg
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import bruteforce as BF
 from bit_w4a4_quantized_b200 import workloads as WL
@@ -80,6 +82,34 @@ def test_scales_fit_e4m3_under_global_scale():
     assert np.all(F.e4m3_decode(scales) <= 448.0)
     # the block holding the tensor max gets the largest scale code (448)
     assert np.max(scales) == 0x7E
+
+
+@settings(max_examples=60, deadline=None)
+@given(seed=st.integers(0, 2**31 - 1), log_scale=st.floats(-12, 12), heavy=st.booleans())
+def test_quantizer_is_idempotent_on_normal_scales(seed, log_scale, heavy):
+    """Q(deq(Q(t)) g) = Q(t) on every block whose E4M3 scale is normal: each
+    block's largest element lands on code 6 (the E4M3 rounding of the scale is
+    within 1/16, so amax / d stays in [5.65, 6.4)), the dequantized block's
+    maximum is then exactly 6 d, and every code value survives the round trip.
+    A scale computed with a q_max other than 6 breaks it (the largest code is
+    then not 6); errors in d alone are left to the brute force and the error
+    bound above, since a consistently rescaled d still round-trips."""
+    g0 = np.random.default_rng(seed)
+    t = g0.standard_normal((16, 128)) * np.exp2(log_scale)
+    if heavy:
+        t = t * np.exp2(g0.integers(-8, 9, size=(16, 8, 1))).repeat(16, axis=2).reshape(16, 128)
+    t = t.astype(np.float32)
+    g = S.global_scale(np.max(np.abs(t)))
+    codes, scales = S.nvfp4_quantize(t, g)
+    deq = (S.nvfp4_dequantize(codes, scales) * np.float64(g)).astype(np.float32)
+    codes2, scales2 = S.nvfp4_quantize(deq, g)
+    normal = F.e4m3_decode(scales) >= 2.0**-6
+    assert np.any(normal)
+    blk = np.repeat(normal, 16, axis=1)
+    np.testing.assert_array_equal(scales2[normal], scales[normal])
+    np.testing.assert_array_equal(codes2[blk], codes[blk])
+    top = np.max(np.abs(F.e2m1_decode(codes)).reshape(16, 8, 16), axis=2)
+    assert np.all(top[normal] == 6.0)
 
 
 # ---------------------------------------------------------------- smoothing
