@@ -196,15 +196,31 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
       L->inv_lam[k] = 1.0f / lam;
     }
 
-    // 2. smoothed weight W_hat^T [K, N] in float64 (exact: float32 x bf16)
-    std::vector<double> R(size_t(K) * N);
-    //    (transposed in 64 x 64 blocks so both sides stay in cache)
+    // 2. smoothed weight W_hat^T [K, N] in float64 (exact: float32 x bf16).
+    //    The buffer is left uninitialised (every element is written below, by
+    //    the thread that owns its rows).  The transpose goes through 64 x 64
+    //    tiles in a local buffer, so that W and R are both walked along rows:
+    //    R's row stride is often a multiple of 4 KB, and walking down its
+    //    columns would keep evicting lines that map to the same cache sets.
+    std::unique_ptr<double[]> r_buf(new double[size_t(K) * N]);
+    double* R = r_buf.get();
     parallel_rows(ceil_div(K, 64), threads, [&](int64_t b0, int64_t b1) {
-      for (int64_t kb = b0 * 64; kb < std::min(K, b1 * 64); kb += 64)
-        for (int64_t nb = 0; nb < N; nb += 64)
-          for (int64_t n = nb; n < std::min(N, nb + 64); ++n)
-            for (int64_t k = kb; k < std::min(K, kb + 64); ++k)
-              R[size_t(k) * N + n] = double(L->lam[k]) * double(bf16_bits_to_f32(d->W[n * K + k]));
+      float tile[64][64];
+      for (int64_t kb = b0 * 64; kb < std::min(K, b1 * 64); kb += 64) {
+        const int64_t kn = std::min<int64_t>(64, K - kb);
+        for (int64_t nb = 0; nb < N; nb += 64) {
+          const int64_t nn = std::min<int64_t>(64, N - nb);
+          for (int64_t j = 0; j < nn; ++j) {
+            const uint16_t* w = d->W + (nb + j) * K + kb;
+            for (int64_t i = 0; i < kn; ++i) tile[i][j] = bf16_bits_to_f32(w[i]);
+          }
+          for (int64_t i = 0; i < kn; ++i) {
+            const double lam = L->lam[kb + i];
+            double* row = R + size_t(kb + i) * N + nb;
+            for (int64_t j = 0; j < nn; ++j) row[j] = lam * double(tile[i][j]);
+          }
+        }
+      }
     });
 
     // 3. low-rank factors, bf16 [K, r] and [r, N]
@@ -215,7 +231,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
       std::memcpy(L->l2.data(), d->L2, sizeof(uint16_t) * L->l2.size());
     } else if (r > 0) {
       SvdFactors f;
-      randomized_svd(R.data(), K, N, r, d->svd_oversample ? d->svd_oversample : 16,
+      randomized_svd(R, K, N, r, d->svd_oversample ? d->svd_oversample : 16,
                      d->svd_power_iters ? d->svd_power_iters : 8, d->svd_seed, threads, &f);
       L->sigma = f.sigma;
       std::vector<double> l1d(size_t(K) * r);
@@ -247,9 +263,11 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
     }
 
     // 4. residual R = W_hat^T - L1 L2 with the bf16 factors, rank-one terms in
-    //    order i = 0 .. r-1 (each product of two bf16 values is exact)
+    //    order i = 0 .. r-1 (each product of two bf16 values is exact), and
+    //    its squared norm per row, summed over the rows in order afterwards
     std::vector<double> l2d(size_t(r) * N);
     for (size_t i = 0; i < l2d.size(); ++i) l2d[i] = bf16_bits_to_f32(L->l2[i]);
+    std::vector<double> row_sq(K, 0.0);
     parallel_rows(K, threads, [&](int64_t k0, int64_t k1) {
       for (int64_t k = k0; k < k1; ++k) {
         double* row = &R[size_t(k) * N];
@@ -258,30 +276,55 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
           const double* v = &l2d[size_t(i) * N];
           for (int64_t n = 0; n < N; ++n) row[n] = row[n] - a * v[n];
         }
+        double sq = 0;
+        for (int64_t n = 0; n < N; ++n) sq += row[n] * row[n];
+        row_sq[k] = sq;
       }
     });
     {
       double s = 0;
-      for (double v : R) s += v * v;
+      for (double v : row_sq) s += v;
       L->resid_bf16 = std::sqrt(s);
     }
 
-    // 5. R^T as float32 [N, K], tensor scale, NVFP4 codes into the image
-    std::vector<float> rt(size_t(N) * K);
+    // 5. R^T as float32 [N, K] (uninitialised, then written whole; tiled as
+    //    in step 2) and its largest magnitude, then the tensor scale and the
+    //    NVFP4 codes into the image
+    std::unique_ptr<float[]> rt_buf(new float[size_t(N) * K]);
+    float* rt = rt_buf.get();
+    std::vector<float> tile_max(ceil_div(N, 64), 0.0f);
     parallel_rows(ceil_div(N, 64), threads, [&](int64_t b0, int64_t b1) {
-      for (int64_t nb = b0 * 64; nb < std::min(N, b1 * 64); nb += 64)
-        for (int64_t kb = 0; kb < K; kb += 64)
-          for (int64_t k = kb; k < std::min(K, kb + 64); ++k)
-            for (int64_t n = nb; n < std::min(N, nb + 64); ++n) rt[size_t(n) * K + k] = float(R[size_t(k) * N + n]);
+      float tile[64][64];
+      for (int64_t nb = b0 * 64; nb < std::min(N, b1 * 64); nb += 64) {
+        const int64_t nn = std::min<int64_t>(64, N - nb);
+        float m = 0.0f;
+        for (int64_t kb = 0; kb < K; kb += 64) {
+          const int64_t kn = std::min<int64_t>(64, K - kb);
+          for (int64_t i = 0; i < kn; ++i) {
+            const double* row = R + size_t(kb + i) * N + nb;
+            for (int64_t j = 0; j < nn; ++j) tile[j][i] = float(row[j]);
+          }
+          for (int64_t j = 0; j < nn; ++j) {
+            float* out = rt + size_t(nb + j) * K + kb;
+            for (int64_t i = 0; i < kn; ++i) {
+              out[i] = tile[j][i];
+              m = std::max(m, std::fabs(tile[j][i]));
+            }
+          }
+        }
+        tile_max[nb / 64] = m;
+      }
     });
     if (d->flags & SVDQ_PREPARE_KEEP_R) {
       L->r32.resize(size_t(K) * N);
-      for (int64_t k = 0; k < K; ++k)
-        for (int64_t n = 0; n < N; ++n) L->r32[size_t(k) * N + n] = float(R[size_t(k) * N + n]);
+      parallel_rows(K, threads, [&](int64_t k0, int64_t k1) {
+        for (int64_t k = k0; k < k1; ++k)
+          for (int64_t n = 0; n < N; ++n) L->r32[size_t(k) * N + n] = float(R[size_t(k) * N + n]);
+      });
     }
-    std::vector<double>().swap(R);
+    r_buf.reset();
     float amax_r = 0.0f;
-    for (float v : rt) amax_r = std::max(amax_r, std::fabs(v));
+    for (float v : tile_max) amax_r = std::max(amax_r, v);
     L->g_w = global_scale(amax_r);
     const float c_w = 1.0f / (6.0f * L->g_w);
 
@@ -307,7 +350,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
     if (d->bias) std::memcpy(img + g.off_bias, d->bias, sizeof(uint16_t) * N);
     parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
       for (int64_t n = n0; n < n1; ++n)
-        quantize_row(&rt[size_t(n) * K], K, L->g_w, c_w,
+        quantize_row(rt + size_t(n) * K, K, L->g_w, c_w,
                      [&](int64_t k, uint8_t byte) { img[bcode_off(g, n, k)] = byte; },
                      [&](int64_t s, uint8_t code) { img[bsf_off(g, n, s)] = code; });
     });
