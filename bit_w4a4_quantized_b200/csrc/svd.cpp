@@ -17,6 +17,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <immintrin.h>
 #include <numeric>
 #include <thread>
 #include <vector>
@@ -63,35 +64,103 @@ void parallel_for(int64_t n, int threads, F&& f) {
   for (auto& th : pool) th.join();
 }
 
-// Y[K x l] = A[K x N] X[N x l], row-major.
+// out[i][c] = fma(M[i][j], V[j][c], out[i][c]) for j = 0 .. jn-1 in order, for
+// rows i < rows and columns c < l (M row stride ldm, V and out row stride l).
+// Every output is one chain of fused multiply-adds in ascending j, whatever
+// the blocking, so callers may split j into consecutive blocks.  Tiles of
+// 4 rows x 8 columns keep 8 accumulators in AVX2 registers.
+void accumulate_rows(const double* M, int64_t ldm, int64_t rows, int64_t jn, const double* V, int l,
+                     double* out) {
+  const int l8 = l / 8 * 8;
+  int64_t i = 0;
+  for (; i + 4 <= rows; i += 4) {
+    const double* m0 = M + i * ldm;
+    const double* m1 = m0 + ldm;
+    const double* m2 = m1 + ldm;
+    const double* m3 = m2 + ldm;
+    double* o = out + i * l;
+    for (int c = 0; c < l8; c += 8) {
+      __m256d a00 = _mm256_loadu_pd(o + c), a01 = _mm256_loadu_pd(o + c + 4);
+      __m256d a10 = _mm256_loadu_pd(o + l + c), a11 = _mm256_loadu_pd(o + l + c + 4);
+      __m256d a20 = _mm256_loadu_pd(o + 2 * l + c), a21 = _mm256_loadu_pd(o + 2 * l + c + 4);
+      __m256d a30 = _mm256_loadu_pd(o + 3 * l + c), a31 = _mm256_loadu_pd(o + 3 * l + c + 4);
+      const double* v = V + c;
+      for (int64_t j = 0; j < jn; ++j, v += l) {
+        const __m256d v0 = _mm256_loadu_pd(v), v1 = _mm256_loadu_pd(v + 4);
+        __m256d b = _mm256_broadcast_sd(m0 + j);
+        a00 = _mm256_fmadd_pd(b, v0, a00);
+        a01 = _mm256_fmadd_pd(b, v1, a01);
+        b = _mm256_broadcast_sd(m1 + j);
+        a10 = _mm256_fmadd_pd(b, v0, a10);
+        a11 = _mm256_fmadd_pd(b, v1, a11);
+        b = _mm256_broadcast_sd(m2 + j);
+        a20 = _mm256_fmadd_pd(b, v0, a20);
+        a21 = _mm256_fmadd_pd(b, v1, a21);
+        b = _mm256_broadcast_sd(m3 + j);
+        a30 = _mm256_fmadd_pd(b, v0, a30);
+        a31 = _mm256_fmadd_pd(b, v1, a31);
+      }
+      _mm256_storeu_pd(o + c, a00);
+      _mm256_storeu_pd(o + c + 4, a01);
+      _mm256_storeu_pd(o + l + c, a10);
+      _mm256_storeu_pd(o + l + c + 4, a11);
+      _mm256_storeu_pd(o + 2 * l + c, a20);
+      _mm256_storeu_pd(o + 2 * l + c + 4, a21);
+      _mm256_storeu_pd(o + 3 * l + c, a30);
+      _mm256_storeu_pd(o + 3 * l + c + 4, a31);
+    }
+    for (int c = l8; c < l; ++c)
+      for (int q = 0; q < 4; ++q) {
+        const double* m = M + (i + q) * ldm;
+        double acc = o[q * l + c];
+        for (int64_t j = 0; j < jn; ++j) acc = std::fma(m[j], V[j * l + c], acc);
+        o[q * l + c] = acc;
+      }
+  }
+  for (; i < rows; ++i) {
+    const double* m = M + i * ldm;
+    double* o = out + i * l;
+    for (int c = 0; c < l; ++c) {
+      double acc = o[c];
+      for (int64_t j = 0; j < jn; ++j) acc = std::fma(m[j], V[j * l + c], acc);
+      o[c] = acc;
+    }
+  }
+}
+
+constexpr int64_t kBlockJ = 256;  // reduction block: 256 x l doubles of V stay in L2
+
+// Y[K x l] = A[K x N] X[N x l], row-major.  Each thread owns a range of rows
+// and walks N in blocks, reusing the block of X across its rows.
 void mul_A_X(const double* A, int64_t K, int64_t N, const double* X, int l, double* Y, int threads) {
   parallel_for(K, threads, [&](int64_t k0, int64_t k1) {
-    std::vector<double> acc(l);
-    for (int64_t k = k0; k < k1; ++k) {
-      std::fill(acc.begin(), acc.end(), 0.0);
-      const double* a = A + k * N;
-      for (int64_t n = 0; n < N; ++n) {
-        const double av = a[n];
-        const double* x = X + n * l;
-        for (int c = 0; c < l; ++c) acc[c] += av * x[c];
-      }
-      std::memcpy(Y + k * l, acc.data(), sizeof(double) * l);
-    }
+    std::fill(Y + k0 * l, Y + k1 * l, 0.0);
+    for (int64_t nb = 0; nb < N; nb += kBlockJ)
+      accumulate_rows(A + k0 * N + nb, N, k1 - k0, std::min(kBlockJ, N - nb), X + nb * l, l, Y + k0 * l);
   });
 }
 
 // Z[N x l] = A^T Q, A [K x N], Q [K x l], row-major.  Each thread owns a
-// column range of A (rows of Z) and sums over k in order.
+// range of rows of Z (columns of A) and walks K in blocks; a 64 x 256 panel of
+// A^T is packed so that its rows are contiguous.
 void mul_At_Q(const double* A, int64_t K, int64_t N, const double* Q, int l, double* Z, int threads) {
-  std::fill(Z, Z + N * l, 0.0);
   parallel_for(N, threads, [&](int64_t n0, int64_t n1) {
-    for (int64_t k = 0; k < K; ++k) {
-      const double* a = A + k * N;
-      const double* q = Q + k * l;
-      for (int64_t n = n0; n < n1; ++n) {
-        const double av = a[n];
-        double* z = Z + n * l;
-        for (int c = 0; c < l; ++c) z[c] += av * q[c];
+    std::fill(Z + n0 * l, Z + n1 * l, 0.0);
+    std::vector<double> panel(size_t(64) * kBlockJ);
+    for (int64_t kb = 0; kb < K; kb += kBlockJ) {
+      const int64_t kn = std::min(kBlockJ, K - kb);
+      for (int64_t nt = n0; nt < n1; nt += 64) {
+        const int64_t nn = std::min<int64_t>(64, n1 - nt);
+        for (int64_t k0 = 0; k0 < kn; k0 += 8)  // in 8 x 8 sub-blocks: whole lines in, whole lines out
+          for (int64_t j0 = 0; j0 < nn; j0 += 8) {
+            const int64_t kc = std::min<int64_t>(8, kn - k0), jc = std::min<int64_t>(8, nn - j0);
+            double t[8][8];
+            for (int64_t a = 0; a < kc; ++a)
+              for (int64_t b = 0; b < jc; ++b) t[a][b] = A[(kb + k0 + a) * N + nt + j0 + b];
+            for (int64_t b = 0; b < jc; ++b)
+              for (int64_t a = 0; a < kc; ++a) panel[size_t(j0 + b) * kBlockJ + k0 + a] = t[a][b];
+          }
+        accumulate_rows(panel.data(), kBlockJ, nn, kn, Q + kb * l, l, Z + nt * l);
       }
     }
   });
