@@ -1,0 +1,70 @@
+"""bench.py on the CPU: the reference arm's JSON line (the oracle timed on the
+host cores), what the other ranks of a multi-rank launch do there, the
+argument guards, and the small helpers the GPU arm's line is built from."""
+
+import json
+
+import pytest
+
+import bench
+
+
+def _line(capsys, argv):
+    assert bench.main(argv) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1, lines
+    return json.loads(lines[0])
+
+
+def test_reference_arm_prints_one_complete_line(capsys, monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    out = _line(capsys, ["--impl", "reference", "--workload", "cfg1", "--steps", "2", "--warmup", "3",
+                         "--cpu-budget", "1"])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in out, key
+    assert out["impl"] == "reference" and out["metric"] == bench.METRIC and out["unit"] == bench.UNIT
+    assert out["steps"] == 2 and out["warmup"] == 3 and out["n_gpus"] == 1
+    assert out["value"] > 0 and out["higher_is_better"] is True
+    assert out["config"]["workload"] == bench.workload_spec("cfg1").name
+    cb = out["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == out["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert out["e2e"] == {"value": out["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_without_work(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    assert bench.main(["--impl", "reference", "--gpus", "2", "--steps", "2", "--warmup", "3"]) == 0
+    assert capsys.readouterr().out.strip() == ""
+
+
+def test_argument_guards(monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--warmup", "2"])  # fewer than 3 warm-up steps
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--gpus", "2", "--warmup", "3"])  # launch and flag disagree
+    with pytest.raises(SystemExit):
+        bench.workload_spec("no_such_workload")
+
+
+def test_line_helpers():
+    spec = bench.workload_spec("cfg2")
+    fp4, lowrank = bench.layer_flops(spec, 32)
+    assert fp4 == 2 * 4096 * 3072 * 3072
+    assert lowrank == 2 * 4096 * 3072 * 32 * 2
+    assert bench.aggregate(5.0, 4, 2.0) == 10.0
+    assert bench.qkv_shape(9216) and not bench.qkv_shape(3072 + 64)
+    assert bench.rank_seed(1, 0) == 1 and bench.rank_seed(1, 3) != bench.rank_seed(1, 2)
+    peak, hbm, origin = bench.measured_peaks()
+    assert peak > 0 and hbm > 0 and origin in ("measured", "fallback")
+    # traffic is taken from a committed ncu summary only for the workload it was captured on
+    assert bench.profiled_traffic("gemm_kernel", "some_other_workload") is None
+    t = bench.profiled_traffic("gemm_kernel", "attn_proj_M4096_K3072_N3072_r32")
+    assert t is None or t > 0
