@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <exception>
 #include <new>
 #include <string>
 
@@ -387,8 +388,17 @@ svdq_status svdq_w4a16_prepare_host(const svdq_w4a16_desc* d, svdq_w4a16** out) 
   if (!out) return fail(SVDQ_ERR_INVALID_ARGUMENT, "out is NULL");
   std::string err;
   auto* L = new (std::nothrow) svdq_w4a16();
-  if (!L) return fail(SVDQ_ERR_INTERNAL, "out of host memory");
-  svdq_status st = svdq::w4a16_quantize(d, &L->image, &L->codes, &L->scales, &L->gscale, &err);
+  if (!L) return fail(SVDQ_ERR_HOST_ALLOC, "host allocation failed");
+  svdq_status st;
+  try {
+    st = svdq::w4a16_quantize(d, &L->image, &L->codes, &L->scales, &L->gscale, &err);
+  } catch (const std::bad_alloc&) {
+    st = SVDQ_ERR_HOST_ALLOC;
+    err = "host allocation failed while quantizing the W4A16 layer";
+  } catch (const std::exception& e) {
+    st = SVDQ_ERR_INTERNAL;
+    err = std::string("W4A16 quantization failed: ") + e.what();
+  }
   if (st != SVDQ_OK) {
     delete L;
     return fail(st, err);

@@ -15,11 +15,13 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <exception>
 #include <memory>
 #include <new>
 #include <thread>
 
 #include "layer.h"
+#include "parallel.h"
 #include "svd.h"
 #include "w4a16.h"
 
@@ -127,22 +129,6 @@ void quantize_row(const float* t, int64_t k, float g, float c, PutByte&& put_byt
   }
 }
 
-template <class F>
-void parallel_rows(int64_t n, int threads, F&& f) {
-  if (threads <= 1 || n < 2) {
-    f(int64_t(0), n);
-    return;
-  }
-  std::vector<std::thread> pool;
-  int64_t per = (n + threads - 1) / threads;
-  for (int t = 0; t < threads; ++t) {
-    int64_t b = t * per, e = std::min(n, b + per);
-    if (b >= e) break;
-    pool.emplace_back([&f, b, e] { f(b, e); });
-  }
-  for (auto& th : pool) th.join();
-}
-
 }  // namespace
 
 svdq_status validate_desc(const svdq_prepare_desc* d, std::string* err) {
@@ -204,7 +190,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
     //    columns would keep evicting lines that map to the same cache sets.
     std::unique_ptr<double[]> r_buf(new double[size_t(K) * N]);
     double* R = r_buf.get();
-    parallel_rows(ceil_div(K, 64), threads, [&](int64_t b0, int64_t b1) {
+    parallel_for(ceil_div(K, 64), threads, [&](int64_t b0, int64_t b1) {
       float tile[64][64];
       for (int64_t kb = b0 * 64; kb < std::min(K, b1 * 64); kb += 64) {
         const int64_t kn = std::min<int64_t>(64, K - kb);
@@ -243,7 +229,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
       for (size_t i = 0; i < L->l2.size(); ++i) L->l2[i] = f64_to_bf16_bits(f.Vt[i]);
       // ||W_hat^T - L1 L2|| with the float64 factors
       std::vector<double> part(K, 0.0);
-      parallel_rows(K, threads, [&](int64_t k0, int64_t k1) {
+      parallel_for(K, threads, [&](int64_t k0, int64_t k1) {
         std::vector<double> row(N);
         for (int64_t k = k0; k < k1; ++k) {
           std::memcpy(row.data(), &R[size_t(k) * N], sizeof(double) * N);
@@ -268,7 +254,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
     std::vector<double> l2d(size_t(r) * N);
     for (size_t i = 0; i < l2d.size(); ++i) l2d[i] = bf16_bits_to_f32(L->l2[i]);
     std::vector<double> row_sq(K, 0.0);
-    parallel_rows(K, threads, [&](int64_t k0, int64_t k1) {
+    parallel_for(K, threads, [&](int64_t k0, int64_t k1) {
       for (int64_t k = k0; k < k1; ++k) {
         double* row = &R[size_t(k) * N];
         for (int i = 0; i < r; ++i) {
@@ -293,7 +279,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
     std::unique_ptr<float[]> rt_buf(new float[size_t(N) * K]);
     float* rt = rt_buf.get();
     std::vector<float> tile_max(ceil_div(N, 64), 0.0f);
-    parallel_rows(ceil_div(N, 64), threads, [&](int64_t b0, int64_t b1) {
+    parallel_for(ceil_div(N, 64), threads, [&](int64_t b0, int64_t b1) {
       float tile[64][64];
       for (int64_t nb = b0 * 64; nb < std::min(N, b1 * 64); nb += 64) {
         const int64_t nn = std::min<int64_t>(64, N - nb);
@@ -317,7 +303,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
     });
     if (d->flags & SVDQ_PREPARE_KEEP_R) {
       L->r32.resize(size_t(K) * N);
-      parallel_rows(K, threads, [&](int64_t k0, int64_t k1) {
+      parallel_for(K, threads, [&](int64_t k0, int64_t k1) {
         for (int64_t k = k0; k < k1; ++k)
           for (int64_t n = 0; n < N; ++n) L->r32[size_t(k) * N + n] = float(R[size_t(k) * N + n]);
       });
@@ -348,7 +334,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
       inv_img[k] = k < K ? L->inv_lam[k] : 1.0f;
     }
     if (d->bias) std::memcpy(img + g.off_bias, d->bias, sizeof(uint16_t) * N);
-    parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
+    parallel_for(N, threads, [&](int64_t n0, int64_t n1) {
       for (int64_t n = n0; n < n1; ++n)
         quantize_row(rt + size_t(n) * K, K, L->g_w, c_w,
                      [&](int64_t k, uint8_t byte) { img[bcode_off(g, n, k)] = byte; },
@@ -366,6 +352,8 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
       }
   } catch (const std::bad_alloc&) {
     return *err = "host allocation failed during preparation", SVDQ_ERR_HOST_ALLOC;
+  } catch (const std::exception& e) {
+    return *err = std::string("preparation failed: ") + e.what(), SVDQ_ERR_INTERNAL;
   }
   *out = L.release();
   return SVDQ_OK;
@@ -404,7 +392,7 @@ svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image
   std::vector<float> part_max(size_t(threads), 0.0f);
   {
     std::atomic<int> next_slot{0};
-    parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
+    parallel_for(N, threads, [&](int64_t n0, int64_t n1) {
       const int slot = next_slot.fetch_add(1);
       std::vector<float> row(static_cast<size_t>(K));
       float m = 0.0f;
@@ -423,7 +411,7 @@ svdq_status w4a16_quantize(const svdq_w4a16_desc* d, std::vector<uint8_t>* image
   scales->assign(size_t(N) * size_t(K / 16), 0);
   uint8_t* cr = codes->data();
   uint8_t* sr = scales->data();
-  parallel_rows(N, threads, [&](int64_t n0, int64_t n1) {
+  parallel_for(N, threads, [&](int64_t n0, int64_t n1) {
     std::vector<float> row(static_cast<size_t>(K));
     for (int64_t n = n0; n < n1; ++n) {
       scaled_row(n, row.data());

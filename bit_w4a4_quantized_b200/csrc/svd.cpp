@@ -14,6 +14,8 @@
 // the result depends only on the inputs and the seed, not on the thread count.
 #include "svd.h"
 
+#include "parallel.h"
+
 #include <algorithm>
 #include <cmath>
 #include <cstring>
@@ -46,23 +48,6 @@ struct Rng {
     }
   }
 };
-
-template <class F>
-void parallel_for(int64_t n, int threads, F&& f) {
-  // f(begin, end) over [0, n) in `threads` contiguous pieces
-  if (threads <= 1 || n < 2) {
-    f(int64_t(0), n);
-    return;
-  }
-  std::vector<std::thread> pool;
-  int64_t per = (n + threads - 1) / threads;
-  for (int t = 0; t < threads; ++t) {
-    int64_t b = t * per, e = std::min(n, b + per);
-    if (b >= e) break;
-    pool.emplace_back([&f, b, e] { f(b, e); });
-  }
-  for (auto& th : pool) th.join();
-}
 
 // out[i][c] = fma(M[i][j], V[j][c], out[i][c]) for j = 0 .. jn-1 in order, for
 // rows i < rows and columns c < l (M row stride ldm, V and out row stride l).
