@@ -147,6 +147,9 @@ svdq_status validate_desc(const svdq_prepare_desc* d, std::string* err) {
   if (d->rank > std::min(d->K, d->N)) return *err = "rank exceeds min(K, N)", SVDQ_ERR_UNSUPPORTED_SHAPE;
   if (d->svd_power_iters < 0 || d->svd_oversample < 0)
     return *err = "svd parameters must be non-negative", SVDQ_ERR_INVALID_ARGUMENT;
+  for (int64_t k = 0; k < d->K; ++k)  // lambda and the activation tensor scale come from these
+    if (!(d->act_amax[k] >= 0.0f) || !std::isfinite(d->act_amax[k]))
+      return *err = "act_amax[" + std::to_string(k) + "] must be finite and >= 0", SVDQ_ERR_INVALID_ARGUMENT;
   return SVDQ_OK;
 }
 

@@ -95,7 +95,8 @@ typedef struct svdq_prepare_desc {
   const uint16_t* bias;    /* host bf16 [N], or NULL                               */
   const float* act_amax;   /* host float [K]: max_i |X_ij| over calibration rows
                               (see svdq_calibrate_amax); sets lambda and the static
-                              activation tensor scale                               */
+                              activation tensor scale.  Finite and >= 0, else
+                              SVDQ_ERR_INVALID_ARGUMENT                             */
   const uint16_t* L1;      /* optional host bf16 [K, rank]: use these low-rank
                               factors (e.g. from a checkpoint) instead of the
                               library's SVD; NULL = compute them                   */

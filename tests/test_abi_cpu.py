@@ -66,6 +66,16 @@ def test_prepare_rejects_bad_descriptors(field, value, status):
     del keep
 
 
+@pytest.mark.parametrize("bad", [-1.0, float("nan"), float("inf")])
+def test_prepare_rejects_bad_calibration_maxima(bad):
+    d, (W, amax) = _desc()
+    amax[17] = bad
+    h = ctypes.c_void_p()
+    assert svdq.lib().svdq_prepare_host(ctypes.byref(d), ctypes.byref(h)) == svdq.ERR_INVALID_ARGUMENT
+    assert "act_amax[17]" in svdq.last_error()
+    assert svdq.lib().svdq_layer_device_bytes(ctypes.byref(d)) == 0
+
+
 def test_null_arguments_are_errors_not_crashes():
     L = svdq.lib()
     assert L.svdq_prepare_host(None, None) == svdq.ERR_INVALID_ARGUMENT
