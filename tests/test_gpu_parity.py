@@ -281,3 +281,42 @@ def test_lora_filling_the_rank_capacity():
     check_y(case, Y, check_act(case, act))
     assert case.layer.info().rank_total == 256
     case.layer.poll_status()
+
+
+def test_graph_replay_of_the_bench_step_matches_direct_launches():
+    """The bench times kernel 1 + kernel 2 captured in one CUDA graph (linked by
+    programmatic dependent launch) over rotating buffer sets.  Replaying such a
+    graph gives the direct launches' output bit for bit, on every set."""
+    import bench
+
+    M = 1024
+    case = _spec_case(WL.CFG2, M=M)
+    act_ref, Y_ref = case.run()
+    check_y(case, Y_ref, check_act(case, act_ref))
+    layers = [case.layer, case.layer.clone(device="cuda")]
+    Xs = [case.Xd, case.Xd.clone()]
+    acts = [L.new_act_buffer(M) for L in layers]
+    Ys = [torch.empty((M, WL.CFG2.N), dtype=torch.bfloat16, device="cuda") for _ in layers]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for i in range(2):  # eager warm-up, as the bench does before capturing
+            layers[i].quantize_act(Xs[i], acts[i])
+            layers[i].linear(acts[i], M, out=Ys[i])
+        stream.synchronize()
+    fns = []
+    for i in range(2):
+        fns.append(lambda i=i: layers[i].quantize_act(Xs[i], acts[i]))
+        fns.append(lambda i=i: layers[i].linear(acts[i], M, out=Ys[i]))
+    graph = bench._capture(fns, stream)
+    for Y in Ys:
+        Y.zero_()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            graph.replay()
+    torch.cuda.synchronize()
+    for Y in Ys:
+        assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16))
+    for L in layers:
+        L.poll_status()
+    del graph
