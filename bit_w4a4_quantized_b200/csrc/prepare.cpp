@@ -90,22 +90,14 @@ inline float e4m3_value(uint8_t c) {
   return e ? std::ldexp(1.0f + m / 8.0f, e - 7) : std::ldexp(float(m), -9);
 }
 // E2M1 code (sign in bit 3) of a float: nearest even on {0, .5, 1, 1.5, 2, 3, 4, 6}, saturating.
-uint8_t e2m1_code(float t) {
+// The magnitude code counts the decision boundaries passed: the midpoints of the
+// grid, each tie going to the even code (0.25 -> 0, 0.75 -> 2, 1.25 -> 2,
+// 1.75 -> 4, 2.5 -> 4, 3.5 -> 6, 5 -> 6), and everything above 5 to 7.
+inline uint8_t e2m1_code(float t) {
   const uint8_t sign = std::signbit(t) ? 0x8 : 0x0;
-  float a = std::fabs(t);
-  if (a >= 6.0f) return sign | 7;
-  if (a == 0.0f) return sign;
-  int e;
-  std::frexp(a, &e);
-  int E = std::max(e - 1, 0);               // binade [2^E, 2^(E+1)), quantum 2^(E-1)
-  float scaled = std::ldexp(a, 1 - E);      // [2, 4) normal, [0, 2) subnormal
-  int m = int(std::nearbyint(scaled));
-  if (m >= 4) {
-    m = 2;
-    E += 1;
-  }
-  if (E == 0 && m < 2) return sign | uint8_t(m);
-  return sign | uint8_t(((E + 1) << 1) | (m - 2));
+  const float a = std::fabs(t);
+  const int m = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+  return sign | uint8_t(m);
 }
 
 float global_scale(float amax) { return amax == 0.0f ? 1.0f : amax / 2688.0f; }
