@@ -174,3 +174,45 @@ def test_all_zero_calibration_batch():
     assert g_a == 1.0 and g_w == ref.g_w and alpha == np.float32(ref.g_a * ref.g_w)
     np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_CODES), F.pack_e2m1(ref.w_codes))
     np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_SCALES), ref.w_scales)
+
+
+def test_host_quantizer_rounds_every_e2m1_tie_like_the_oracle():
+    """Rank 0 and lambda = 1 make R^T = W.  With max|W| = 2.625 the tensor scale
+    is 2^-10, and a block whose largest value is 1.5 gets the block scale 256, so
+    d = 0.25 and each weight times 1/d is exact: the weights 0.0625, 0.1875,
+    0.3125, 0.4375, 0.625, 0.875 and 1.25 land on the E2M1 ties 0.25 ... 5 (ties
+    go to the even code), and their bf16 neighbours one step off them."""
+    from ml_dtypes import bfloat16
+
+    K, N = 64, 64
+    ties = np.array([0.0625, 0.1875, 0.3125, 0.4375, 0.625, 0.875, 1.25], np.float32)
+    bits = ties.astype(bfloat16).view(np.uint16)
+    below = (bits - 1).view(bfloat16).astype(np.float32)  # the bf16 neighbours of each tie
+    above = (bits + 1).view(bfloat16).astype(np.float32)
+    vals = np.concatenate([ties, below, above])  # 21 values
+    W = np.zeros((N, K), np.float32)
+    for n in range(N):
+        for b in range(K // 16):
+            blk = np.zeros(16, np.float32)
+            blk[0] = 1.5  # block maximum: scale 256, d = 0.25
+            pick = np.random.default_rng([n, b]).choice(vals.size, 15, replace=False)
+            blk[1:] = vals[pick] * np.where(np.random.default_rng([b, n]).random(15) < 0.5, -1, 1)
+            W[n, 16 * b:16 * b + 16] = blk
+    W[0, 0] = 2.625  # the tensor maximum: g_w = 2^-10
+    Wb = W.astype(bfloat16)
+    assert np.array_equal(Wb.astype(np.float32), W)
+    amax = np.max(np.abs(W), axis=0)  # act_amax = max|W_:,j| gives lambda = 1
+    ref = S.prepare(W, amax, 0)
+    assert np.all(ref.lam == 1.0) and ref.g_w == np.float32(2.0**-10)
+    assert np.count_nonzero(ref.w_scales == 0x78) > N  # E4M3 256: d = 0.25 on those blocks
+    layer = svdq.Layer(Wb, amax, 0, threads=3)
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_CODES), F.pack_e2m1(ref.w_codes))
+    np.testing.assert_array_equal(layer.export(svdq.EXPORT_W_SCALES), ref.w_scales)
+    # the ties themselves went to the even code (0.25 -> 0, 0.75 -> 2, 1.25 -> 2, 1.75 -> 4, 2.5 -> 4, 3.5 -> 6, 5 -> 6)
+    deq_rows = ref.w_codes.reshape(N, K // 16, 16)
+    Wr = np.abs(W.reshape(N, K // 16, 16))
+    want = {0.0625: 0, 0.1875: 2, 0.3125: 2, 0.4375: 4, 0.625: 4, 0.875: 6, 1.25: 6}
+    for v, code in want.items():
+        sel = (Wr == np.float32(v)) & (ref.w_scales[..., None] == 0x78)
+        assert np.any(sel)
+        assert np.all((deq_rows[sel] & 7) == code), v
