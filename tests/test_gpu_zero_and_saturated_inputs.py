@@ -10,6 +10,8 @@
   static, so larger runtime values saturate, the block scale at E4M3's 448 and
   the elements at E2M1's +-6, on both sides.
 - An empty batch is refused before any launch.
+- Exact E2M1 ties: the device conversion takes each tie to the even code, as
+  the oracle does.
 
 Codes and scales are compared bit for bit, Y within the layer tolerance."""
 
@@ -171,3 +173,44 @@ def test_qkv_norm_rope_on_zero_heads():
     _v_passes_through(Yf, Yp)
     for m in (0, M // 3, M - 1):
         assert not torch.any(Yf[m].float() != 0).item()
+
+
+def _tie_inputs(M=64, K=128, N=64):
+    """X whose blocks have the maximum 1.5 and values on (or one bf16 step off)
+    the E2M1 ties after scaling, with max|X| = 2.625; W's column maxima equal
+    X's, so lambda = 1, x_hat = x, g_a = 2^-10, the block scale is 256 and
+    1/d = 4 exactly."""
+    ties = np.array([0.0625, 0.1875, 0.3125, 0.4375, 0.625, 0.875, 1.25], np.float32)
+    bits = ties.astype(bfloat16).view(np.uint16)
+    vals = np.concatenate([ties, (bits - 1).view(bfloat16).astype(np.float32),
+                           (bits + 1).view(bfloat16).astype(np.float32)])
+    X = np.zeros((M, K), np.float32)
+    g = np.random.default_rng(71)
+    for m in range(M):
+        for b in range(K // 16):
+            X[m, 16 * b] = 1.5
+            X[m, 16 * b + 1:16 * b + 16] = vals[g.choice(vals.size, 15, replace=False)] * np.where(
+                g.random(15) < 0.5, -1, 1)
+    X[0, 0] = 2.625
+    W = WL.make_w(N, K, seed=71).astype(np.float32)
+    W[0] = np.max(np.abs(X), axis=0)
+    return X.astype(bfloat16), W.astype(bfloat16), ties
+
+
+def test_activation_codes_on_exact_e2m1_ties():
+    """Kernel 1's hardware conversion (round to nearest even, satfinite) takes
+    every E2M1 tie to the even code, as the oracle's reading does: 0.25 -> 0,
+    0.75 -> 2, 1.25 -> 2, 1.75 -> 4, 2.5 -> 4, 3.5 -> 6, 5 -> 6."""
+    X, W, ties = _tie_inputs()
+    case = Case(X, W, 0)
+    assert np.all(case.ref.lam == 1.0) and case.ref.g_a == np.float32(2.0**-10)
+    act, Y = case.run()
+    ref = check_act(case, act)  # codes and scales bit for bit
+    check_y(case, Y, ref)
+    blocks = np.abs(X.astype(np.float32)).reshape(X.shape[0], -1, 16)
+    codes = ref.codes.reshape(blocks.shape)
+    on_256 = (ref.scales == 0x78)[..., None]
+    for v, code in zip(ties, (0, 2, 2, 4, 4, 6, 6)):
+        sel = (blocks == v) & on_256
+        assert np.count_nonzero(sel) > 100
+        assert np.all((codes[sel] & 7) == code), v
