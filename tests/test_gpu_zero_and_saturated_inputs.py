@@ -10,8 +10,8 @@
   static, so larger runtime values saturate, the block scale at E4M3's 448 and
   the elements at E2M1's +-6, on both sides.
 - An empty batch is refused before any launch.
-- Exact E2M1 ties: the device conversion takes each tie to the even code, as
-  the oracle does.
+- Exact E2M1 ties and exact E4M3 ties of the block scale: the device
+  conversions take each tie to the even code, as the oracle does.
 
 Codes and scales are compared bit for bit, Y within the layer tolerance."""
 
@@ -214,3 +214,50 @@ def test_activation_codes_on_exact_e2m1_ties():
         sel = (blocks == v) & on_256
         assert np.count_nonzero(sel) > 100
         assert np.all((codes[sel] & 7) == code), v
+
+
+def _e4m3_tie_inputs(N=64, K=128):
+    """Block maxima on every E4M3 midpoint (normal binades 2^-6 .. 2^7 and the
+    subnormal range), bf16-exact; one extra row holds the tensor maximum 448, so
+    g_a = f32(1/6), 6 g_a rounds to 1 and the block scale is E4M3(block max)
+    itself.  W's column maxima equal X's (lambda = 1)."""
+    mids = [(2.0**e * (1 + m / 8 + 1 / 16), m) for e in range(-6, 8) for m in range(8)]
+    mids += [((m + 0.5) * 2.0**-9, m) for m in range(8)]
+    per_row = K // 16
+    M = (len(mids) + per_row - 1) // per_row + 1
+    g = np.random.default_rng(72)
+    X = np.zeros((M, K), np.float32)
+    for i, (v, _) in enumerate(mids):
+        m, b = divmod(i, per_row)
+        blk = np.float32(v) * g.uniform(-1, 1, 16).astype(np.float32)
+        blk[g.integers(16)] = v if g.random() < 0.5 else -v
+        X[m, 16 * b:16 * b + 16] = blk
+    X[M - 1, 0] = 448.0
+    X = X.astype(bfloat16)
+    W = WL.make_w(N, K, seed=72).astype(np.float32)
+    W[0] = np.max(np.abs(X.astype(np.float32)), axis=0)
+    return X, W.astype(bfloat16), mids
+
+
+def test_block_scales_on_exact_e4m3_ties():
+    """Kernel 1's E4M3 block scale (round to nearest even, satfinite) on block
+    maxima that sit exactly between two E4M3 values: the even mantissa wins,
+    in the normal binades and among the subnormal scales (the midpoint 2^-10
+    goes to the scale 0, whose block then has all codes 0)."""
+    X, W, mids = _e4m3_tie_inputs()
+    case = Case(X, W, 0)
+    assert np.all(case.ref.lam == 1.0)
+    assert np.float32(np.float32(1.0) / np.float32(np.float32(6.0) * case.ref.g_a)) == 1.0
+    act, Y = case.run()
+    ref = check_act(case, act)  # codes and scales bit for bit
+    check_y(case, Y, ref)
+    scale = F.e4m3_decode(ref.scales)
+    per_row = X.shape[1] // 16
+    for i, (v, m) in enumerate(mids):
+        r, b = divmod(i, per_row)
+        if v < 2.0**-6:
+            lo, hi = m * 2.0**-9, (m + 1) * 2.0**-9
+        else:
+            e = np.floor(np.log2(v))
+            lo, hi = 2.0**e * (1 + m / 8), 2.0**e * (1 + (m + 1) / 8)
+        assert scale[r, b] == (lo if m % 2 == 0 else hi), (v, scale[r, b])
