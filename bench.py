@@ -167,12 +167,35 @@ class ClockSampler:
                 "samples": len(rows), "samples_under_load": len(sm)}
 
 
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}  # an earlier measurement on the same B200 pool
+
+
 def measured_peaks():
+    """(bf16 TFLOP/s, HBM GB/s, origin) from MEASURED_PEAKS.json; a value that is
+    missing, unreadable or not positive is replaced by the fallback, and the
+    origin then says so."""
+    d = {}
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
-        return d.get("bf16_tflops"), d.get("hbm_gbs"), "measured"
-    return 1590.0, 6650.0, "fallback"
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+    except (OSError, ValueError):
+        d = {}
+    out, fell_back = [], []
+    for key in ("bf16_tflops", "hbm_gbs"):
+        v = d.get(key) if isinstance(d, dict) else None
+        if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+            out.append(float(v))
+        else:
+            out.append(FALLBACK_PEAKS[key])
+            fell_back.append(key)
+    if not fell_back:
+        origin = "measured"
+    elif len(fell_back) == 2:
+        origin = "fallback"
+    else:
+        origin = "measured, fallback for " + ", ".join(fell_back)
+    return out[0], out[1], origin
 
 
 KERNEL_SOURCES = {

@@ -68,3 +68,14 @@ def test_line_helpers():
     assert bench.profiled_traffic("gemm_kernel", "some_other_workload") is None
     t = bench.profiled_traffic("gemm_kernel", "attn_proj_M4096_K3072_N3072_r32")
     assert t is None or t > 0
+
+
+def test_measured_peaks_fall_back_per_value(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_peaks() == (1590.0, 6650.0, "fallback")  # no file
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6551.0, "bf16_tflops": 1666.4}')
+    assert bench.measured_peaks() == (1666.4, 6551.0, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6551.0, "bf16_tflops": null}')
+    assert bench.measured_peaks() == (1590.0, 6551.0, "measured, fallback for bf16_tflops")
+    (tmp_path / "MEASURED_PEAKS.json").write_text("not json")
+    assert bench.measured_peaks() == (1590.0, 6650.0, "fallback")
