@@ -79,3 +79,20 @@ def test_measured_peaks_fall_back_per_value(tmp_path, monkeypatch):
     assert bench.measured_peaks() == (1590.0, 6551.0, "measured, fallback for bf16_tflops")
     (tmp_path / "MEASURED_PEAKS.json").write_text("not json")
     assert bench.measured_peaks() == (1590.0, 6650.0, "fallback")
+
+
+def test_clock_summary_keeps_the_benchmarked_gpu_under_load():
+    c = bench.ClockSampler(uuid="GPU-bbbb")
+    c.lines = [
+        "GPU-aaaa, 1965, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, Active",
+        "GPU-bbbb, 345, 1965, 120.0, 0x0, Not Active, Not Active, Not Active, Not Active",  # idle: below the floor
+        "GPU-bbbb, 1965, 1965, 800.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "GPU-bbbb, 1905, 1965, 1000.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "GPU-bbbb, 1935, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+    ]
+    s = c.summary()
+    assert s["sm_mhz"] == 1935.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 4 and s["samples_under_load"] == 3
+    empty = bench.ClockSampler().summary()
+    assert empty["sm_mhz"] is None and empty["samples"] == 0
