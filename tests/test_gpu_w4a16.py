@@ -3,8 +3,9 @@ activation-aware scale s per input channel) against oracle.w4a16.
 
 Codes and scales are checked bit for bit on the host (tests/test_w4a16_host.py);
 here Y is compared with max|Y - Y_ref| / max|Y_ref| <= 1e-2 over several row
-counts (the kernel takes X 8 rows per launch), ragged N, the smallest K, bias
-and s, and the FLUX-like modulation shape on sampled output features."""
+counts (the kernel takes X 8 rows per launch), ragged N, the smallest and the
+largest K, bias and s, and the FLUX-like modulation shape on sampled output
+features."""
 
 import numpy as np
 import pytest
@@ -45,6 +46,22 @@ def test_parity(M, K, N, with_s, with_bias):
     err = S.max_rel_err(y_to_f64(Y), want)
     assert err <= Y_TOL, err
     print(f"W4A16 M{M} K{K} N{N}: max rel err {err:.2e}")
+
+
+@pytest.mark.parametrize("M,K,N", [(3, 4096, 200), (1, 12288, 40), (8, 12288, 40), (9, 12288, 17)])
+def test_largest_k_and_several_passes_over_k(M, K, N):
+    """K above 3072 takes each warp through K in several passes of 6 tiles
+    (K = 4096: a partial second pass); K = 12288 is the largest K the layer
+    takes, and 8 rows of it the largest shared-memory request (196 KB).  Nine
+    rows run as one 8-row launch on the tensor cores and one 1-row launch on the
+    CUDA cores."""
+    X, W, s, b = _case(M, K, N, 51 + M, True, True)
+    L = svdq.W4A16Layer(W, s=s, bias=b, device="cuda")
+    Y = L.linear(_dev(X))
+    torch.cuda.synchronize()
+    ref = W4.prepare(W.astype(np.float32), s=s, bias=b.astype(np.float32))
+    err = S.max_rel_err(y_to_f64(Y), W4.linear(ref, X.astype(np.float32)))
+    assert err <= Y_TOL, err
 
 
 @pytest.mark.parametrize("M", [1, 2, 4])
