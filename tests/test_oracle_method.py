@@ -75,6 +75,32 @@ def test_quantizer_error_within_half_grid_spacing():
         assert np.all(np.abs(q - v) <= bound + 1e-12)
 
 
+@settings(max_examples=60, deadline=None)
+@given(seed=st.integers(0, 2**31 - 1), log_scale=st.floats(-20, 20), spread=st.integers(0, 12),
+       zeros=st.floats(0, 0.5))
+def test_quantizer_error_bound_on_random_blocks(seed, log_scale, spread, zeros):
+    """Every element lands within half the local E2M1 grid spacing of t / d
+    (0.25 below 2, 0.5 below 4, 1 above), or on 6 when t / d exceeds 6; a block
+    with d = 0 has only zero codes.  Random magnitudes over 40 binades, blocks
+    whose scales differ by up to 2^12, and exact zeros."""
+    g0 = np.random.default_rng(seed)
+    t = g0.standard_normal((8, 256)) * np.exp2(log_scale)
+    t = t * np.exp2(g0.integers(-spread, spread + 1, size=(8, 16, 1))).repeat(16, axis=2).reshape(8, 256)
+    t[g0.random(t.shape) < zeros] = 0.0
+    t = t.astype(np.float32)
+    g = S.global_scale(np.max(np.abs(t)))
+    codes, scales = S.nvfp4_quantize(t, g)
+    d = (F.e4m3_decode(scales).astype(np.float32) * g).astype(np.float64)  # [8, 16]
+    v = np.abs(t.astype(np.float64)).reshape(8, 16, 16)
+    q = np.abs(F.e2m1_decode(codes)).reshape(8, 16, 16)
+    zero = d == 0
+    assert np.all(q[zero] == 0)
+    r = v[~zero] / d[~zero][:, None]
+    half = np.where(r < 2, 0.25, np.where(r < 4, 0.5, 1.0))
+    bound = np.where(r > 6, r - 6, half) * (1 + 1e-6)
+    assert np.all(np.abs(q[~zero] - r) <= bound + 1e-12)
+
+
 def test_scales_fit_e4m3_under_global_scale():
     t = np.random.default_rng(5).standard_normal((64, 256)).astype(np.float32) * 7
     g = S.global_scale(np.max(np.abs(t)))
