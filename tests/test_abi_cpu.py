@@ -210,3 +210,35 @@ def test_binding_refuses_tensors_the_abi_cannot_check():
             f()
     with pytest.raises(ValueError):
         svdq.rope_pack(torch.zeros((4, 64, 2), dtype=torch.float32))  # host memory
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include "svdq.h"
+
+int main(void) {
+  svdq_prepare_desc d = {0};
+  size_t bytes = 1;
+  if (svdq_abi_version() != SVDQ_ABI_VERSION) return 1;
+  if (svdq_layer_device_bytes(&d) != 0) return 2;             /* W missing: refused, size 0 */
+  if (svdq_rope_packed_bytes(128, 128, &bytes) != SVDQ_OK || bytes == 0) return 3;
+  if (svdq_quantize_act(NULL, NULL, 1, NULL, 0, NULL) != SVDQ_ERR_INVALID_ARGUMENT) return 4;
+  printf("%s\n", svdq_last_error());
+  return 0;
+}
+"""
+
+
+@pytest.mark.skipif(subprocess.run(["which", "gcc"], capture_output=True).returncode != 0, reason="needs gcc")
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    """include/svdq.h compiles as strict C99 and a C program links against
+    libsvdq.so and calls it (host-only entry points; no CUDA call)."""
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    lib_dir = os.path.dirname(svdq.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I" + os.path.join(ROOT, "include"),
+                    str(src), "-L" + lib_dir, "-lsvdq", "-Wl,-rpath," + lib_dir, "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.strip()  # the refusal left its message in svdq_last_error()
