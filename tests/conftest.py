@@ -2,6 +2,11 @@ import os
 import sys
 
 import pytest
+from hypothesis import settings
+
+# property tests draw the same examples on every run, so the suite's result does not depend on the run
+settings.register_profile("repo", derandomize=True, database=None)
+settings.load_profile("repo")
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
