@@ -272,13 +272,16 @@ svdq_status svdq_w4a4_linear_qkv_norm_rope(const svdq_layer* L, const void* act_
 }
 
 svdq_status svdq_lora_swap(svdq_layer* L, const void* A, const void* B, int32_t r_e, float scale, void* stream) {
-  svdq_status st = check_uploaded(L);
-  if (st != SVDQ_OK) return st;
+  if (!L) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is NULL");
   if (r_e < 0 || r_e % 16) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "LoRA rank must be a multiple of 16");
   if (L->g.rank + r_e > L->g.rcap)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank + LoRA rank exceeds rank_capacity (" + std::to_string(L->g.rcap) + ")");
   if (r_e > 0 && (!A || !B)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "A and B are required");
+  if (r_e > 0 && (!aligned(A, 2) || !aligned(B, 2)))
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "A and B must be 2-byte aligned (bf16 elements)");
   if (!std::isfinite(scale)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "scale must be finite");
+  svdq_status st = check_uploaded(L);
+  if (st != SVDQ_OK) return st;
   svdq::LoraLaunch a{};
   a.layer = static_cast<uint8_t*>(L->dev_buf);
   a.lg = L->g;

@@ -228,7 +228,7 @@ SVDQ_API svdq_status svdq_rope_pack(const void* rope, int64_t M, int32_t head_di
 /*
  * Attach a LoRA adapter to the low-rank branch without touching R (abstract of
  * arXiv 2411.05007: off-the-shelf LoRAs without re-quantization).  Device
- * bf16 A [K, r_e] and B [r_e, N] (row-major); the layer computes
+ * bf16 A [K, r_e] and B [r_e, N] (row-major, 2-byte aligned); the layer computes
  * Y += scale X A B by storing L1' = [L1 | bf16(lambda A scale)], L2' = [L2 ; B].
  * r_e = 0 detaches the current adapter.  rank + r_e <= rank_capacity.
  * Stream ordered, no host synchronization; calls on `layer` issued after this

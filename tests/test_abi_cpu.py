@@ -76,6 +76,25 @@ def test_prepare_rejects_bad_calibration_maxima(bad):
     assert svdq.lib().svdq_layer_device_bytes(ctypes.byref(d)) == 0
 
 
+def test_lora_swap_checks_its_arguments_before_the_device():
+    """Shape, capacity, missing and misaligned adapters and the scale are
+    refused from the arguments alone (no pointer is read), before the layer's
+    device state is looked at."""
+    spec = WL.CFG1
+    layer = svdq.Layer(spec.w(), svdq.calibrate_amax(spec.x()), 16, rank_capacity=48)
+    lib = svdq.lib()
+    h = layer._h
+    assert lib.svdq_lora_swap(h, 64, 128, 8, 1.0, None) == svdq.ERR_UNSUPPORTED_SHAPE  # not a multiple of 16
+    assert lib.svdq_lora_swap(h, 64, 128, 48, 1.0, None) == svdq.ERR_UNSUPPORTED_SHAPE  # 16 + 48 > 48
+    assert lib.svdq_lora_swap(h, None, 128, 16, 1.0, None) == svdq.ERR_INVALID_ARGUMENT
+    assert lib.svdq_lora_swap(h, 65, 128, 16, 1.0, None) == svdq.ERR_INVALID_ARGUMENT
+    assert "aligned" in svdq.last_error()
+    assert lib.svdq_lora_swap(h, 64, 129, 16, 1.0, None) == svdq.ERR_INVALID_ARGUMENT
+    assert lib.svdq_lora_swap(h, 64, 128, 16, float("inf"), None) == svdq.ERR_INVALID_ARGUMENT
+    assert lib.svdq_lora_swap(h, 64, 128, 16, 1.0, None) == svdq.ERR_INVALID_ARGUMENT  # valid, but not uploaded
+    assert "uploaded" in svdq.last_error()
+
+
 def test_null_arguments_are_errors_not_crashes():
     L = svdq.lib()
     assert L.svdq_prepare_host(None, None) == svdq.ERR_INVALID_ARGUMENT
