@@ -743,6 +743,37 @@ def run_reference(args):
     return 0
 
 
+def _free_port():
+    import socket
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_command(nproc, argv, port):
+    """The torch.distributed.run command that starts `nproc` ranks of this script with `argv`."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={nproc}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + list(argv)
+
+
+def relaunch(args, argv):
+    """`--gpus N` (N > 1) started as a plain process: start N ranks under torch.distributed.run
+    and return its exit status, so a multi-GPU run never silently measures one replica.  Our arm
+    refuses at once when fewer than N GPUs are visible; the reference arm runs on rank 0's host
+    cores and needs none."""
+    if args.impl == "ours":
+        import torch
+
+        have = torch.cuda.device_count()
+        if have < args.gpus:
+            raise SystemExit(f"--gpus {args.gpus} but only {have} CUDA device(s) are visible")
+    cmd = relaunch_command(args.gpus, argv, _free_port())
+    sys.stdout.flush()
+    return subprocess.run(cmd, env={k: v for k, v in os.environ.items() if k not in
+                                    ("RANK", "WORLD_SIZE", "LOCAL_RANK", "LOCAL_WORLD_SIZE")}).returncode
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -761,9 +792,13 @@ def main(argv=None):
         return run_sweep(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
     _, world, _ = dist_env()
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(args, sys.argv[1:] if argv is None else list(argv))
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -75,3 +75,41 @@ def test_single_process_helpers_are_identities():
     assert bench.aggregate(10.0, 1, 2.0) == 5.0
     assert bench.rank_seed(7, 0) == 7
     bench.barrier()  # no process group: a no-op
+
+
+def _bench(argv, timeout=300):
+    import subprocess
+
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + argv, capture_output=True, text=True,
+                          timeout=timeout, env=env, cwd=ROOT)
+
+
+def test_plain_launch_with_several_gpus_starts_one_rank_each():
+    """`bench.py --gpus 2` run as a plain process starts two ranks under torch.distributed.run;
+    the reference arm needs no GPU, so the whole launch runs here: rank 0 prints the one line,
+    with n_gpus = 2."""
+    import json
+
+    r = _bench(["--gpus", "2", "--impl", "reference", "--workload", "cfg1", "--steps", "1", "--warmup", "3",
+                "--cpu-budget", "0.5"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    out = json.loads(lines[0])
+    assert out["impl"] == "reference" and out["n_gpus"] == 2
+
+
+def test_plain_launch_refuses_more_gpus_than_visible():
+    """Our arm with more ranks than visible GPUs fails loudly instead of measuring one replica."""
+    r = _bench(["--gpus", "2", "--steps", "1", "--warmup", "3"], timeout=120)
+    assert r.returncode != 0
+    assert "CUDA device" in r.stderr
+    assert "{" not in r.stdout
+
+
+def test_relaunch_command_names_every_rank_and_the_loopback_address():
+    cmd = bench.relaunch_command(4, ["--gpus", "4", "--steps", "5"], 29500)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd and "--master-port=29500" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "5"]
