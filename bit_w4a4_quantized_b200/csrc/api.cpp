@@ -70,6 +70,28 @@ svdq_status check_uploaded(const svdq_layer* L) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Note that act_buf now holds activations quantized under the handle's current factors.
+void note_act(const svdq_layer* L, const void* act_buf) {
+  auto& N = L->notes;
+  std::lock_guard<std::mutex> lk(N.mu);
+  for (auto& n : N.ring)
+    if (n.buf == act_buf) {
+      n.gen = L->swap_gen;
+      return;
+    }
+  N.ring[N.next] = {act_buf, L->swap_gen};
+  N.next = (N.next + 1) % svdq_layer::ActNotes::kSize;
+}
+
+// True when act_buf was last quantized through this handle under other low-rank factors.
+bool act_is_stale(const svdq_layer* L, const void* act_buf) {
+  auto& N = L->notes;
+  std::lock_guard<std::mutex> lk(N.mu);
+  for (const auto& n : N.ring)
+    if (n.buf == act_buf) return n.gen != L->swap_gen;
+  return false;
+}
+
 }  // namespace
 
 extern "C" {
@@ -175,6 +197,7 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   const char* why = "";
   cudaError_t e = svdq::launch_act_quant(a, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
+  note_act(L, act_buf);
   return SVDQ_OK;
 }
 
@@ -194,6 +217,9 @@ svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_b
   if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");
   if (M * L->g.N > (int64_t(1) << 31) * 2 || M > (int64_t(1) << 31) - 1)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M too large");
+  if (act_is_stale(L, act_buf))
+    return fail(SVDQ_ERR_INVALID_ARGUMENT,
+                "act_buf was quantized before the layer's last LoRA swap; quantize X again (svdq_quantize_act)");
   if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
   svdq::GemmLaunch a = qkv ? *qkv : svdq::GemmLaunch{};
   a.act = static_cast<const uint8_t*>(act_buf);
@@ -274,7 +300,7 @@ svdq_status svdq_w4a4_linear_qkv_norm_rope(const svdq_layer* L, const void* act_
 svdq_status svdq_lora_swap(svdq_layer* L, const void* A, const void* B, int32_t r_e, float scale, void* stream) {
   if (!L) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is NULL");
   if (r_e < 0 || r_e % 16) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "LoRA rank must be a multiple of 16");
-  if (L->g.rank + r_e > L->g.rcap)
+  if (r_e > L->g.rcap - L->g.rank)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank + LoRA rank exceeds rank_capacity (" + std::to_string(L->g.rcap) + ")");
   if (r_e > 0 && (!A || !B)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "A and B are required");
   if (r_e > 0 && (!aligned(A, 2) || !aligned(B, 2)))
@@ -292,6 +318,7 @@ svdq_status svdq_lora_swap(svdq_layer* L, const void* A, const void* B, int32_t 
   cudaError_t e = svdq::launch_lora_swap(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "launch of the LoRA swap kernel");
   L->r_tot = L->g.rank + r_e;
+  ++L->swap_gen;
   return SVDQ_OK;
 }
 

@@ -3,6 +3,7 @@
 
 #include <stdint.h>
 
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -20,6 +21,26 @@ struct svdq_layer {
   double resid_f64 = -1.0, resid_bf16 = -1.0;
   float g_a = 1.f, g_w = 1.f, alpha = 1.f, inv_alpha = 1.f, c_a = 1.f;
   int32_t r_tot = 0;  // ranks in use: base rank + attached adapter rank
+  // Which low-rank factors the activation buffers were last filled under.  Every LoRA swap
+  // bumps swap_gen; svdq_quantize_act notes (buffer, swap_gen) in a small ring, and the
+  // linear calls refuse a noted buffer whose generation differs from the handle's, since its
+  // lr' columns were computed with the factors the swap replaced.  A copy of the handle
+  // starts with no notes.
+  struct ActNotes {
+    static constexpr int kSize = 64;
+    struct Note {
+      const void* buf = nullptr;
+      uint64_t gen = 0;
+    };
+    std::mutex mu;
+    Note ring[kSize];
+    int next = 0;
+    ActNotes() = default;
+    ActNotes(const ActNotes&) {}
+    ActNotes& operator=(const ActNotes&) { return *this; }
+  };
+  mutable ActNotes notes;
+  uint64_t swap_gen = 0;
   bool has_bias = false;
   // device state (after upload)
   void* dev_buf = nullptr;

@@ -174,7 +174,11 @@ SVDQ_API svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, i
  * section): Y = act(g_a g_w (Q(X_hat) Q(R) + lr' L2) + b) with the FP4
  * block-scaled MMA and the bf16 up projection accumulating into the same
  * tensor-memory tile.
- * act_buf: the buffer svdq_quantize_act filled for the same M.
+ * act_buf: the buffer svdq_quantize_act filled for the same M, through this
+ *   handle, after its last svdq_lora_swap.  The handle notes the last 64 act_bufs
+ *   it filled; one of those filled before a later swap holds lr' columns of the
+ *   replaced factors, and is refused with SVDQ_ERR_INVALID_ARGUMENT (quantize X
+ *   again).  A buffer filled through another handle is not checked.
  * Y: device bf16 [M, N] row-major, 32-byte aligned.
  * epilogue: SVDQ_EPI_NONE or SVDQ_EPI_GELU_TANH (bias is added first).
  */
@@ -232,8 +236,10 @@ SVDQ_API svdq_status svdq_rope_pack(const void* rope, int64_t M, int32_t head_di
  * Y += scale X A B by storing L1' = [L1 | bf16(lambda A scale)], L2' = [L2 ; B].
  * r_e = 0 detaches the current adapter.  rank + r_e <= rank_capacity.
  * Stream ordered, no host synchronization; calls on `layer` issued after this
- * one (on any stream ordered after s) see the new rank.  Not thread safe
- * against concurrent calls on the same handle.
+ * one (on any stream ordered after s) see the new rank.  Activation buffers
+ * filled before the swap must be filled again before the next linear call (the
+ * linear calls refuse them).  Not thread safe against concurrent calls on the
+ * same handle.
  */
 SVDQ_API svdq_status svdq_lora_swap(svdq_layer* layer, const void* A, const void* B, int32_t r_e, float scale,
                            void* stream);

@@ -15,6 +15,7 @@ from oracle import formats as F
 from oracle import svdquant as S
 
 Y_TOL = 1e-2       # max|Y - Y_ref| / max|Y_ref| (the layer tolerance)
+ROW_TOL = 1e-2     # the same bound per row, each row against its own max (floored at 0.1 rms of Y_ref)
 LR_TOL = 2.0**-7   # lr' is rounded to bf16 once: relative error <= 2^-9, margin for fp32 sums
 
 
@@ -78,11 +79,52 @@ def check_act(case, act, rows=None):
     return ref
 
 
-def check_y(case, Y, ref_act, epilogue=svdq.EPI_NONE, rows=None):
+def row_rel_err(y, y_ref):
+    """max over rows i of max_j|y - y_ref|_ij / max(max_j|y_ref|_ij, 0.1 rms(y_ref)).
+
+    The global bound divides by the tensor's max, which a few outlier rows set; a whole tile of
+    small outputs could be off by percents of its own scale under it.  Here each row answers to
+    its own scale, floored at a tenth of the tensor's rms so that rows of near-zero outputs are
+    held to an absolute bound instead of a relative one."""
+    y = np.asarray(y, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    if y_ref.size == 0:
+        return 0.0
+    floor = 0.1 * float(np.sqrt(np.mean(y_ref * y_ref)))
+    den = np.maximum(np.max(np.abs(y_ref), axis=-1), floor)
+    den = np.where(den > 0, den, 1.0)
+    return float(np.max(np.max(np.abs(y - y_ref), axis=-1) / den))
+
+
+def elementwise_rel_err(y, y_ref):
+    """max |y - y_ref| / |y_ref| over the elements with |y_ref| >= 0.1 rms(y_ref) (a report, not a bound:
+    near zero crossings bf16 output rounding alone makes this ratio large)."""
+    y = np.asarray(y, np.float64)
+    y_ref = np.asarray(y_ref, np.float64)
+    if y_ref.size == 0:
+        return 0.0
+    rms = float(np.sqrt(np.mean(y_ref * y_ref)))
+    sel = np.abs(y_ref) >= 0.1 * rms
+    if not np.any(sel) or rms == 0:
+        return 0.0
+    return float(np.max(np.abs(y[sel] - y_ref[sel]) / np.abs(y_ref[sel])))
+
+
+def assert_y_close(y, y_ref, report=None):
+    """Both bounds on float64 arrays: the global max-norm one and the per-row one; returns the global."""
+    err = S.max_rel_err(y, y_ref)
+    assert err <= Y_TOL, err
+    rerr = row_rel_err(y, y_ref)
+    assert rerr <= ROW_TOL, rerr
+    if report is not None:
+        report.update(global_rel=err, row_rel=rerr, elementwise_rel=elementwise_rel_err(y, y_ref))
+    return err
+
+
+def check_y(case, Y, ref_act, epilogue=svdq.EPI_NONE, rows=None, report=None):
+    """Y against the oracle: the global bound and the per-row bound, both asserted; the
+    element-wise ratio is added to `report` (a dict) when one is given."""
     y = y_to_f64(Y)
     if rows is not None:
         y = y[rows]
-    y_ref = S.linear(case.ref, ref_act, epilogue)
-    err = S.max_rel_err(y, y_ref)
-    assert err <= Y_TOL, err
-    return err
+    return assert_y_close(y, S.linear(case.ref, ref_act, epilogue), report)

@@ -86,6 +86,8 @@ def test_lora_swap_checks_its_arguments_before_the_device():
     h = layer._h
     assert lib.svdq_lora_swap(h, 64, 128, 8, 1.0, None) == svdq.ERR_UNSUPPORTED_SHAPE  # not a multiple of 16
     assert lib.svdq_lora_swap(h, 64, 128, 48, 1.0, None) == svdq.ERR_UNSUPPORTED_SHAPE  # 16 + 48 > 48
+    # a rank whose sum with the base rank overflows int32 is still over capacity
+    assert lib.svdq_lora_swap(h, 64, 128, 2147483632, 1.0, None) == svdq.ERR_UNSUPPORTED_SHAPE
     assert lib.svdq_lora_swap(h, None, 128, 16, 1.0, None) == svdq.ERR_INVALID_ARGUMENT
     assert lib.svdq_lora_swap(h, 65, 128, 16, 1.0, None) == svdq.ERR_INVALID_ARGUMENT
     assert "aligned" in svdq.last_error()

@@ -13,7 +13,7 @@ import torch
 
 from bit_w4a4_quantized_b200 import svdq
 from bit_w4a4_quantized_b200 import workloads as WL
-from gpu_cases import Y_TOL, Case, check_act, y_to_f64
+from gpu_cases import Case, assert_y_close, check_act, y_to_f64
 from oracle import qkv as QO
 from oracle import svdquant as S
 
@@ -41,8 +41,7 @@ def _check(case, Yf, ref_act, host, rows=None):
     errs = []
     for part in range(3):
         cols = slice(part * C, (part + 1) * C)
-        err = S.max_rel_err(got[:, cols], want[:, cols])
-        assert err <= Y_TOL, (part, err)
+        err = assert_y_close(got[:, cols], want[:, cols])
         errs.append(err)
     return errs
 

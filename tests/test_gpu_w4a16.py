@@ -13,7 +13,7 @@ import torch
 
 from bit_w4a4_quantized_b200 import svdq
 from bit_w4a4_quantized_b200 import workloads as WL
-from gpu_cases import Y_TOL, y_to_f64
+from gpu_cases import assert_y_close, y_to_f64
 from oracle import svdquant as S
 from oracle import w4a16 as W4
 
@@ -43,8 +43,7 @@ def test_parity(M, K, N, with_s, with_bias):
     torch.cuda.synchronize()
     ref = W4.prepare(W.astype(np.float32), s=s, bias=None if b is None else b.astype(np.float32))
     want = W4.linear(ref, X.astype(np.float32))
-    err = S.max_rel_err(y_to_f64(Y), want)
-    assert err <= Y_TOL, err
+    err = assert_y_close(y_to_f64(Y), want)
     print(f"W4A16 M{M} K{K} N{N}: max rel err {err:.2e}")
 
 
@@ -60,8 +59,7 @@ def test_largest_k_and_several_passes_over_k(M, K, N):
     Y = L.linear(_dev(X))
     torch.cuda.synchronize()
     ref = W4.prepare(W.astype(np.float32), s=s, bias=b.astype(np.float32))
-    err = S.max_rel_err(y_to_f64(Y), W4.linear(ref, X.astype(np.float32)))
-    assert err <= Y_TOL, err
+    assert_y_close(y_to_f64(Y), W4.linear(ref, X.astype(np.float32)))
 
 
 @pytest.mark.parametrize("M", [1, 2, 4])
@@ -75,8 +73,7 @@ def test_modulation_shape_on_sampled_features(M):
     cols = np.sort(np.concatenate([[0, spec.N - 1], g.choice(spec.N, 512, replace=False)]))
     ref = W4.prepare(W.astype(np.float32), s=s, bias=b.astype(np.float32), rows=cols)
     want = W4.linear(ref, X.astype(np.float32))
-    err = S.max_rel_err(Y[:, cols], want)
-    assert err <= Y_TOL, err
+    err = assert_y_close(Y[:, cols], want)
     print(f"W4A16 modulation M{M}: max rel err {err:.2e}")
 
 

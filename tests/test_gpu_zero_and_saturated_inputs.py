@@ -22,7 +22,7 @@ from ml_dtypes import bfloat16
 
 from bit_w4a4_quantized_b200 import svdq
 from bit_w4a4_quantized_b200 import workloads as WL
-from gpu_cases import Case, check_act, check_y, y_to_f64
+from gpu_cases import Case, assert_y_close, check_act, check_y, y_to_f64
 from oracle import formats as F
 from oracle import svdquant as S
 
@@ -89,8 +89,7 @@ def test_activations_beyond_calibration_saturate(factor):
     np.testing.assert_array_equal(scales, ref.scales)
     lr_gpu = F.bf16_from_bits(lr).astype(np.float64) * case.ref.alpha
     assert np.max(np.abs(lr_gpu - ref.lr)) <= 2.0**-7 * np.max(np.abs(ref.lr))
-    err = S.max_rel_err(y_to_f64(Y), S.linear(case.ref, ref))
-    assert err <= 1e-2, err
+    assert_y_close(y_to_f64(Y), S.linear(case.ref, ref))
 
 
 def test_empty_batch_is_refused():
@@ -117,8 +116,7 @@ def _w4a16_check(X, W, s=None, bias=None):
     torch.cuda.synchronize()
     ref = W4.prepare(W.astype(np.float32), s=s, bias=None if bias is None else bias.astype(np.float32))
     want = W4.linear(ref, X.astype(np.float32))
-    err = S.max_rel_err(y_to_f64(Y), want)
-    assert err <= 1e-2, err
+    assert_y_close(y_to_f64(Y), want)
     return Y, ref
 
 
