@@ -23,7 +23,7 @@ CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 
 CU_SOURCES = ["act_quant.cu", "gemm.cu", "lora.cu", "w4a16.cu"]
-CPP_SOURCES = ["api.cpp", "prepare.cpp", "svd.cpp"]
+CPP_SOURCES = ["api.cpp", "blob.cpp", "prepare.cpp", "svd.cpp"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

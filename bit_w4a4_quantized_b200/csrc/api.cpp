@@ -393,6 +393,28 @@ svdq_status svdq_layer_clone(const svdq_layer* L, svdq_layer** out) {
   return SVDQ_OK;
 }
 
+svdq_status svdq_layer_serialize(const svdq_layer* L, void* host_dst, size_t bytes, size_t* bytes_needed) {
+  if (!L) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is NULL");
+  const size_t need = svdq::blob_bytes(L);
+  if (bytes_needed) *bytes_needed = need;
+  if (!host_dst) {
+    if (!bytes_needed) return fail(SVDQ_ERR_INVALID_ARGUMENT, "give host_dst or bytes_needed");
+    return SVDQ_OK;
+  }
+  std::string err;
+  svdq_status st = svdq::blob_write(L, static_cast<uint8_t*>(host_dst), bytes, &err);
+  if (st != SVDQ_OK) return fail(st, err);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_layer_import(const void* blob, size_t bytes, svdq_layer** out) {
+  if (!blob || !out) return fail(SVDQ_ERR_INVALID_ARGUMENT, "blob and out are required");
+  std::string err;
+  svdq_status st = svdq::blob_read(static_cast<const uint8_t*>(blob), bytes, out, &err);
+  if (st != SVDQ_OK) return fail(st, err);
+  return SVDQ_OK;
+}
+
 void svdq_test_override_device_arch(int sm) { g_arch_override.store(sm); }
 
 svdq_status svdq_test_bounded_wait(uint64_t timeout_ns, uint32_t* status_out, void* stream) {

@@ -57,6 +57,11 @@ svdq_status validate_desc(const svdq_prepare_desc* d, std::string* err);
 
 // Logical views of the image / of an activation buffer (prepare.cpp).
 svdq_status export_array(const svdq_layer* L, int what, void* dst, size_t bytes, std::string* err);
+// The flat, versioned blob of a prepared layer (blob.cpp).
+size_t blob_bytes(const svdq_layer* L);
+svdq_status blob_write(const svdq_layer* L, uint8_t* dst, size_t bytes, std::string* err);
+svdq_status blob_read(const uint8_t* src, size_t bytes, svdq_layer** out, std::string* err);
+
 svdq_status act_unpack(const svdq_layer* L, int64_t M, const uint8_t* act, size_t bytes, uint8_t* codes,
                        uint8_t* scales, uint16_t* lr, std::string* err);
 

@@ -49,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "svdq_test_bounded_wait", "svdq_layer_clone", "svdq_w4a4_linear_qkv_norm_rope",
     "svdq_rope_packed_bytes", "svdq_rope_pack", "svdq_w4a16_device_bytes", "svdq_w4a16_prepare_host",
     "svdq_w4a16_upload", "svdq_w4a16_linear", "svdq_w4a16_export", "svdq_w4a16_destroy",
+    "svdq_layer_serialize", "svdq_layer_import",
 )
 
 
@@ -121,6 +122,8 @@ def lib():
         "svdq_poll_status": ([vp, vp], st),
         "svdq_layer_destroy": ([vp], None),
         "svdq_layer_clone": ([vp, ctypes.POINTER(vp)], st),
+        "svdq_layer_serialize": ([vp, vp, sz, ctypes.POINTER(sz)], st),
+        "svdq_layer_import": ([vp, sz, ctypes.POINTER(vp)], st),
         "svdq_w4a16_device_bytes": ([ctypes.POINTER(W4A16Desc)], sz),
         "svdq_w4a16_prepare_host": ([ctypes.POINTER(W4A16Desc), ctypes.POINTER(vp)], st),
         "svdq_w4a16_upload": ([vp, vp, sz, vp], st),
@@ -286,6 +289,29 @@ class Layer:
         c = Layer.__new__(Layer)
         c._h, c._keep, c.desc = h, None, self.desc
         c.N, c.K, c.rank, c.device_bytes, c.dev_buf = self.N, self.K, self.rank, self.device_bytes, None
+        if device is not None:
+            c.upload(device, stream)
+        return c
+
+    def serialize(self):
+        """The prepared layer as one flat, versioned blob (bytes), for a checkpoint."""
+        n = ctypes.c_size_t()
+        check(lib().svdq_layer_serialize(self._h, None, 0, ctypes.byref(n)))
+        buf = ctypes.create_string_buffer(n.value)
+        check(lib().svdq_layer_serialize(self._h, buf, n.value, ctypes.byref(n)))
+        return buf.raw[:n.value]
+
+    @classmethod
+    def from_blob(cls, blob, device=None, stream=None):
+        """A layer from a blob that ``serialize`` wrote: no SVD and no quantization run."""
+        h = ctypes.c_void_p()
+        b = bytes(blob)
+        check(lib().svdq_layer_import(b, len(b), ctypes.byref(h)))
+        c = cls.__new__(cls)
+        c._h, c._keep, c.desc, c.dev_buf = h, None, None, None
+        i = LayerInfo()
+        check(lib().svdq_get_layer_info(h, ctypes.byref(i)))
+        c.N, c.K, c.rank, c.device_bytes = i.N, i.K, i.rank, i.device_bytes
         if device is not None:
             c.upload(device, stream)
         return c
@@ -506,3 +532,61 @@ def test_bounded_wait(timeout_ns, stream=None):
 
 def override_device_arch(sm):
     lib().svdq_test_override_device_arch(int(sm))
+
+
+class HostPipeline:
+    """Forward passes of one layer over batches that live in host memory.
+
+    Each batch's X is copied in, run through both kernels and its Y copied out.  Two slots
+    (device X, activation buffer and Y each) and three streams let the host-to-device copy of
+    batch i + 1 and the device-to-host copy of batch i - 1 run in both directions of the link
+    while batch i computes.  Host tensors should be pinned, or the copies do not overlap.
+    Stream and copy plumbing only: the layer's kernels do the work."""
+
+    def __init__(self, layer, M, epilogue=EPI_NONE):
+        import torch
+
+        dev = layer._device()
+        self.layer, self.M, self.epilogue = layer, M, epilogue
+        self.X = [torch.empty((M, layer.K), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.act = [layer.new_act_buffer(M) for _ in range(2)]
+        self.Y = [torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.h2d_bytes = 2 * M * layer.K
+        self.d2h_bytes = 2 * M * layer.N
+
+    def run(self, xs_host, ys_host):
+        """Y_i = layer(X_i) for host bf16 X_i [M, K] into host bf16 Y_i [M, N]; returns once
+        every copy is queued (the last one is done when `done_event()` is)."""
+        import torch
+
+        n = len(xs_host)
+        if len(ys_host) != n:
+            raise ValueError("xs_host and ys_host differ in length")
+        ran = [None] * n
+        out = [None] * n
+        for i in range(n):
+            j = i % 2
+            with torch.cuda.stream(self.s_in):
+                if i >= 2:
+                    self.s_in.wait_event(ran[i - 2])  # slot j's X and act are free
+                self.X[j].copy_(xs_host[i], non_blocking=True)
+                copied = torch.cuda.Event()
+                copied.record(self.s_in)
+            with torch.cuda.stream(self.s_run):
+                self.s_run.wait_event(copied)
+                if i >= 2:
+                    self.s_run.wait_event(out[i - 2])  # slot j's Y has been read out
+                self.layer.forward(self.X[j], out=self.Y[j], epilogue=self.epilogue, act=self.act[j],
+                                   stream=self.s_run)
+                ran[i] = torch.cuda.Event()
+                ran[i].record(self.s_run)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(ran[i])
+                ys_host[i].copy_(self.Y[j], non_blocking=True)
+                out[i] = torch.cuda.Event()
+                out[i].record(self.s_out)
+        self._last = out[n - 1] if n else None
+
+    def done_event(self):
+        return self._last

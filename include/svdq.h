@@ -271,6 +271,27 @@ SVDQ_API svdq_status svdq_layer_export(const svdq_layer* layer, int what, void* 
 SVDQ_API svdq_status svdq_act_unpack(const svdq_layer* layer, int64_t M, const void* act_host, size_t bytes,
                             uint8_t* codes, uint8_t* scales, uint16_t* lr);
 
+/*
+ * The prepared layer as one flat, versioned host blob: what a checkpoint
+ * stores in place of W (the Diffusers/Nunchaku page, the sections on loading a
+ * quantized checkpoint with its quantization_config: a quantized model is
+ * saved and loaded without quantizing again).  The blob holds the device image
+ * in its base state (rank r, no adapter: an attached LoRA is not saved), the
+ * smoothing factors, the bf16 factors L1 and L2, the scalars and, when the
+ * library's SVD made the factors, the singular values; a 64-bit FNV-1a
+ * checksum covers everything after its 128-byte header.  Host only.
+ * svdq_layer_serialize: with host_dst NULL, only *bytes_needed is set; else
+ *   writes the blob (SVDQ_ERR_BUFFER_TOO_SMALL if bytes is short).  R itself
+ *   (SVDQ_EXPORT_R) is not saved.
+ * svdq_layer_import: a new host handle from a blob (validated: magic, version,
+ *   shape, section sizes, checksum; SVDQ_ERR_INVALID_ARGUMENT or
+ *   SVDQ_ERR_UNSUPPORTED_SHAPE otherwise); upload it with svdq_layer_upload.
+ *   The caller keeps ownership of the blob and may free it on return.
+ */
+SVDQ_API svdq_status svdq_layer_serialize(const svdq_layer* layer, void* host_dst, size_t bytes,
+                                          size_t* bytes_needed);
+SVDQ_API svdq_status svdq_layer_import(const void* blob, size_t bytes, svdq_layer** out);
+
 typedef struct svdq_layer_info {
   int64_t K, N;
   int32_t rank, rank_total, rank_capacity, format;

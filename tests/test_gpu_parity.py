@@ -364,3 +364,19 @@ def test_graph_replay_of_the_bench_step_matches_direct_launches():
     for L in layers:
         L.poll_status()
     del graph
+
+
+def test_layer_imported_from_a_blob_gives_the_same_output():
+    """A checkpoint round trip: serialize, import, upload; the imported layer's activation buffer
+    and Y are bit-identical to the original's, and within tolerance of the oracle."""
+    spec = WL.CFG1
+    case = _spec_case(spec)
+    act0, Y0 = case.run()
+    b = svdq.Layer.from_blob(case.layer.serialize(), device="cuda")
+    act1 = b.quantize_act(case.Xd)
+    Y1 = b.linear(act1, spec.M)
+    torch.cuda.synchronize()
+    assert torch.equal(act0, act1)
+    assert torch.equal(Y0.view(torch.int16), Y1.view(torch.int16))
+    check_y(case, Y1, check_act(case, act1))
+    b.poll_status()
