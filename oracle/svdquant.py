@@ -338,6 +338,23 @@ def forward(layer, X, epilogue=EPI_NONE):
     return linear(layer, quantize_act(layer, X), epilogue)
 
 
+def mlp_pair(layer1, layer2, X):
+    """Two layers of a transformer MLP run as one fused pair (Diffusers/Nunchaku page, the
+    fused GELU/MLP path of the 4-bit kernel family).  Fusion moves where fc2's activation
+    quantization happens (into fc1's output tile), not what it computes, so the pair is the
+    composition of the two layers:
+
+        h    = bf16(GELU(fc1(X)))        fc1's output in its output type, rounded once
+        act2 = quantize_act(fc2, h)      fc2's smoothing, NVFP4 codes and scales, h_hat L1
+        Y    = linear(fc2, act2)
+
+    Returns (h as float32 holding bf16 values, act2, Y in float64).
+    """
+    h = bf16_from_f64(forward(layer1, X, EPI_GELU_TANH)).astype(np.float32)
+    act2 = quantize_act(layer2, h)
+    return h, act2, linear(layer2, act2)
+
+
 # --------------------------------------------------------------------------
 # error measures (section 4.1, "Problem formulation")
 # --------------------------------------------------------------------------
