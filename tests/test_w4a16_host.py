@@ -75,3 +75,20 @@ def test_host_quantization_matches_the_oracle_on_random_layers(kt, n, seed, with
     np.testing.assert_array_equal(L.export(svdq.EXPORT_W_SCALES), ref.scales)
     assert L.export(svdq.EXPORT_SCALARS)[0] == ref.g
     L.close()
+
+
+def test_modulation_workloads_stay_in_the_f16_operand_range():
+    """The W4A16 layer rounds x / s to f16 (not bf16): values above 65504 would saturate and values below
+    2^-14 would lose bits.  Every modulation workload's nonzero |x / s| lies inside [2^-14, 65504] up to a
+    handful of tiny values, so the f16 operand changes nothing there."""
+    from bit_w4a4_quantized_b200 import workloads as WL
+
+    for N in (18432, 9216):
+        for M in (1, 2, 4, 8):
+            spec = WL.w4a16_spec(M, N=N)
+            x = spec.x().astype(np.float64)
+            inv = (np.float32(1.0) / spec.s().astype(np.float32)).astype(np.float64)
+            v = np.abs(x * inv[None, :])
+            assert v.max() < 65504.0
+            nz = v[v > 0]
+            assert np.mean(nz < 2.0**-14) < 1e-3
