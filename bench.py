@@ -687,6 +687,80 @@ def w4a16_point(spec, device, steps):
     return out
 
 
+def mlp_pair_point(device, steps):
+    """The MLP pair of the workload (fc1 3072 -> 12288 with GELU, fc2 12288 -> 3072, M = 4608, rank 32):
+    the unfused pair (fc1's output written and read back) against the fused pair (fc1's epilogue
+    writes fc2's activation buffer, then the partial-sum reduction), both over rotating buffer sets."""
+    import torch
+
+    from bit_w4a4_quantized_b200 import svdq
+    from bit_w4a4_quantized_b200 import workloads as WL
+
+    s1, s2 = WL.CFG3_FC1, WL.CFG3_FC2
+    M = s1.M
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.uint16).astype(np.int16)).view(
+        torch.bfloat16).to(device)
+    X = s1.x()
+    amax1 = svdq.calibrate_amax(X)
+    g = np.random.default_rng([s1.seed, 99])
+    # random bf16 factors stand in for the SVD (timing does not depend on their values)
+    fac = lambda K, N, r: (WL.to_bf16(g.normal(0, 0.05, (K, r))), WL.to_bf16(g.normal(0, 0.05, (r, N))))
+    fc1 = svdq.Layer(s1.w(), amax1, s1.rank, factors=fac(s1.K, s1.N, s1.rank), device=device)
+    # fc2's calibration: the GELU output of fc1 on the batch, from the library's own unfused pass
+    act = fc1.quantize_act(to_dev(X))
+    h = fc1.linear(act, M, epilogue=svdq.EPI_GELU_TANH)
+    hb = h.view(torch.int16).cpu().numpy().view(np.uint16)
+    amax2 = svdq.calibrate_amax(hb.view(WL.BF16))
+    fc2 = svdq.Layer(s2.w(), amax2, s2.rank, factors=fac(s2.K, s2.N, s2.rank), device=device)
+    nsets = 2
+    L1s = [fc1] + [fc1.clone(device=device) for _ in range(nsets - 1)]
+    L2s = [fc2] + [fc2.clone(device=device) for _ in range(nsets - 1)]
+    Xs = [to_dev(X) for _ in range(nsets)]
+    a1 = [L.new_act_buffer(M) for L in L1s]
+    a2 = [L.new_act_buffer(M) for L in L2s]
+    H = [torch.empty((M, s1.N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+    Y = [torch.empty((M, s2.N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+    ws = [torch.empty(fc1.mlp_workspace_bytes(fc2, M), dtype=torch.uint8, device=device) for _ in range(nsets)]
+    stream = torch.cuda.Stream(device)
+
+    def unfused(i):
+        L1s[i].quantize_act(Xs[i], a1[i])
+        L1s[i].linear(a1[i], M, out=H[i], epilogue=svdq.EPI_GELU_TANH)
+        L2s[i].quantize_act(H[i], a2[i])
+        L2s[i].linear(a2[i], M, out=Y[i])
+
+    def fused(i):
+        L1s[i].quantize_act(Xs[i], a1[i])
+        L1s[i].linear_mlp(a1[i], M, L2s[i], act2=a2[i], workspace=ws[i])
+        L2s[i].linear(a2[i], M, out=Y[i])
+
+    def fused_gemm(i):
+        L1s[i].linear_mlp(a1[i], M, L2s[i], act2=a2[i], workspace=ws[i])
+
+    def plain_gemm(i):
+        L1s[i].linear(a1[i], M, out=H[i], epilogue=svdq.EPI_GELU_TANH)
+
+    with torch.cuda.stream(stream):
+        for i in range(nsets):
+            unfused(i)
+            fused(i)
+        stream.synchronize()
+    out = {"workload": "mlp_pair_M4608_3072_12288_3072_r32", "M": M, "fc1": [s1.K, s1.N], "fc2": [s2.K, s2.N]}
+    for tag, fn in (("unfused_pair", unfused), ("fused_pair", fused), ("fc1_gemm_plain", plain_gemm),
+                    ("fc1_gemm_mlp_fused", fused_gemm)):
+        gr = _capture([lambda i=i: fn(i) for i in range(nsets)], stream)
+        out[f"{tag}_us"] = round(_graph_seconds(gr, nsets, steps, stream, device) * 1e6, 3)
+        del gr
+    flops = 2 * M * (s1.N * s1.K + s2.N * s2.K)
+    out["unfused_pair_TFLOPs"] = round(flops / out["unfused_pair_us"] / 1e6, 1)
+    out["fused_pair_TFLOPs"] = round(flops / out["fused_pair_us"] / 1e6, 1)
+    out["fused_speedup"] = round(out["unfused_pair_us"] / out["fused_pair_us"], 3)
+    for L in L1s + L2s:
+        L.poll_status()
+        L.close()
+    return out
+
+
 def run_sweep(args):
     import torch
 
@@ -703,13 +777,17 @@ def run_sweep(args):
             specs += WL.sweep()
         elif n == "w4a16":
             specs += [WL.w4a16_spec(m, N=nn) for nn in (18432, 9216) for m in (1, 2, 4)]
+        elif n == "mlp":
+            specs.append("mlp")
         else:
             specs.append(workload_spec(n))
     cache = {}
     props = torch.cuda.get_device_properties(device)
     for spec in specs:
         with ClockSampler(getattr(props, "uuid", None)) as clk:
-            if isinstance(spec, WL.W4A16Spec):
+            if spec == "mlp":
+                row = mlp_pair_point(device, args.sweep_steps)
+            elif isinstance(spec, WL.W4A16Spec):
                 row = w4a16_point(spec, device, args.sweep_steps)
             else:
                 row = sweep_point(spec, device, args.sweep_steps, cache)
@@ -784,7 +862,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", default=None,
-                    help="per-shape report instead of the bench line: 'all', 'sweep', 'w4a16' or workload names, "
+                    help="per-shape report instead of the bench line: 'all', 'sweep', 'w4a16', 'mlp' or workload names, "
                          "comma separated")
     ap.add_argument("--sweep-steps", type=int, default=50)
     args = ap.parse_args(argv)

@@ -29,6 +29,9 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "kernels.h"
 #include "ptx.cuh"
@@ -56,6 +59,8 @@ struct ActQuantParams {
   uint8_t* sf;           // act + off_sf
   uint8_t* lr;           // act + off_lr
   uint32_t* status;      // layer status word
+  uint32_t* sk_flags;    // the activation buffer's stream-K flags (cleared by CTA 0)
+  int32_t sk_flag_words;
   int32_t MT, KT, KC, RJ, r_tot, rc16, splits;
   int32_t push;          // split partials are pushed to the owning CTA (else pulled)
   int32_t rows_per;      // rows of a row tile each CTA of the cluster reduces
@@ -174,6 +179,8 @@ __global__ void __launch_bounds__(kThreads1, 2)
   // X may be the previous kernel's output and the activation buffer its input
   griddep_wait();
   griddep_launch_dependents();
+  if (blockIdx.x == 0 && blockIdx.y == 0)  // the GEMM's stream-K flags start cleared
+    for (int i = int(threadIdx.x); i < p.sk_flag_words; i += int(blockDim.x)) p.sk_flags[i] = 0u;
 
   auto fail = [&](uint32_t code) {
     *abort_flag = 1u;
@@ -463,6 +470,8 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   p.sf = a.act + ag.off_sf;
   p.lr = a.act + ag.off_lr;
   p.status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.layer) + lg.off_status);
+  p.sk_flags = a.sk_flags;
+  p.sk_flag_words = a.sk_flags ? a.sk_flag_words : 0;
   p.MT = int32_t(ag.MT);
   p.KT = int32_t(lg.KT);
   p.KC = int32_t(lg.KC);
@@ -509,14 +518,25 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   size_t smem = 0;
   int push = 0, rows_per = kBM;
   uint32_t rb_bytes = 0;
+  // the split count is planned once per device and shape (it queries the runtime's cluster occupancy)
+  using PlanKey = std::tuple<int, int64_t, int32_t, int32_t, int>;
+  static std::mutex plan_mu;
+  static std::map<PlanKey, int> planned;
+  const PlanKey key{dev, ag.MT, p.KC, a.r_tot, a.num_sms};
+  int cached = 0;
+  {
+    std::lock_guard<std::mutex> lk(plan_mu);
+    auto it = planned.find(key);
+    if (it != planned.end()) cached = it->second;
+  }
   plan(1, &smem, &push, &rows_per, &rb_bytes);
   const int per_sm = smem <= 113 * 1024 ? 2 : 1;
-  int splits = int((int64_t(per_sm) * a.num_sms) / ag.MT);
+  int splits = cached > 0 ? cached : int((int64_t(per_sm) * a.num_sms) / ag.MT);
   const int max_splits = lowrank ? kMaxPushSplits : 64;
   if (splits > max_splits) splits = max_splits;
   if (splits > p.KC) splits = p.KC;
   if (splits < 1) splits = 1;
-  if (lowrank) {
+  if (lowrank && cached == 0) {
     static std::atomic<int> nonportable[64];
     if (nonportable[dev & 63].load() == 0) {
       // clusters of up to 16 CTAs for the pushed partials (small M, long K)
@@ -551,6 +571,11 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
           int64_t(clusters) >= ag.MT)
         break;
     }
+  }
+  if (cached == 0) {
+    std::lock_guard<std::mutex> lk(plan_mu);
+    if (planned.size() > 4096) planned.clear();
+    planned[key] = splits;
   }
   plan(splits, &smem, &push, &rows_per, &rb_bytes);
   p.splits = splits;

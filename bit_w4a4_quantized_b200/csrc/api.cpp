@@ -70,6 +70,32 @@ svdq_status check_uploaded(const svdq_layer* L) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The activation buffer of M rows: what kernel 1 writes (codes, scales, lr'), then the GEMM's
+// stream-K area sized for every CTA pair the device can run (half its SMs).
+struct ActLayout {
+  svdq::ActGeom ag;
+  size_t sk_off, sk_bytes, total;
+  int sk_pairs;
+};
+ActLayout act_layout(const svdq_layer* L, int64_t M) {
+  ActLayout o{};
+  o.ag = svdq::make_act_geom(L->g, M);
+  int sms = L->num_sms;
+  if (sms <= 0) {  // not uploaded yet: the current device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 0;
+    cudaGetLastError();  // a CPU-only process has no device: no stream-K area
+  }
+  o.sk_pairs = sms / 2;
+  const int64_t ntiles = (o.ag.MT / 2) * L->g.NT;
+  o.sk_off = o.ag.total;
+  o.sk_bytes = svdq::sk_area_bytes(ntiles, o.sk_pairs);
+  o.total = o.sk_off + o.sk_bytes;
+  return o;
+}
+
 // Note that act_buf now holds activations quantized under the handle's current factors.
 void note_act(const svdq_layer* L, const void* act_buf) {
   auto& N = L->notes;
@@ -167,7 +193,7 @@ svdq_status svdq_prepare_weights(const svdq_prepare_desc* d, void* dev_buf, size
 svdq_status svdq_act_buffer_bytes(const svdq_layer* L, int64_t M, size_t* bytes) {
   if (!L || !bytes) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and bytes are required");
   if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
-  *bytes = svdq::make_act_geom(L->g, M).total;
+  *bytes = act_layout(L, M).total;
   return SVDQ_OK;
 }
 
@@ -179,10 +205,15 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
   if (!aligned(X, 16)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "X must be 16-byte aligned");
   if (!aligned(act_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf must be 256-byte aligned");
-  const size_t need = svdq::make_act_geom(L->g, M).total;
+  const ActLayout lay = act_layout(L, M);
+  const size_t need = lay.total;
   if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");
   if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
   svdq::ActQuantLaunch a{};
+  if (lay.sk_bytes) {
+    a.sk_flags = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(act_buf) + lay.sk_off);
+    a.sk_flag_words = 2 * lay.sk_pairs;
+  }
   a.X = X;
   a.layer = static_cast<const uint8_t*>(L->dev_buf);
   a.act = static_cast<uint8_t*>(act_buf);
@@ -213,7 +244,8 @@ svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_b
     return fail(SVDQ_ERR_INVALID_ARGUMENT, "unknown epilogue");
   if (!aligned(Y, 32)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "Y must be 32-byte aligned");
   if (!aligned(act_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf must be 256-byte aligned");
-  const size_t need = svdq::make_act_geom(L->g, M).total;
+  const ActLayout lay = act_layout(L, M);
+  const size_t need = lay.total;
   if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");
   if (M * L->g.N > (int64_t(1) << 31) * 2 || M > (int64_t(1) << 31) - 1)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M too large");
@@ -233,6 +265,10 @@ svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_b
   a.alpha = L->alpha;
   a.num_sms = L->num_sms;
   a.timeout_ns = svdq::kDefaultTimeoutNs;
+  if (lay.sk_bytes) {  // the GEMM's scratch for the last wave's split tiles
+    a.sk_area = const_cast<uint8_t*>(static_cast<const uint8_t*>(act_buf)) + lay.sk_off;
+    a.sk_max_pairs = lay.sk_pairs;
+  }
   const char* why = "";
   cudaError_t e = svdq::launch_gemm(a, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
@@ -244,6 +280,86 @@ svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_b
 svdq_status svdq_w4a4_linear(const svdq_layer* L, const void* act_buf, size_t act_buf_bytes, int64_t M, void* Y,
                              int epilogue, void* stream) {
   return linear_launch(L, act_buf, act_buf_bytes, M, Y, epilogue, nullptr, stream);
+}
+
+svdq_status svdq_mlp_workspace_bytes(const svdq_layer* fc1, const svdq_layer* fc2, int64_t M, size_t* bytes) {
+  if (!fc1 || !fc2 || !bytes) return fail(SVDQ_ERR_INVALID_ARGUMENT, "fc1, fc2 and bytes are required");
+  if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
+  if (fc2->g.K != fc1->g.N) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "fc2's K must equal fc1's N");
+  *bytes = fc2->r_tot > 0 ? svdq::mlp_partial_bytes(fc1->g.NT, svdq::make_act_geom(fc1->g, M).MT, fc2->r_tot) : 0;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act1, size_t act1_bytes, int64_t M,
+                                 const svdq_layer* fc2, void* act2, size_t act2_bytes, void* workspace,
+                                 size_t workspace_bytes, int epilogue, void* stream) {
+  svdq_status st = check_uploaded(fc1);
+  if (st != SVDQ_OK) return st;
+  if ((st = check_uploaded(fc2)) != SVDQ_OK) return st;
+  if (!act1 || !act2) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act1 and act2 are required");
+  if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
+  if (M > (int64_t(1) << 31) - 1) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M too large");
+  if (epilogue != SVDQ_EPI_NONE && epilogue != SVDQ_EPI_GELU_TANH)
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "unknown epilogue");
+  if (fc2->g.K != fc1->g.N) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "fc2's K must equal fc1's N");
+  if (!aligned(act1, 256) || !aligned(act2, 256))
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "act1 and act2 must be 256-byte aligned");
+  const ActLayout lay2 = act_layout(fc2, M);
+  const size_t need1 = act_layout(fc1, M).total, need2 = lay2.total;
+  if (act1_bytes < need1) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act1 needs " + std::to_string(need1) + " bytes");
+  if (act2_bytes < need2) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act2 needs " + std::to_string(need2) + " bytes");
+  const svdq::ActGeom ag1 = svdq::make_act_geom(fc1->g, M);
+  const size_t needw = fc2->r_tot > 0 ? svdq::mlp_partial_bytes(fc1->g.NT, ag1.MT, fc2->r_tot) : 0;
+  if (needw > 0 && !workspace) return fail(SVDQ_ERR_INVALID_ARGUMENT, "workspace is required when fc2 has ranks");
+  if (needw > 0 && !aligned(workspace, 16)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "workspace must be 16-byte aligned");
+  if (workspace_bytes < needw)
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "workspace needs " + std::to_string(needw) + " bytes");
+  if (act_is_stale(fc1, act1))
+    return fail(SVDQ_ERR_INVALID_ARGUMENT,
+                "act1 was quantized before fc1's last LoRA swap; quantize X again (svdq_quantize_act)");
+  if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
+  svdq::GemmLaunch a{};
+  a.act = static_cast<const uint8_t*>(act1);
+  a.layer = static_cast<const uint8_t*>(fc1->dev_buf);
+  a.Y = nullptr;
+  a.lg = fc1->g;
+  a.M = M;
+  a.r_tot = fc1->r_tot;
+  a.has_bias = fc1->has_bias ? 1 : 0;
+  a.epilogue = epilogue;
+  a.alpha = fc1->alpha;
+  a.num_sms = fc1->num_sms;
+  a.timeout_ns = svdq::kDefaultTimeoutNs;
+  a.mlp_act2 = static_cast<uint8_t*>(act2);
+  a.mlp_layer2 = static_cast<const uint8_t*>(fc2->dev_buf);
+  a.mlp_lg2 = fc2->g;
+  a.mlp_r2 = fc2->r_tot;
+  a.mlp_g_a2 = fc2->g_a;
+  a.mlp_c_a2 = fc2->c_a;
+  a.mlp_partial = static_cast<float*>(workspace);
+  const char* why = "";
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = svdq::launch_gemm(a, s, &why);
+  if (e != cudaSuccess) return cuda_fail(e, why);
+  if (fc2->r_tot > 0 || lay2.sk_bytes) {  // lr'2, and fc2's stream-K flags cleared
+    const svdq::ActGeom ag2 = svdq::make_act_geom(fc2->g, M);
+    svdq::MlpReduceLaunch r{};
+    r.partial = static_cast<const float*>(workspace);
+    r.nt = int32_t(fc1->g.NT);
+    r.rows = ag1.MT * svdq::kBM;
+    r.r2 = fc2->r_tot;
+    r.inv_alpha2 = fc2->inv_alpha;
+    r.lr2 = static_cast<uint8_t*>(act2) + ag2.off_lr;
+    r.RJ2 = int32_t(ag2.RJ);
+    if (lay2.sk_bytes) {
+      r.sk_flags2 = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(act2) + lay2.sk_off);
+      r.sk_flag_words2 = 2 * lay2.sk_pairs;
+    }
+    e = svdq::launch_mlp_reduce(r, s);
+    if (e != cudaSuccess) return cuda_fail(e, "launch of the MLP partial reduction failed");
+  }
+  note_act(fc2, act2);
+  return SVDQ_OK;
 }
 
 svdq_status svdq_rope_packed_bytes(int64_t M, int32_t head_dim, size_t* bytes) {

@@ -88,17 +88,35 @@ constexpr uint32_t kNormBytes = kEpiWarps * 64 * 4;  // QKV: per epilogue warp, 
 // row-strided stores per instruction.  Two buffers per warp (one in the QKV
 // instance, whose exchange and weights take the room).
 constexpr uint32_t kYRows = 32, kYCols = 16, kYBufBytes = kYRows * kYCols * 2;
-template <bool kQkv>
+// The epilogue instances of the kernel.
+enum EpiKind : int {
+  kEpiPlain = 0,  // Y = bf16(act(alpha acc + b))
+  kEpiQkv = 1,    // fused Q | K | V: per-head RMSNorm of Q and K, rotary turn, V unchanged
+  kEpiMlp = 2,    // fused MLP pair: the next layer's NVFP4 activations instead of Y
+};
+// MLP instance: per epilogue warp, its 64 columns of the next layer's 1/lambda (float) and a
+// 1 KB staging buffer of 32 rows x 16 columns of x_hat (the A fragments of the down
+// projection).  After the down projection the four staging buffers of a lane quarter's warps
+// hold the 32 rows x 32 ranks of partial x_hat L1 the four warps sum.
+constexpr uint32_t kInv2Bytes = kEpiWarps * 64 * 4;
+constexpr uint32_t kStgBytes = kEpiWarps * 1024;
+constexpr uint32_t kRedBytes = 0;
+template <int kEpi>
 struct EpiSmem {
-  static constexpr int kYBufs = kQkv ? 1 : 2;
+  static constexpr bool kQkv = kEpi == kEpiQkv, kMlp = kEpi == kEpiMlp;
+  static constexpr int kYBufs = kMlp ? 0 : kQkv ? 1 : 2;
   static constexpr uint32_t kXch = kStages2 * kStage2 + kCtrl2 + kBiasBytes;  // QKV only
   static constexpr uint32_t kNorm = kXch + (kQkv ? kXchBytes : 0);
   static constexpr uint32_t kY = (kNorm + (kQkv ? kNormBytes : 0) + 1023u) & ~1023u;
-  static constexpr uint32_t kEnd = kY + kEpiWarps * kYBufs * kYBufBytes;
+  static constexpr uint32_t kInv2 = kY + kEpiWarps * kYBufs * kYBufBytes;  // MLP only
+  static constexpr uint32_t kStg = kInv2 + (kMlp ? kInv2Bytes : 0);
+  static constexpr uint32_t kRed = kStg + (kMlp ? kStgBytes : 0);
+  static constexpr uint32_t kEnd = kRed + (kMlp ? kRedBytes : 0);
 };
-static_assert(EpiSmem<false>::kEnd + 1024 <= 227 * 1024, "shared memory budget (plain)");
+static_assert(EpiSmem<kEpiPlain>::kEnd + 1024 <= 227 * 1024, "shared memory budget (plain)");
 static_assert(kEpiWarps * 4 * kYBufBytes <= kStages2 * kStage2, "last-tile staging fits in the stage ring");
-static_assert(EpiSmem<true>::kEnd + 1024 <= 227 * 1024, "shared memory budget (QKV)");
+static_assert(EpiSmem<kEpiQkv>::kEnd + 1024 <= 227 * 1024, "shared memory budget (QKV)");
+static_assert(EpiSmem<kEpiMlp>::kEnd + 1024 <= 227 * 1024, "shared memory budget (MLP)");
 constexpr uint32_t kTmemCols2 = 512;
 constexpr uint32_t kColSFA = 256, kColSFB = kColSFA + 16 * kStages2;
 constexpr uint16_t kPairMask = 0x3;
@@ -137,7 +155,74 @@ struct GemmParams {
   const float* rope;       // packed rotary table: [row tile][32 chunks][128 rows] x 16 bytes
   float eps;
   int32_t qkv_cols;  // N / 3
+  // MLP instance only: fc2's activation buffer (codes, scales), 1/lambda2, L1_2^T chunks
+  uint8_t* codes2;
+  uint8_t* sf2;
+  const float* inv_lam2;
+  const uint8_t* l1t2;
+  float* partial;     // [NT][MP * 256][r2] fp32
+  int32_t KT2, rc16_2, r2;
+  float g_a2, c_a2;
+  // stream-K of the last wave (plain instance): sk_tiles tiles split over the first sk_pairs pairs
+  int32_t sk_tiles, sk_pairs;
+  uint32_t* sk_flags;   // [pair][CTA]: 1 = that CTA's partial tile is written
+  float4* sk_partial;   // [pair][CTA][64 column groups][128 rows]
 };
+
+// One segment of a pair's work: k-tiles [k_lo, k_hi) of tile `tile`.  `fin`: this pair finishes
+// the tile (it owns k-tile 0: it adds the other pairs' partials, the up projection and the
+// epilogue); otherwise it leaves a partial for the finishing pair.
+struct Seg {
+  int tile, k_lo, k_hi;
+  bool fin;
+};
+// A pair's work in order: its data-parallel tiles (tile = pair, pair + npairs, ... below D =
+// ntiles - sk_tiles, each with the whole K), then its share [lin, lin_end) of the stream-K
+// phase's k-tiles, which runs over tiles D .. ntiles - 1 in order.  Every role of both CTAs walks
+// the same list.  The state is three integers; the rest comes from the kernel parameters.
+struct SegIter {
+  int next_dp, lin, lin_end;
+  __device__ SegIter(const GemmParams& p, int pair) {
+    next_dp = pair;
+    const int64_t I = int64_t(p.sk_tiles) * p.KT;
+    if (p.sk_tiles > 0 && pair < p.sk_pairs) {
+      lin = int(int64_t(pair) * I / p.sk_pairs);
+      lin_end = int(int64_t(pair + 1) * I / p.sk_pairs);
+    } else {
+      lin = lin_end = 0;
+    }
+  }
+  __device__ bool has_next(const GemmParams& p, int ntiles) const {
+    return next_dp < ntiles - p.sk_tiles || lin < lin_end;
+  }
+  __device__ bool next(const GemmParams& p, int npairs, int ntiles, Seg& s) {
+    const int D = ntiles - p.sk_tiles;
+    if (next_dp < D) {
+      s = Seg{next_dp, 0, p.KT, true};
+      next_dp += npairs;
+      return true;
+    }
+    if (lin < lin_end) {
+      const int t = lin / p.KT;
+      s.tile = D + t;
+      s.k_lo = lin - t * p.KT;
+      s.k_hi = lin_end - t * p.KT < p.KT ? lin_end - t * p.KT : p.KT;
+      s.fin = s.k_lo == 0;
+      lin = s.k_hi == p.KT ? (t + 1) * p.KT : lin_end;
+      return true;
+    }
+    return false;
+  }
+};
+
+// The pairs whose stream-K range starts strictly inside tile D + t (they leave partials for it),
+// in pair order: [q0, q1).
+__device__ __forceinline__ void sk_contributors(const GemmParams& p, int t, int fin_pair, int& q0, int& q1) {
+  const int64_t I = int64_t(p.sk_tiles) * p.KT;
+  q0 = fin_pair + 1;
+  q1 = q0;
+  while (q1 < p.sk_pairs && int64_t(q1) * I / p.sk_pairs < int64_t(t + 1) * p.KT) ++q1;
+}
 
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float k0 = 0.7978845608028654f;  // sqrt(2 / pi)
@@ -229,6 +314,51 @@ __device__ __forceinline__ void norm_rope_chunks(uint32_t* out, float inv, const
   }
 }
 
+// Fused MLP pair, second step: lr'2 = bf16(sum_t partial[t] / alpha2), the weight tiles t of
+// fc1 added in order (deterministic), into fc2's activation buffer.
+__global__ void mlp_reduce_kernel(const float* __restrict__ partial, int32_t nt, int64_t rows, int32_t r2,
+                                  float inv_alpha2, uint8_t* lr2, int32_t RJ2, uint32_t* sk_flags2,
+                                  int32_t sk_flag_words2) {
+  griddep_wait();  // the partials are the previous kernel's output
+  if (blockIdx.x == 0)  // fc2's activation buffer is complete now: its GEMM's stream-K flags start cleared
+    for (int i = int(threadIdx.x); i < sk_flag_words2; i += int(blockDim.x)) sk_flags2[i] = 0u;
+  const int groups = r2 / 4;
+  const int64_t total = rows * groups;
+  const size_t plane = size_t(rows) * size_t(r2);
+  for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t m = idx / groups;
+    const int c = int(idx % groups) * 4;
+    const float* src = partial + size_t(m) * r2 + c;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int t = 0;
+    for (; t + 8 <= nt; t += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __ldg(reinterpret_cast<const float4*>(src + size_t(t + j) * plane));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        acc.x += v[j].x;
+        acc.y += v[j].y;
+        acc.z += v[j].z;
+        acc.w += v[j].w;
+      }
+    }
+    for (; t < nt; ++t) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src + size_t(t) * plane));
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    uint2 w;
+    w.x = f32x2_to_bf16x2(__fmul_rn(acc.x, inv_alpha2), __fmul_rn(acc.y, inv_alpha2));
+    w.y = f32x2_to_bf16x2(__fmul_rn(acc.z, inv_alpha2), __fmul_rn(acc.w, inv_alpha2));
+    uint8_t* tile = lr2 + (size_t(m / kBM) * RJ2 + size_t(c / kRChunk)) * kATileBytes;
+    *reinterpret_cast<uint2*>(tile + sw128(uint32_t(m % kBM), uint32_t(c % kRChunk) * 2u)) = w;
+  }
+}
+
 __global__ void rope_pack_kernel(const float4* rope, int64_t M, float4* packed, int64_t total) {
   for (int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += int64_t(gridDim.x) * blockDim.x) {
@@ -238,8 +368,9 @@ __global__ void rope_pack_kernel(const float4* rope, int64_t M, float4* packed, 
   }
 }
 
-template <bool kQkv>
+template <int kEpi>
 __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
+  constexpr bool kQkv = kEpi == kEpiQkv, kMlp = kEpi == kEpiMlp;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -260,7 +391,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   const uint32_t SFULL = ctrl_s + 112u;  // 5 barriers: this CTA's scales of a stage have landed
   uint32_t* bias_s = reinterpret_cast<uint32_t*>(ctrl + kCtrl2);  // [warp][32 bf16 pairs]
   const uint32_t XCH = ctrl_s + 152u;  // QKV: 8 barriers, one per warp pair sharing a head
-  using ES = EpiSmem<kQkv>;
+  using ES = EpiSmem<kEpi>;
   float* xch = reinterpret_cast<float*>(smem + ES::kXch);
   uint32_t* norm_s = reinterpret_cast<uint32_t*>(smem + ES::kNorm);
 
@@ -307,11 +438,13 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       prefetch_tensormap(&maps.bsf);
       uint32_t it = 0;
       bool stop = false;
-      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+      SegIter work(p, pair);
+      Seg sg;
+      while (!stop && work.next(p, npairs, ntiles, sg)) {
         int mp, nt;
-        tile_coords(p, tile, mp, nt);
+        tile_coords(p, sg.tile, mp, nt);
         const int mt = 2 * mp + int(rank);
-        for (int kt = 0; kt < p.KT; ++kt) {
+        for (int kt = sg.k_lo; kt < sg.k_hi; ++kt) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
             fail(0x10u);
@@ -328,7 +461,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           tma_load_2d(st + kOffSFB, &maps.bsf, 0, (nt * p.KT + kt) * kRowsSFB, SFULL + 8u * s);
           ++it;
         }
-        for (int j = 0; j < nlr && !stop; ++j) {
+        for (int j = 0; j < (sg.fin ? nlr : 0) && !stop; ++j) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
             fail(0x10u);
@@ -357,13 +490,15 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       const uint32_t id_fp4 = idesc_nvfp4_m256(kBN), id_bf16 = idesc_bf16_m256(kBN);
       uint32_t it = 0, tc = 0;
       bool stop = false, any = false;
-      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+      SegIter work(p, pair);
+      Seg sg;
+      while (!stop && work.next(p, npairs, ntiles, sg)) {
         if (!mbar_wait(ACCE, (tc & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
           fail(0x20u);
           break;
         }
         tc_fence_after();
-        for (int kt = 0; kt < p.KT; ++kt) {
+        for (int kt = sg.k_lo; kt < sg.k_hi; ++kt) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
             fail(0x20u);
@@ -376,12 +511,12 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
 #pragma unroll
           for (uint32_t kb = 0; kb < 4; ++kb)
             umma_nvfp4_pair(tmem, sdesc_sw128(st + kOffA + 32u * kb), sdesc_sw128(st + kOffB + 32u * kb), id_fp4,
-                            sfa + 4u * kb, sfb + 8u * kb, (kt | int(kb)) ? 1u : 0u);
+                            sfa + 4u * kb, sfb + 8u * kb, ((kt - sg.k_lo) | int(kb)) ? 1u : 0u);
           tc_commit_pair_mc(EMPTY + 8u * s, kPairMask);
           any = true;
           ++it;
         }
-        for (int j = 0; j < nlr && !stop; ++j) {
+        for (int j = 0; j < (sg.fin ? nlr : 0) && !stop; ++j) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
             fail(0x20u);
@@ -418,8 +553,11 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     const uint32_t lanes = (32u * q) << 16;
     uint32_t it = 0;
     bool stop = false;
-    for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
-      for (int k = 0; k < p.KT + nlr && !stop; ++k) {
+    SegIter work(p, pair);
+    Seg sg;
+    while (!stop && work.next(p, npairs, ntiles, sg)) {
+      const int nk = sg.k_hi - sg.k_lo;
+      for (int k = 0; k < nk + (sg.fin ? nlr : 0) && !stop; ++k) {
         const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
         bool ok = mbar_wait(SFULL + 8u * s, ph, abort_flag, p.timeout_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
@@ -428,7 +566,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           stop = true;
           break;
         }
-        if (k < p.KT) {
+        if (k < nk) {
           const uint8_t* st = smem + s * kStage2;
           {
             uint32_t r[16];
@@ -468,6 +606,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     uint8_t* ybuf = smem + ES::kY + uint32_t(warp) * ES::kYBufs * kYBufBytes;
     const uint32_t ybuf_s = sbase + ES::kY + uint32_t(warp) * ES::kYBufs * kYBufBytes;
     uint32_t* norm_w = norm_s + warp * 64;  // QKV: [Q, K][32 bf16 pairs] of this warp's columns
+    float* inv2_w = reinterpret_cast<float*>(smem + ES::kInv2) + warp * 64;  // MLP: 1/lambda2 of its columns
     if (kQkv) {
       const int half = colq & 1;
       norm_w[lane] = *reinterpret_cast<const uint32_t*>(p.norm_q + half * 64 + 2 * lane);
@@ -476,7 +615,10 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     }
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colq * 64);
-    for (int tile = pair; tile < ntiles; tile += npairs) {
+    SegIter work(p, pair);
+    Seg sg;
+    while (work.next(p, npairs, ntiles, sg)) {
+      const int tile = sg.tile;
       int mp, nt;
       tile_coords(p, tile, mp, nt);
       const int mt = 2 * mp + int(rank);
@@ -484,6 +626,14 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       uint32_t* bias_w = bias_s + warp * 32;
       __syncwarp();
       if (p.bias) bias_w[lane] = *reinterpret_cast<const uint32_t*>(p.bias + size_t(nt) * kBN + colq * 64 + lane * 2);
+      if constexpr (kMlp) {  // and its 64 values of the next layer's 1/lambda (its input channels)
+        const int n0s = nt * kBN + colq * 64;
+        if (n0s < p.N) {
+          const float2 w2 = *reinterpret_cast<const float2*>(p.inv_lam2 + n0s + 2 * lane);
+          inv2_w[2 * lane] = w2.x;
+          inv2_w[2 * lane + 1] = w2.y;
+        }
+      }
       __syncwarp();
       bool ok = mbar_wait(ACCF, tc & 1u, abort_flag, p.timeout_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);
@@ -492,6 +642,14 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         break;
       }
       tc_fence_after();
+      // stream-K finisher of a split tile (its pair's last segment: nothing waits behind it): the
+      // pairs that ran the tile's later k-tiles must have left their partials
+      int q0 = 0, q1 = 0;
+      if (sg.fin && sg.k_hi < p.KT) {
+        sk_contributors(p, tile - (ntiles - p.sk_tiles), pair, q0, q1);
+        for (int q = q0; q < q1; ++q)
+          if (!wait_flag(p.sk_flags + q * 2 + int(rank), 1u, p.timeout_ns) && lane == 0) fail(0x200u);
+      }
       uint32_t v[64];
       tmem_ld32(tl, v);
       tmem_ld32(tl + 32u, v + 32);
@@ -499,12 +657,45 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
-      const int64_t row = int64_t(mt) * kBM + row_in_tile;
+      if (!sg.fin) {
+        // stream-K contributor: this CTA's float32 partial of the tile, then its flag (a pair
+        // contributes once, so its slot is its own)
+        float4* dst = p.sk_partial + ((size_t(pair) * 2 + rank) * 64 + size_t(colq) * 16) * kBM + row_in_tile;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          dst[j * kBM] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        __threadfence();
+        named_sync(5, 32 * kEpiWarps);
+        if (threadIdx.x == 0) st_release_gpu(p.sk_flags + pair * 2 + int(rank), 1u);
+        ++tc;
+        continue;
+      }
+      if (sg.k_hi < p.KT) {
+        // stream-K finisher: add the partials of the pairs that ran this tile's later k-tiles,
+        // in pair order (deterministic), then clear their flags for the next launch
+        for (int q = q0; q < q1; ++q) {
+          const float4* src =
+              p.sk_partial + ((size_t(q) * 2 + rank) * 64 + size_t(colq) * 16) * kBM + row_in_tile;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float4 pv = __ldcg(src + j * kBM);
+            v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + pv.x);
+            v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + pv.y);
+            v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + pv.z);
+            v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + pv.w);
+            asm volatile("" ::: "memory");  // one load in flight at a time: no registers for the rest
+          }
+        }
+        named_sync(5, 32 * kEpiWarps);  // every warp has read every partial
+        if (threadIdx.x == 0)
+          for (int q = q0; q < q1; ++q) p.sk_flags[q * 2 + int(rank)] = 0u;
+      }
       const int32_t y0 = mt * kBM + quarter * 32;  // first row of this warp's share
       // On its last tile the CTA's stage ring is idle (every MMA that read it
       // has completed): each warp stages its 4 stores there, 4 KB apart, and
       // never waits for a buffer.
-      const bool last = tile + npairs >= ntiles;
+      const bool last = !work.has_next(p, ntiles);
       if (last) yslot = 0;
       uint8_t* const sbuf = last ? smem + uint32_t(warp) * 4u * kYBufBytes : ybuf;
       const uint32_t sbuf_s = last ? sbase + uint32_t(warp) * 4u * kYBufBytes : ybuf_s;
@@ -563,6 +754,151 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           // rows past M are clipped by the tensor store
 #pragma unroll
           for (int j = 0; j < 4; ++j) put16(out + 8 * j, n0 + 16 * j);
+        }
+      } else if constexpr (kMlp) {
+        // the next layer's (fc2's) activations from this row's 64 outputs: x_hat2 =
+        // bf16(y / lambda2), NVFP4 codes and block scales into fc2's activation buffer (fc1's
+        // weight tile nt is fc2's k-tile nt, this warp's 64 columns its chunk colq), then the
+        // partial x_hat2 L1_2 over these 64 inputs on the warp-level tensor cores
+        const int n0 = nt * kBN + colq * 64;
+        const bool in = n0 < p.N;  // warp-uniform: N % 64 == 0
+        uint32_t xh[32];
+        uint32_t cw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u}, sc4 = 0u;
+        if (in) {
+          uint32_t y[32];
+          finish_chunk(p, v, p.bias ? bias_w : nullptr, y);
+          finish_chunk(p, v + 32, p.bias ? bias_w + 16 : nullptr, y + 16);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            float xf[16];
+            float amax = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float lo = __fmul_rn(bf16lo(y[8 * b + j]), inv2_w[16 * b + 2 * j]);
+              const float hi = __fmul_rn(bf16hi(y[8 * b + j]), inv2_w[16 * b + 2 * j + 1]);
+              const uint32_t h = f32x2_to_bf16x2(lo, hi);
+              xh[8 * b + j] = h;
+              xf[2 * j] = bf16lo(h);
+              xf[2 * j + 1] = bf16hi(h);
+              amax = fmaxf(amax, fmaxf(fabsf(xf[2 * j]), fabsf(xf[2 * j + 1])));
+            }
+            const uint32_t sc = f32_to_e4m3(__fmul_rn(amax, p.c_a2));
+            const float d = __fmul_rn(e4m3_value(sc), p.g_a2);
+            const float rcp = d == 0.0f ? 0.0f : __frcp_rn(d);
+            cw[2 * b] = f32x8_to_e2m1(__fmul_rn(xf[0], rcp), __fmul_rn(xf[1], rcp), __fmul_rn(xf[2], rcp),
+                                      __fmul_rn(xf[3], rcp), __fmul_rn(xf[4], rcp), __fmul_rn(xf[5], rcp),
+                                      __fmul_rn(xf[6], rcp), __fmul_rn(xf[7], rcp));
+            cw[2 * b + 1] = f32x8_to_e2m1(__fmul_rn(xf[8], rcp), __fmul_rn(xf[9], rcp), __fmul_rn(xf[10], rcp),
+                                          __fmul_rn(xf[11], rcp), __fmul_rn(xf[12], rcp), __fmul_rn(xf[13], rcp),
+                                          __fmul_rn(xf[14], rcp), __fmul_rn(xf[15], rcp));
+            sc4 |= sc << (8 * b);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) xh[j] = 0u;
+        }
+        {  // columns past N (fc2's K) get zero codes and scales, like padding read past the end of X
+          uint8_t* ctile = p.codes2 + (size_t(mt) * p.KT2 + nt) * kATileBytes;
+          *reinterpret_cast<uint4*>(ctile + sw128(uint32_t(row_in_tile), uint32_t(colq) * 32u)) =
+              make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          *reinterpret_cast<uint4*>(ctile + sw128(uint32_t(row_in_tile), uint32_t(colq) * 32u + 16u)) =
+              make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          uint8_t* stile = p.sf2 + (size_t(mt) * p.KT2 + nt) * kSFATileBytes + size_t(colq) * kSFAtomBytes;
+          *reinterpret_cast<uint32_t*>(stile + sf_atom(uint32_t(row_in_tile), 0u)) = sc4;
+        }
+        // partial x_hat2 L1_2, up to 32 ranks at a time: the warp's 32 rows x 16 inputs of x_hat2
+        // go through its staging buffer (row = lane, 16-byte halves swizzled by bit 2 of the
+        // row) into A fragments; L1_2^T words straight from global memory are the B fragments
+        uint8_t* stg = smem + ES::kStg + uint32_t(warp) * 1024u;
+        const uint32_t stg_s = sbase + ES::kStg + uint32_t(warp) * 1024u;
+        // the reduction slot of fragment value f (0..31) of this lane: the staging buffer of the
+        // quarter's warp quarter + 4 (f / 8), float (f % 8) * 32 + lane
+        auto red_slot = [&](int f) {
+          return reinterpret_cast<float*>(smem + ES::kStg + uint32_t(quarter + 4 * (f >> 3)) * 1024u) +
+                 (f & 7) * 32 + lane;
+        };
+        const uint8_t* l1c = p.l1t2 + size_t(in ? n0 / 64 : 0) * size_t(p.rc16_2) * 128u;
+        const uint32_t swz = (uint32_t(lane) >> 2) & 1u;
+        for (int rc = 0; rc < p.r2; rc += 32) {
+          const int nb8 = p.r2 - rc >= 32 ? 4 : 2;  // ranks come in multiples of 16
+          float acc[2][4][4];
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.0f;
+          if (in) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              uint32_t bf[4][2];
+#pragma unroll
+              for (int n8 = 0; n8 < 4; ++n8) {  // B fragments first: their loads overlap the staging
+                const uint32_t rho = uint32_t(rc + 8 * n8 + (lane >> 2));
+                const uint32_t kb = uint32_t(32 * kk + 4 * (lane & 3));
+                bf[n8][0] = n8 < nb8 ? __ldg(reinterpret_cast<const unsigned int*>(l1c + sw128(rho, kb))) : 0u;
+                bf[n8][1] = n8 < nb8 ? __ldg(reinterpret_cast<const unsigned int*>(l1c + sw128(rho, kb + 16u))) : 0u;
+              }
+              *reinterpret_cast<uint4*>(stg + lane * 32 + 16u * swz) =
+                  make_uint4(xh[8 * kk], xh[8 * kk + 1], xh[8 * kk + 2], xh[8 * kk + 3]);
+              *reinterpret_cast<uint4*>(stg + lane * 32 + 16u * (swz ^ 1u)) =
+                  make_uint4(xh[8 * kk + 4], xh[8 * kk + 5], xh[8 * kk + 6], xh[8 * kk + 7]);
+              __syncwarp();
+              uint32_t af[2][4];
+#pragma unroll
+              for (int m16 = 0; m16 < 2; ++m16) {
+                const uint32_t row = uint32_t(m16 * 16 + (lane & 7) + ((lane >> 3) & 1) * 8);
+                const uint32_t kh = uint32_t(lane >> 4);
+                ldsm_x4(stg_s + row * 32u + ((kh ^ ((row >> 2) & 1u)) * 16u), af[m16]);
+              }
+              __syncwarp();
+#pragma unroll
+              for (int n8 = 0; n8 < 4; ++n8)
+                if (n8 < nb8) {
+                  mma_bf16_16816(acc[0][n8], af[0], bf[n8][0], bf[n8][1]);
+                  mma_bf16_16816(acc[1][n8], af[1], bf[n8][0], bf[n8][1]);
+                }
+            }
+          }
+          // the quarter's four warps add their partials in column order (deterministic), the
+          // last one writes the tile's partial of these 32 rows x nb8 * 8 ranks; the staging
+          // buffers become the sum's storage once all four warps are past their MMAs
+          const uint32_t bar = 1u + uint32_t(quarter);
+          named_sync(bar, 128);
+#pragma unroll
+          for (int step = 0; step < 4; ++step) {
+            if (colq == step) {
+#pragma unroll
+              for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                  if (b < nb8) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                      float* slot = red_slot((a * 4 + b) * 4 + e);
+                      if (step) acc[a][b][e] += *slot;
+                      if (step < 3) *slot = acc[a][b][e];
+                    }
+                  }
+              if (step == 3) {
+                const int64_t rows = int64_t(p.MP) * 2 * kBM;
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                  for (int b = 0; b < 4; ++b)
+                    if (b < nb8) {
+#pragma unroll
+                      for (int hh = 0; hh < 2; ++hh) {
+                        const int64_t r = int64_t(mt) * kBM + quarter * 32 + a * 16 + (lane >> 2) + 8 * hh;
+                        const int rk = rc + 8 * b + 2 * (lane & 3);
+                        *reinterpret_cast<float2*>(p.partial + (size_t(nt) * rows + r) * p.r2 + rk) =
+                            make_float2(acc[a][b][2 * hh], acc[a][b][2 * hh + 1]);
+                      }
+                    }
+              }
+            }
+            named_sync(bar, 128);
+          }
         }
       } else {
 #pragma unroll
@@ -637,11 +973,13 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   GemmMaps maps;
   const uint8_t* act = a.act;
   const uint8_t* lay = a.layer;
+  const bool mlp = a.mlp_act2 != nullptr;
   bool ok = encode_rows(&maps.a, act + ag.off_codes, uint64_t(ag.MT) * ag.KT * kATileBytes, kRowsA) &&
             encode_rows(&maps.asf, act + ag.off_sf, uint64_t(ag.MT) * ag.KT * kSFATileBytes, kRowsSFA) &&
             encode_rows(&maps.b, lay + lg.off_bcodes, uint64_t(lg.NT) * lg.KT * kBTileBytes, kRowsA) &&
             encode_rows(&maps.bsf, lay + lg.off_sfb, uint64_t(lg.NT) * lg.KT * kSFBTileBytes, kRowsSFB) &&
-            encode_y(&maps.y, a.Y, a.M, lg.N);
+            (mlp || encode_y(&maps.y, a.Y, a.M, lg.N));
+  if (mlp) maps.y = maps.a;  // the MLP instance writes no Y
   if (ok && lg.RJ > 0) {
     ok = encode_rows(&maps.lr, act + ag.off_lr, uint64_t(ag.MT) * ag.RJ * kATileBytes, kRowsA) &&
          encode_rows(&maps.l2, lay + lg.off_l2t, uint64_t(lg.NT) * lg.RJ * kBTileBytes, kRowsA);
@@ -673,18 +1011,36 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   p.rope = a.rope;
   p.eps = a.eps;
   p.qkv_cols = a.qkv_cols;
-  auto kernel = qkv ? gemm_kernel<true> : gemm_kernel<false>;
+  if (mlp) {
+    const LayerGeom& g2 = a.mlp_lg2;
+    const ActGeom ag2 = make_act_geom(g2, a.M);
+    p.codes2 = a.mlp_act2 + ag2.off_codes;
+    p.sf2 = a.mlp_act2 + ag2.off_sf;
+    p.inv_lam2 = reinterpret_cast<const float*>(a.mlp_layer2 + g2.off_inv_lam);
+    p.l1t2 = a.mlp_layer2 + g2.off_l1t;
+    p.partial = a.mlp_partial;
+    p.KT2 = int32_t(g2.KT);
+    p.rc16_2 = int32_t(g2.RC16);
+    p.r2 = a.mlp_r2;
+    p.g_a2 = a.mlp_g_a2;
+    p.c_a2 = a.mlp_c_a2;
+  }
+  const int kind = qkv ? kEpiQkv : mlp ? kEpiMlp : kEpiPlain;
+  auto kernel = qkv ? gemm_kernel<kEpiQkv> : mlp ? gemm_kernel<kEpiMlp> : gemm_kernel<kEpiPlain>;
 
   const int64_t ntiles = int64_t(p.MP) * lg.NT;
   if (ntiles > (int64_t(1) << 30)) {
     *why = "problem too large for one launch";
     return cudaErrorInvalidValue;
   }
-  const size_t smem = size_t(qkv ? EpiSmem<true>::kEnd : EpiSmem<false>::kEnd) + 1024;
-  static std::atomic<int> max_pairs_of[2][64];
+  const size_t smem = size_t(qkv   ? EpiSmem<kEpiQkv>::kEnd
+                             : mlp ? EpiSmem<kEpiMlp>::kEnd
+                                   : EpiSmem<kEpiPlain>::kEnd) +
+                      1024;
+  static std::atomic<int> max_pairs_of[3][64];
   int dev = 0;
   cudaGetDevice(&dev);
-  std::atomic<int>* max_pairs = max_pairs_of[qkv ? 1 : 0];
+  std::atomic<int>* max_pairs = max_pairs_of[kind];
   if (max_pairs[dev & 63].load() == 0) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e == cudaSuccess)
@@ -714,7 +1070,20 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
     max_pairs[dev & 63].store(clusters);
   }
   const int cap = max_pairs[dev & 63].load();
-  const int pairs = int(ntiles < cap ? ntiles : cap);
+  int pairs = int(ntiles < cap ? ntiles : cap);
+  // stream-K of the last wave (plain epilogue only), within the area the activation buffer holds:
+  // the data-parallel tiles stride over all `cap` pairs, the last wave's k-tiles are shared
+  if (kind == kEpiPlain && a.sk_area && cap <= a.sk_max_pairs) {
+    const SkPlan sk = make_sk_plan(ntiles, lg.KT, cap);
+    const size_t need = sk.tiles ? sk_flag_bytes(a.sk_max_pairs) + size_t(sk.pairs) * 2 * kSkCtaBytes : 0;
+    if (sk.tiles && need <= sk_area_bytes(ntiles, a.sk_max_pairs)) {
+      p.sk_tiles = sk.tiles;
+      p.sk_pairs = sk.pairs;
+      p.sk_flags = reinterpret_cast<uint32_t*>(a.sk_area);
+      p.sk_partial = reinterpret_cast<float4*>(a.sk_area + sk_flag_bytes(a.sk_max_pairs));
+      pairs = ntiles > sk.tiles ? cap : sk.pairs;  // all pairs when tiles run whole too
+    }
+  }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
   cfg.blockDim = dim3(kThreads2, 1, 1);
@@ -732,6 +1101,28 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, maps, p);
   if (e != cudaSuccess) *why = "launch of the GEMM kernel failed";
   return e;
+}
+
+size_t mlp_partial_bytes(int64_t NT1, int64_t MT, int32_t r2) {
+  return size_t(NT1) * size_t(MT) * kBM * size_t(r2) * sizeof(float);
+}
+
+cudaError_t launch_mlp_reduce(const MlpReduceLaunch& a, cudaStream_t s) {
+  const int64_t total = a.rows * (a.r2 / 4);  // 0 when fc2 has no ranks: only the flags are cleared
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 8192) blocks = 8192;
+  if (blocks < 1) blocks = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, mlp_reduce_kernel, a.partial, a.nt, a.rows, a.r2, a.inv_alpha2, a.lr2, a.RJ2,
+                            a.sk_flags2, a.sk_flags2 ? a.sk_flag_words2 : 0);
 }
 
 cudaError_t launch_rope_pack(const float* rope, int64_t M, float* packed, cudaStream_t s) {

@@ -20,6 +20,8 @@ struct ActQuantLaunch {
   float g_a, c_a, inv_alpha;
   int num_sms;
   uint64_t timeout_ns;
+  uint32_t* sk_flags;    // the activation buffer's stream-K flags, cleared by this kernel
+  int32_t sk_flag_words;
 };
 cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char** why);
 
@@ -43,8 +45,37 @@ struct GemmLaunch {
   const uint16_t* norm_k;  // device bf16 [128]
   const float* rope;       // device packed rotary table (rope_packed_bytes(M) bytes)
   float eps;
+  // fused MLP pair (mlp_act2 != null): instead of Y, the epilogue writes the next layer's
+  // (fc2's) NVFP4 codes and block scales of x_hat2 = bf16(y bf16 / lambda2) into its
+  // activation buffer, and per weight tile the partial x_hat2 L1_2 into mlp_partial
+  // [NT][MT * 128][r2] (fp32); launch_mlp_reduce then sums the partials into fc2's lr'.
+  uint8_t* mlp_act2;        // fc2's activation buffer
+  const uint8_t* mlp_layer2; // fc2's device image
+  LayerGeom mlp_lg2;
+  int32_t mlp_r2;           // fc2's ranks in use
+  float mlp_g_a2, mlp_c_a2;
+  float* mlp_partial;
+  // the activation buffer's stream-K area (flags, then partial tiles) and the pairs it was sized for
+  uint8_t* sk_area;
+  int32_t sk_max_pairs;
 };
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why);
+
+// Fused MLP pair, second step: lr'2[m][rho] = bf16(sum over weight tiles t of
+// partial[t][m][rho] / alpha2) into fc2's activation buffer, tiles in a fixed order.
+struct MlpReduceLaunch {
+  const float* partial;  // [nt][rows][r2]
+  int32_t nt;            // weight tiles of fc1 (partials per row)
+  int64_t rows;          // MT * 128 rows of fc2's activation buffer
+  int32_t r2;
+  float inv_alpha2;
+  uint8_t* lr2;          // fc2's act buffer + off_lr
+  int32_t RJ2;           // fc2's low-rank chunks per row tile
+  uint32_t* sk_flags2;   // fc2's act buffer stream-K flags, cleared here
+  int32_t sk_flag_words2;
+};
+cudaError_t launch_mlp_reduce(const MlpReduceLaunch& a, cudaStream_t s);
+size_t mlp_partial_bytes(int64_t NT1, int64_t MT, int32_t r2);
 
 // [M][64][2] float (cos, sin) -> the packed layout of rope_packed_bytes(M).
 cudaError_t launch_rope_pack(const float* rope, int64_t M, float* packed, cudaStream_t s);

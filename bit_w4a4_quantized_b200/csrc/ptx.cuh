@@ -371,6 +371,44 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   return v;
 }
 
+// Four 8 x 8 matrices of 16-bit elements from shared memory (lane l gives the address of
+// row l % 8 of matrix l / 8), in the A-fragment order of the warp-level MMA.
+__device__ __forceinline__ void ldsm_x4(uint32_t saddr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+// D (f32, 16 x 8) += A (bf16, 16 x 16, row) * B (bf16, 16 x 8, col), one warp.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Global-memory flag handshake between CTAs of one grid (all resident): a release store
+// after the data, an acquire load before reading it.
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded wait for *flag == want (false after timeout_ns).
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t want, uint64_t timeout_ns) {
+  if (ld_acquire_gpu(flag) == want) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(flag) == want) return true;
+    if (globaltimer() - t0 > timeout_ns) return false;
+  }
+}
+
 // Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -403,6 +441,16 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1(float v0, float v1, float v2, 
       : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
   return out;
 }
+// Two products at once (Blackwell's packed float32 multiply): {a.x * b.x, a.y * b.y}, each
+// rounded to nearest even exactly as a single float32 multiply.
+__device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {
+  uint64_t d;
+  const uint64_t x = (uint64_t(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+  const uint64_t y = (uint64_t(__float_as_uint(b.y)) << 32) | __float_as_uint(b.x);
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(y));
+  return make_float2(__uint_as_float(uint32_t(d)), __uint_as_float(uint32_t(d >> 32)));
+}
+
 // Two floats -> packed bf16x2 (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
   uint32_t out;

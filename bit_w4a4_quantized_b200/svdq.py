@@ -49,7 +49,7 @@ EXPORTED_SYMBOLS = (
     "svdq_test_bounded_wait", "svdq_layer_clone", "svdq_w4a4_linear_qkv_norm_rope",
     "svdq_rope_packed_bytes", "svdq_rope_pack", "svdq_w4a16_device_bytes", "svdq_w4a16_prepare_host",
     "svdq_w4a16_upload", "svdq_w4a16_linear", "svdq_w4a16_export", "svdq_w4a16_destroy",
-    "svdq_layer_serialize", "svdq_layer_import",
+    "svdq_layer_serialize", "svdq_layer_import", "svdq_mlp_workspace_bytes", "svdq_w4a4_linear_mlp",
 )
 
 
@@ -123,6 +123,8 @@ def lib():
         "svdq_layer_destroy": ([vp], None),
         "svdq_layer_clone": ([vp, ctypes.POINTER(vp)], st),
         "svdq_layer_serialize": ([vp, vp, sz, ctypes.POINTER(sz)], st),
+        "svdq_mlp_workspace_bytes": ([vp, vp, i64, ctypes.POINTER(sz)], st),
+        "svdq_w4a4_linear_mlp": ([vp, vp, sz, i64, vp, vp, sz, vp, sz, ctypes.c_int, vp], st),
         "svdq_layer_import": ([vp, sz, ctypes.POINTER(vp)], st),
         "svdq_w4a16_device_bytes": ([ctypes.POINTER(W4A16Desc)], sz),
         "svdq_w4a16_prepare_host": ([ctypes.POINTER(W4A16Desc), ctypes.POINTER(vp)], st),
@@ -389,6 +391,31 @@ class Layer:
                                                    0 if rope_packed is None else _nbytes(rope_packed),
                                                    int(head_dim), float(eps), _stream(stream)))
         return out
+
+    def mlp_workspace_bytes(self, fc2, M):
+        n = ctypes.c_size_t()
+        check(lib().svdq_mlp_workspace_bytes(self._h, fc2._h, M, ctypes.byref(n)))
+        return n.value
+
+    def linear_mlp(self, act, M, fc2, act2=None, workspace=None, epilogue=EPI_GELU_TANH, stream=None):
+        """This layer as fc1 of a fused MLP pair: fc2's activation buffer from this layer's
+        output tile, without writing the output; returns act2 (pass it to fc2.linear)."""
+        import torch
+
+        dev = self._device()
+        _need(act, "act", dev)
+        if act2 is None:
+            act2 = fc2.new_act_buffer(M)
+        _need(act2, "act2", dev)
+        wb = self.mlp_workspace_bytes(fc2, M)
+        if workspace is None and wb:
+            workspace = torch.empty(wb, dtype=torch.uint8, device=dev)
+        if workspace is not None:
+            _need(workspace, "workspace", dev)
+        check(lib().svdq_w4a4_linear_mlp(self._h, _ptr(act), _nbytes(act), M, fc2._h, _ptr(act2), _nbytes(act2),
+                                         _ptr(workspace), 0 if workspace is None else _nbytes(workspace),
+                                         epilogue, _stream(stream)))
+        return act2
 
     def forward(self, X, out=None, epilogue=EPI_NONE, act=None, stream=None):
         act = self.quantize_act(X, act, stream)

@@ -153,8 +153,12 @@ SVDQ_API svdq_status svdq_prepare_weights(const svdq_prepare_desc* d, void* dev_
 
 /*
  * Bytes of the per-call activation buffer for M tokens: NVFP4 codes and block
- * scales of X_hat in the GEMM's tiled layout, and the bf16 down-projection
- * lr' = (X_hat L1) / (g_a g_w) for rank_capacity ranks.  Host only.
+ * scales of X_hat in the GEMM's tiled layout, the bf16 down-projection
+ * lr' = (X_hat L1) / (g_a g_w) for rank_capacity ranks, then the GEMM's
+ * scratch for the tiles of its last wave when they are split across CTA pairs
+ * (flags and float32 partial tiles, sized for half the device's SMs; cleared by
+ * svdq_quantize_act).  Host only; the size depends on the layer's device (the
+ * current device before upload).
  */
 SVDQ_API svdq_status svdq_act_buffer_bytes(const svdq_layer* layer, int64_t M, size_t* bytes);
 
@@ -175,7 +179,9 @@ SVDQ_API svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, i
  * block-scaled MMA and the bf16 up projection accumulating into the same
  * tensor-memory tile.
  * act_buf: the buffer svdq_quantize_act filled for the same M, through this
- *   handle, after its last svdq_lora_swap.  The handle notes the last 64 act_bufs
+ *   handle, after its last svdq_lora_swap.  The GEMM also uses the buffer's
+ *   scratch tail (partial tiles of the last wave), so two calls whose kernels
+ *   may overlap on the GPU must not share one act_buf.  The handle notes the last 64 act_bufs
  *   it filled; one of those filled before a later swap holds lr' columns of the
  *   replaced factors, and is refused with SVDQ_ERR_INVALID_ARGUMENT (quantize X
  *   again).  A buffer filled through another handle is not checked.
@@ -215,6 +221,30 @@ SVDQ_API svdq_status svdq_w4a4_linear_qkv_norm_rope(const svdq_layer* layer, con
                                            const void* norm_k, const void* rope_packed,
                                            size_t rope_packed_bytes, int32_t head_dim, float eps,
                                            void* stream);
+
+/*
+ * The fused MLP pair (Diffusers/Nunchaku page, the kernel-family list: the
+ * fused GELU/MLP path).  Runs fc1's kernel 2 on act1, and instead of writing
+ * fc1's output y = bf16(act(g_a g_w (Q(X_hat) Q(R) + lr' L2) + b)) it turns each
+ * row of it straight into fc2's activation buffer: x_hat2 = bf16(y / lambda2)
+ * with fc2's smoothing factors, its NVFP4 codes and E4M3 block scales under
+ * fc2's static g_a, and lr'2 = bf16((x_hat2 L1_2) / (g_a2 g_w2)) -- exactly what
+ * svdq_quantize_act(fc2, y) computes from the bf16 y, without y ever reaching
+ * memory.  Then svdq_w4a4_linear(fc2, act2, ...) finishes the pair.
+ * fc2's K must equal fc1's N.  act1: filled by svdq_quantize_act(fc1) for the
+ * same M.  act2: >= svdq_act_buffer_bytes(fc2, M) bytes, 256-byte aligned.
+ * workspace: device, 16-byte aligned, >= svdq_mlp_workspace_bytes bytes (0 when
+ *   fc2 has no ranks): float partials of x_hat2 L1_2, one per 256 of fc1's
+ *   outputs, which a second kernel on the same stream sums in a fixed order.
+ *   It is scratch: reused by the next call, caller-owned.
+ * epilogue: SVDQ_EPI_GELU_TANH (the MLP's activation) or SVDQ_EPI_NONE.
+ * Stream ordered; both layers on the current device.
+ */
+SVDQ_API svdq_status svdq_mlp_workspace_bytes(const svdq_layer* fc1, const svdq_layer* fc2, int64_t M,
+                                              size_t* bytes);
+SVDQ_API svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act1, size_t act1_bytes, int64_t M,
+                                          const svdq_layer* fc2, void* act2, size_t act2_bytes, void* workspace,
+                                          size_t workspace_bytes, int epilogue, void* stream);
 
 /* Bytes of the packed rotary table for M rows (head_dim 128).  Host only. */
 SVDQ_API svdq_status svdq_rope_packed_bytes(int64_t M, int32_t head_dim, size_t* bytes);
@@ -363,6 +393,11 @@ SVDQ_API svdq_status svdq_w4a16_upload(svdq_w4a16* layer, void* dev_buf, size_t 
  * 16-byte aligned; Y: device bf16 [M, N] row-major, 2-byte aligned; any M >= 1
  * (rows go 8 at a time, one launch each, stream ordered).  No bounded waits:
  * the kernel's CTAs never wait on one another.
+ * Range: the divided activation x / s is rounded to f16, not kept as bf16.
+ * Magnitudes above 65504 saturate to +-65504 and magnitudes below 2^-14 lose
+ * bits (f16 subnormals, zero below 2^-25); between them f16 keeps 3 more bits
+ * than bf16.  Inputs with |x / s| outside [2^-14, 65504] are therefore not
+ * represented as a bf16 operand would represent them.
  */
 SVDQ_API svdq_status svdq_w4a16_linear(const svdq_w4a16* layer, const void* X, int64_t M, void* Y, void* stream);
 
