@@ -59,8 +59,6 @@ struct ActQuantParams {
   uint8_t* sf;           // act + off_sf
   uint8_t* lr;           // act + off_lr
   uint32_t* status;      // layer status word
-  uint32_t* sk_flags;    // the activation buffer's stream-K flags (cleared by CTA 0)
-  int32_t sk_flag_words;
   int32_t MT, KT, KC, RJ, r_tot, rc16, splits;
   int32_t push;          // split partials are pushed to the owning CTA (else pulled)
   int32_t rows_per;      // rows of a row tile each CTA of the cluster reduces
@@ -179,8 +177,6 @@ __global__ void __launch_bounds__(kThreads1, 2)
   // X may be the previous kernel's output and the activation buffer its input
   griddep_wait();
   griddep_launch_dependents();
-  if (blockIdx.x == 0 && blockIdx.y == 0)  // the GEMM's stream-K flags start cleared
-    for (int i = int(threadIdx.x); i < p.sk_flag_words; i += int(blockDim.x)) p.sk_flags[i] = 0u;
 
   auto fail = [&](uint32_t code) {
     *abort_flag = 1u;
@@ -470,8 +466,6 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   p.sf = a.act + ag.off_sf;
   p.lr = a.act + ag.off_lr;
   p.status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.layer) + lg.off_status);
-  p.sk_flags = a.sk_flags;
-  p.sk_flag_words = a.sk_flags ? a.sk_flag_words : 0;
   p.MT = int32_t(ag.MT);
   p.KT = int32_t(lg.KT);
   p.KC = int32_t(lg.KC);

@@ -70,32 +70,6 @@ svdq_status check_uploaded(const svdq_layer* L) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// The activation buffer of M rows: what kernel 1 writes (codes, scales, lr'), then the GEMM's
-// stream-K area sized for every CTA pair the device can run (half its SMs).
-struct ActLayout {
-  svdq::ActGeom ag;
-  size_t sk_off, sk_bytes, total;
-  int sk_pairs;
-};
-ActLayout act_layout(const svdq_layer* L, int64_t M) {
-  ActLayout o{};
-  o.ag = svdq::make_act_geom(L->g, M);
-  int sms = L->num_sms;
-  if (sms <= 0) {  // not uploaded yet: the current device
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      sms = 0;
-    cudaGetLastError();  // a CPU-only process has no device: no stream-K area
-  }
-  o.sk_pairs = sms / 2;
-  const int64_t ntiles = (o.ag.MT / 2) * L->g.NT;
-  o.sk_off = o.ag.total;
-  o.sk_bytes = svdq::sk_area_bytes(ntiles, o.sk_pairs);
-  o.total = o.sk_off + o.sk_bytes;
-  return o;
-}
-
 // Note that act_buf now holds activations quantized under the handle's current factors.
 void note_act(const svdq_layer* L, const void* act_buf) {
   auto& N = L->notes;
@@ -193,7 +167,7 @@ svdq_status svdq_prepare_weights(const svdq_prepare_desc* d, void* dev_buf, size
 svdq_status svdq_act_buffer_bytes(const svdq_layer* L, int64_t M, size_t* bytes) {
   if (!L || !bytes) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer and bytes are required");
   if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
-  *bytes = act_layout(L, M).total;
+  *bytes = svdq::make_act_geom(L->g, M).total;
   return SVDQ_OK;
 }
 
@@ -205,15 +179,10 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
   if (!aligned(X, 16)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "X must be 16-byte aligned");
   if (!aligned(act_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf must be 256-byte aligned");
-  const ActLayout lay = act_layout(L, M);
-  const size_t need = lay.total;
+  const size_t need = svdq::make_act_geom(L->g, M).total;
   if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");
   if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
   svdq::ActQuantLaunch a{};
-  if (lay.sk_bytes) {
-    a.sk_flags = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(act_buf) + lay.sk_off);
-    a.sk_flag_words = 2 * lay.sk_pairs;
-  }
   a.X = X;
   a.layer = static_cast<const uint8_t*>(L->dev_buf);
   a.act = static_cast<uint8_t*>(act_buf);
@@ -244,8 +213,7 @@ svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_b
     return fail(SVDQ_ERR_INVALID_ARGUMENT, "unknown epilogue");
   if (!aligned(Y, 32)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "Y must be 32-byte aligned");
   if (!aligned(act_buf, 256)) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act_buf must be 256-byte aligned");
-  const ActLayout lay = act_layout(L, M);
-  const size_t need = lay.total;
+  const size_t need = svdq::make_act_geom(L->g, M).total;
   if (act_buf_bytes < need) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act_buf needs " + std::to_string(need) + " bytes");
   if (M * L->g.N > (int64_t(1) << 31) * 2 || M > (int64_t(1) << 31) - 1)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M too large");
@@ -265,10 +233,6 @@ svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_b
   a.alpha = L->alpha;
   a.num_sms = L->num_sms;
   a.timeout_ns = svdq::kDefaultTimeoutNs;
-  if (lay.sk_bytes) {  // the GEMM's scratch for the last wave's split tiles
-    a.sk_area = const_cast<uint8_t*>(static_cast<const uint8_t*>(act_buf)) + lay.sk_off;
-    a.sk_max_pairs = lay.sk_pairs;
-  }
   const char* why = "";
   cudaError_t e = svdq::launch_gemm(a, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
@@ -304,8 +268,7 @@ svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act1, size_t
   if (fc2->g.K != fc1->g.N) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "fc2's K must equal fc1's N");
   if (!aligned(act1, 256) || !aligned(act2, 256))
     return fail(SVDQ_ERR_INVALID_ARGUMENT, "act1 and act2 must be 256-byte aligned");
-  const ActLayout lay2 = act_layout(fc2, M);
-  const size_t need1 = act_layout(fc1, M).total, need2 = lay2.total;
+  const size_t need1 = svdq::make_act_geom(fc1->g, M).total, need2 = svdq::make_act_geom(fc2->g, M).total;
   if (act1_bytes < need1) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act1 needs " + std::to_string(need1) + " bytes");
   if (act2_bytes < need2) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "act2 needs " + std::to_string(need2) + " bytes");
   const svdq::ActGeom ag1 = svdq::make_act_geom(fc1->g, M);
@@ -341,7 +304,7 @@ svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act1, size_t
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = svdq::launch_gemm(a, s, &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
-  if (fc2->r_tot > 0 || lay2.sk_bytes) {  // lr'2, and fc2's stream-K flags cleared
+  if (fc2->r_tot > 0) {
     const svdq::ActGeom ag2 = svdq::make_act_geom(fc2->g, M);
     svdq::MlpReduceLaunch r{};
     r.partial = static_cast<const float*>(workspace);
@@ -351,10 +314,6 @@ svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act1, size_t
     r.inv_alpha2 = fc2->inv_alpha;
     r.lr2 = static_cast<uint8_t*>(act2) + ag2.off_lr;
     r.RJ2 = int32_t(ag2.RJ);
-    if (lay2.sk_bytes) {
-      r.sk_flags2 = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(act2) + lay2.sk_off);
-      r.sk_flag_words2 = 2 * lay2.sk_pairs;
-    }
     e = svdq::launch_mlp_reduce(r, s);
     if (e != cudaSuccess) return cuda_fail(e, "launch of the MLP partial reduction failed");
   }

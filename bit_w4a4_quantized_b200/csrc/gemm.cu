@@ -163,66 +163,7 @@ struct GemmParams {
   float* partial;     // [NT][MP * 256][r2] fp32
   int32_t KT2, rc16_2, r2;
   float g_a2, c_a2;
-  // stream-K of the last wave (plain instance): sk_tiles tiles split over the first sk_pairs pairs
-  int32_t sk_tiles, sk_pairs;
-  uint32_t* sk_flags;   // [pair][CTA]: 1 = that CTA's partial tile is written
-  float4* sk_partial;   // [pair][CTA][64 column groups][128 rows]
 };
-
-// One segment of a pair's work: k-tiles [k_lo, k_hi) of tile `tile`.  `fin`: this pair finishes
-// the tile (it owns k-tile 0: it adds the other pairs' partials, the up projection and the
-// epilogue); otherwise it leaves a partial for the finishing pair.
-struct Seg {
-  int tile, k_lo, k_hi;
-  bool fin;
-};
-// A pair's work in order: its data-parallel tiles (tile = pair, pair + npairs, ... below D =
-// ntiles - sk_tiles, each with the whole K), then its share [lin, lin_end) of the stream-K
-// phase's k-tiles, which runs over tiles D .. ntiles - 1 in order.  Every role of both CTAs walks
-// the same list.  The state is three integers; the rest comes from the kernel parameters.
-struct SegIter {
-  int next_dp, lin, lin_end;
-  __device__ SegIter(const GemmParams& p, int pair) {
-    next_dp = pair;
-    const int64_t I = int64_t(p.sk_tiles) * p.KT;
-    if (p.sk_tiles > 0 && pair < p.sk_pairs) {
-      lin = int(int64_t(pair) * I / p.sk_pairs);
-      lin_end = int(int64_t(pair + 1) * I / p.sk_pairs);
-    } else {
-      lin = lin_end = 0;
-    }
-  }
-  __device__ bool has_next(const GemmParams& p, int ntiles) const {
-    return next_dp < ntiles - p.sk_tiles || lin < lin_end;
-  }
-  __device__ bool next(const GemmParams& p, int npairs, int ntiles, Seg& s) {
-    const int D = ntiles - p.sk_tiles;
-    if (next_dp < D) {
-      s = Seg{next_dp, 0, p.KT, true};
-      next_dp += npairs;
-      return true;
-    }
-    if (lin < lin_end) {
-      const int t = lin / p.KT;
-      s.tile = D + t;
-      s.k_lo = lin - t * p.KT;
-      s.k_hi = lin_end - t * p.KT < p.KT ? lin_end - t * p.KT : p.KT;
-      s.fin = s.k_lo == 0;
-      lin = s.k_hi == p.KT ? (t + 1) * p.KT : lin_end;
-      return true;
-    }
-    return false;
-  }
-};
-
-// The pairs whose stream-K range starts strictly inside tile D + t (they leave partials for it),
-// in pair order: [q0, q1).
-__device__ __forceinline__ void sk_contributors(const GemmParams& p, int t, int fin_pair, int& q0, int& q1) {
-  const int64_t I = int64_t(p.sk_tiles) * p.KT;
-  q0 = fin_pair + 1;
-  q1 = q0;
-  while (q1 < p.sk_pairs && int64_t(q1) * I / p.sk_pairs < int64_t(t + 1) * p.KT) ++q1;
-}
 
 __device__ __forceinline__ float gelu_tanh(float x) {
   const float k0 = 0.7978845608028654f;  // sqrt(2 / pi)
@@ -317,11 +258,8 @@ __device__ __forceinline__ void norm_rope_chunks(uint32_t* out, float inv, const
 // Fused MLP pair, second step: lr'2 = bf16(sum_t partial[t] / alpha2), the weight tiles t of
 // fc1 added in order (deterministic), into fc2's activation buffer.
 __global__ void mlp_reduce_kernel(const float* __restrict__ partial, int32_t nt, int64_t rows, int32_t r2,
-                                  float inv_alpha2, uint8_t* lr2, int32_t RJ2, uint32_t* sk_flags2,
-                                  int32_t sk_flag_words2) {
+                                  float inv_alpha2, uint8_t* lr2, int32_t RJ2) {
   griddep_wait();  // the partials are the previous kernel's output
-  if (blockIdx.x == 0)  // fc2's activation buffer is complete now: its GEMM's stream-K flags start cleared
-    for (int i = int(threadIdx.x); i < sk_flag_words2; i += int(blockDim.x)) sk_flags2[i] = 0u;
   const int groups = r2 / 4;
   const int64_t total = rows * groups;
   const size_t plane = size_t(rows) * size_t(r2);
@@ -438,13 +376,11 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       prefetch_tensormap(&maps.bsf);
       uint32_t it = 0;
       bool stop = false;
-      SegIter work(p, pair);
-      Seg sg;
-      while (!stop && work.next(p, npairs, ntiles, sg)) {
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
         int mp, nt;
-        tile_coords(p, sg.tile, mp, nt);
+        tile_coords(p, tile, mp, nt);
         const int mt = 2 * mp + int(rank);
-        for (int kt = sg.k_lo; kt < sg.k_hi; ++kt) {
+        for (int kt = 0; kt < p.KT; ++kt) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
             fail(0x10u);
@@ -461,7 +397,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           tma_load_2d(st + kOffSFB, &maps.bsf, 0, (nt * p.KT + kt) * kRowsSFB, SFULL + 8u * s);
           ++it;
         }
-        for (int j = 0; j < (sg.fin ? nlr : 0) && !stop; ++j) {
+        for (int j = 0; j < nlr && !stop; ++j) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
             fail(0x10u);
@@ -490,15 +426,13 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       const uint32_t id_fp4 = idesc_nvfp4_m256(kBN), id_bf16 = idesc_bf16_m256(kBN);
       uint32_t it = 0, tc = 0;
       bool stop = false, any = false;
-      SegIter work(p, pair);
-      Seg sg;
-      while (!stop && work.next(p, npairs, ntiles, sg)) {
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
         if (!mbar_wait(ACCE, (tc & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
           fail(0x20u);
           break;
         }
         tc_fence_after();
-        for (int kt = sg.k_lo; kt < sg.k_hi; ++kt) {
+        for (int kt = 0; kt < p.KT; ++kt) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
             fail(0x20u);
@@ -511,12 +445,12 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
 #pragma unroll
           for (uint32_t kb = 0; kb < 4; ++kb)
             umma_nvfp4_pair(tmem, sdesc_sw128(st + kOffA + 32u * kb), sdesc_sw128(st + kOffB + 32u * kb), id_fp4,
-                            sfa + 4u * kb, sfb + 8u * kb, ((kt - sg.k_lo) | int(kb)) ? 1u : 0u);
+                            sfa + 4u * kb, sfb + 8u * kb, (kt | int(kb)) ? 1u : 0u);
           tc_commit_pair_mc(EMPTY + 8u * s, kPairMask);
           any = true;
           ++it;
         }
-        for (int j = 0; j < (sg.fin ? nlr : 0) && !stop; ++j) {
+        for (int j = 0; j < nlr && !stop; ++j) {
           const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
           if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
             fail(0x20u);
@@ -553,11 +487,8 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     const uint32_t lanes = (32u * q) << 16;
     uint32_t it = 0;
     bool stop = false;
-    SegIter work(p, pair);
-    Seg sg;
-    while (!stop && work.next(p, npairs, ntiles, sg)) {
-      const int nk = sg.k_hi - sg.k_lo;
-      for (int k = 0; k < nk + (sg.fin ? nlr : 0) && !stop; ++k) {
+    for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+      for (int k = 0; k < p.KT + nlr && !stop; ++k) {
         const uint32_t s = it % kStages2, ph = (it / kStages2) & 1u;
         bool ok = mbar_wait(SFULL + 8u * s, ph, abort_flag, p.timeout_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
@@ -566,7 +497,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
           stop = true;
           break;
         }
-        if (k < nk) {
+        if (k < p.KT) {
           const uint8_t* st = smem + s * kStage2;
           {
             uint32_t r[16];
@@ -615,10 +546,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
     }
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colq * 64);
-    SegIter work(p, pair);
-    Seg sg;
-    while (work.next(p, npairs, ntiles, sg)) {
-      const int tile = sg.tile;
+    for (int tile = pair; tile < ntiles; tile += npairs) {
       int mp, nt;
       tile_coords(p, tile, mp, nt);
       const int mt = 2 * mp + int(rank);
@@ -642,14 +570,6 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
         break;
       }
       tc_fence_after();
-      // stream-K finisher of a split tile (its pair's last segment: nothing waits behind it): the
-      // pairs that ran the tile's later k-tiles must have left their partials
-      int q0 = 0, q1 = 0;
-      if (sg.fin && sg.k_hi < p.KT) {
-        sk_contributors(p, tile - (ntiles - p.sk_tiles), pair, q0, q1);
-        for (int q = q0; q < q1; ++q)
-          if (!wait_flag(p.sk_flags + q * 2 + int(rank), 1u, p.timeout_ns) && lane == 0) fail(0x200u);
-      }
       uint32_t v[64];
       tmem_ld32(tl, v);
       tmem_ld32(tl + 32u, v + 32);
@@ -657,45 +577,11 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
-      if (!sg.fin) {
-        // stream-K contributor: this CTA's float32 partial of the tile, then its flag (a pair
-        // contributes once, so its slot is its own)
-        float4* dst = p.sk_partial + ((size_t(pair) * 2 + rank) * 64 + size_t(colq) * 16) * kBM + row_in_tile;
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          dst[j * kBM] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                     __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-        __threadfence();
-        named_sync(5, 32 * kEpiWarps);
-        if (threadIdx.x == 0) st_release_gpu(p.sk_flags + pair * 2 + int(rank), 1u);
-        ++tc;
-        continue;
-      }
-      if (sg.k_hi < p.KT) {
-        // stream-K finisher: add the partials of the pairs that ran this tile's later k-tiles,
-        // in pair order (deterministic), then clear their flags for the next launch
-        for (int q = q0; q < q1; ++q) {
-          const float4* src =
-              p.sk_partial + ((size_t(q) * 2 + rank) * 64 + size_t(colq) * 16) * kBM + row_in_tile;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float4 pv = __ldcg(src + j * kBM);
-            v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + pv.x);
-            v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + pv.y);
-            v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + pv.z);
-            v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + pv.w);
-            asm volatile("" ::: "memory");  // one load in flight at a time: no registers for the rest
-          }
-        }
-        named_sync(5, 32 * kEpiWarps);  // every warp has read every partial
-        if (threadIdx.x == 0)
-          for (int q = q0; q < q1; ++q) p.sk_flags[q * 2 + int(rank)] = 0u;
-      }
       const int32_t y0 = mt * kBM + quarter * 32;  // first row of this warp's share
       // On its last tile the CTA's stage ring is idle (every MMA that read it
       // has completed): each warp stages its 4 stores there, 4 KB apart, and
       // never waits for a buffer.
-      const bool last = !work.has_next(p, ntiles);
+      const bool last = tile + npairs >= ntiles;
       if (last) yslot = 0;
       uint8_t* const sbuf = last ? smem + uint32_t(warp) * 4u * kYBufBytes : ybuf;
       const uint32_t sbuf_s = last ? sbase + uint32_t(warp) * 4u * kYBufBytes : ybuf_s;
@@ -1070,20 +956,7 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
     max_pairs[dev & 63].store(clusters);
   }
   const int cap = max_pairs[dev & 63].load();
-  int pairs = int(ntiles < cap ? ntiles : cap);
-  // stream-K of the last wave (plain epilogue only), within the area the activation buffer holds:
-  // the data-parallel tiles stride over all `cap` pairs, the last wave's k-tiles are shared
-  if (kind == kEpiPlain && a.sk_area && cap <= a.sk_max_pairs) {
-    const SkPlan sk = make_sk_plan(ntiles, lg.KT, cap);
-    const size_t need = sk.tiles ? sk_flag_bytes(a.sk_max_pairs) + size_t(sk.pairs) * 2 * kSkCtaBytes : 0;
-    if (sk.tiles && need <= sk_area_bytes(ntiles, a.sk_max_pairs)) {
-      p.sk_tiles = sk.tiles;
-      p.sk_pairs = sk.pairs;
-      p.sk_flags = reinterpret_cast<uint32_t*>(a.sk_area);
-      p.sk_partial = reinterpret_cast<float4*>(a.sk_area + sk_flag_bytes(a.sk_max_pairs));
-      pairs = ntiles > sk.tiles ? cap : sk.pairs;  // all pairs when tiles run whole too
-    }
-  }
+  const int pairs = int(ntiles < cap ? ntiles : cap);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
   cfg.blockDim = dim3(kThreads2, 1, 1);
@@ -1108,7 +981,7 @@ size_t mlp_partial_bytes(int64_t NT1, int64_t MT, int32_t r2) {
 }
 
 cudaError_t launch_mlp_reduce(const MlpReduceLaunch& a, cudaStream_t s) {
-  const int64_t total = a.rows * (a.r2 / 4);  // 0 when fc2 has no ranks: only the flags are cleared
+  const int64_t total = a.rows * (a.r2 / 4);
   int64_t blocks = (total + 255) / 256;
   if (blocks > 8192) blocks = 8192;
   if (blocks < 1) blocks = 1;
@@ -1121,8 +994,7 @@ cudaError_t launch_mlp_reduce(const MlpReduceLaunch& a, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, mlp_reduce_kernel, a.partial, a.nt, a.rows, a.r2, a.inv_alpha2, a.lr2, a.RJ2,
-                            a.sk_flags2, a.sk_flags2 ? a.sk_flag_words2 : 0);
+  return cudaLaunchKernelEx(&cfg, mlp_reduce_kernel, a.partial, a.nt, a.rows, a.r2, a.inv_alpha2, a.lr2, a.RJ2);
 }
 
 cudaError_t launch_rope_pack(const float* rope, int64_t M, float* packed, cudaStream_t s) {

@@ -20,8 +20,6 @@ struct ActQuantLaunch {
   float g_a, c_a, inv_alpha;
   int num_sms;
   uint64_t timeout_ns;
-  uint32_t* sk_flags;    // the activation buffer's stream-K flags, cleared by this kernel
-  int32_t sk_flag_words;
 };
 cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char** why);
 
@@ -55,9 +53,6 @@ struct GemmLaunch {
   int32_t mlp_r2;           // fc2's ranks in use
   float mlp_g_a2, mlp_c_a2;
   float* mlp_partial;
-  // the activation buffer's stream-K area (flags, then partial tiles) and the pairs it was sized for
-  uint8_t* sk_area;
-  int32_t sk_max_pairs;
 };
 cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why);
 
@@ -71,8 +66,6 @@ struct MlpReduceLaunch {
   float inv_alpha2;
   uint8_t* lr2;          // fc2's act buffer + off_lr
   int32_t RJ2;           // fc2's low-rank chunks per row tile
-  uint32_t* sk_flags2;   // fc2's act buffer stream-K flags, cleared here
-  int32_t sk_flag_words2;
 };
 cudaError_t launch_mlp_reduce(const MlpReduceLaunch& a, cudaStream_t s);
 size_t mlp_partial_bytes(int64_t NT1, int64_t MT, int32_t r2);

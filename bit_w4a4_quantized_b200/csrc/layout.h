@@ -144,41 +144,6 @@ SVDQ_HD ActGeom make_act_geom(const LayerGeom& lg, int64_t M) {
   return a;
 }
 
-// Stream-K for the GEMM's last wave: when the 256 x 256 output tiles do not fill the CTA pairs
-// evenly, the tiles of the partial last wave have their K loop split across all pairs (every
-// pair then runs about the same number of k-tiles).  The pair that owns a split tile's first
-// k-tile finishes it; every other pair whose range starts inside the tile leaves a float32
-// partial of its k-tiles (per CTA: 64 column groups x 128 rows of float4 = 128 KB) and raises a
-// flag.  A pair contributes to at most one tile.  The partials and flags sit after the rest of
-// the activation buffer; kernel 1 clears the flags and each finishing CTA clears the flags it
-// consumed.
-struct SkPlan {
-  int32_t tiles;  // tiles in the stream-K phase (0: every tile runs whole on one pair)
-  int32_t pairs;  // pairs sharing them
-};
-constexpr int kSkMaxSplits = 4;      // at most 4 pairs per split tile (bounded fix-up reads)
-constexpr size_t kSkCtaBytes = size_t(kBM) * kBN * 4;  // one CTA's partial tile
-SVDQ_HD SkPlan make_sk_plan(int64_t tiles, int64_t KT, int64_t pairs) {
-  SkPlan s{0, 0};
-  if (pairs < 2 || tiles < 1) return s;
-  const int64_t R = tiles % pairs;
-  if (R == 0) return s;
-  const int64_t per = KT < kSkMaxSplits ? KT : kSkMaxSplits;
-  int64_t P = R * per < pairs ? R * per : pairs;
-  if (R * KT < 2 * P) return s;  // too little work to share: each pair would get under 2 k-tiles
-  s.tiles = int32_t(R);
-  s.pairs = int32_t(P);
-  return s;
-}
-// Bytes of the stream-K area for `tiles` output tiles on at most `max_pairs` pairs: a flag per
-// (pair, CTA), padded to 256 B, then the partial tiles.
-SVDQ_HD size_t sk_flag_bytes(int64_t max_pairs) { return align256(size_t(max_pairs) * 2 * 4); }
-SVDQ_HD size_t sk_area_bytes(int64_t tiles, int64_t max_pairs) {
-  if (tiles < 1 || max_pairs < 2) return 0;
-  const int64_t P = tiles * kSkMaxSplits < max_pairs ? tiles * kSkMaxSplits : max_pairs;
-  return sk_flag_bytes(max_pairs) + size_t(P) * 2 * kSkCtaBytes;
-}
-
 SVDQ_HD size_t acode_off(const ActGeom& a, int64_t m, int64_t k) {
   size_t tile = size_t(m / kBM) * a.KT + size_t(k / kBK);
   return a.off_codes + tile * kATileBytes + sw128(uint32_t(m % kBM), uint32_t((k % kBK) / 2));

@@ -388,27 +388,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Global-memory flag handshake between CTAs of one grid (all resident): a release store
-// after the data, an acquire load before reading it.
-__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-// Bounded wait for *flag == want (false after timeout_ns).
-__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t want, uint64_t timeout_ns) {
-  if (ld_acquire_gpu(flag) == want) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    __nanosleep(128);
-    if (ld_acquire_gpu(flag) == want) return true;
-    if (globaltimer() - t0 > timeout_ns) return false;
-  }
-}
-
 // Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -154,11 +154,7 @@ SVDQ_API svdq_status svdq_prepare_weights(const svdq_prepare_desc* d, void* dev_
 /*
  * Bytes of the per-call activation buffer for M tokens: NVFP4 codes and block
  * scales of X_hat in the GEMM's tiled layout, the bf16 down-projection
- * lr' = (X_hat L1) / (g_a g_w) for rank_capacity ranks, then the GEMM's
- * scratch for the tiles of its last wave when they are split across CTA pairs
- * (flags and float32 partial tiles, sized for half the device's SMs; cleared by
- * svdq_quantize_act).  Host only; the size depends on the layer's device (the
- * current device before upload).
+ * lr' = (X_hat L1) / (g_a g_w) for rank_capacity ranks.  Host only.
  */
 SVDQ_API svdq_status svdq_act_buffer_bytes(const svdq_layer* layer, int64_t M, size_t* bytes);
 
@@ -179,9 +175,7 @@ SVDQ_API svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, i
  * block-scaled MMA and the bf16 up projection accumulating into the same
  * tensor-memory tile.
  * act_buf: the buffer svdq_quantize_act filled for the same M, through this
- *   handle, after its last svdq_lora_swap.  The GEMM also uses the buffer's
- *   scratch tail (partial tiles of the last wave), so two calls whose kernels
- *   may overlap on the GPU must not share one act_buf.  The handle notes the last 64 act_bufs
+ *   handle, after its last svdq_lora_swap.  The handle notes the last 64 act_bufs
  *   it filled; one of those filled before a later swap holds lr' columns of the
  *   replaced factors, and is refused with SVDQ_ERR_INVALID_ARGUMENT (quantize X
  *   again).  A buffer filled through another handle is not checked.
