@@ -22,7 +22,7 @@ LIB = os.path.join(PKG, "libsvdq.so")
 CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 
-CU_SOURCES = ["act_quant.cu", "gemm.cu", "lora.cu", "w4a16.cu"]
+CU_SOURCES = ["act_quant.cu", "gemm.cu", "lora.cu", "mlp_static.cu", "w4a16.cu"]
 CPP_SOURCES = ["api.cpp", "blob.cpp", "prepare.cpp", "svd.cpp"]
 
 NVCC_FLAGS = [

@@ -321,6 +321,25 @@ svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act1, size_t
   return SVDQ_OK;
 }
 
+svdq_status svdq_w4a4_linear_mlp_static(const svdq_layer* fc1, const void* act1, size_t act1_bytes, int64_t M,
+                                        const svdq_layer* fc2, void* act2, size_t act2_bytes, int epilogue,
+                                        void* stream) {
+  if (!fc1 || !fc2) return fail(SVDQ_ERR_INVALID_ARGUMENT, "fc1 and fc2 are required");
+  size_t need = 0;
+  svdq_status st = svdq_mlp_workspace_bytes(fc1, fc2, M, &need);
+  if (st != SVDQ_OK) return st;
+  if (need > svdq::kMlpStaticBytes)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE,
+                "this pair needs " + std::to_string(need) + " bytes of scratch; the library's static area holds " +
+                    std::to_string(svdq::kMlpStaticBytes) + " (pass a workspace to svdq_w4a4_linear_mlp)");
+  if ((st = check_uploaded(fc1)) != SVDQ_OK) return st;
+  void* scratch = nullptr;
+  cudaError_t e = svdq::mlp_static_scratch(fc1->device, &scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(the static MLP scratch)");
+  return svdq_w4a4_linear_mlp(fc1, act1, act1_bytes, M, fc2, act2, act2_bytes, scratch, svdq::kMlpStaticBytes,
+                              epilogue, stream);
+}
+
 svdq_status svdq_rope_packed_bytes(int64_t M, int32_t head_dim, size_t* bytes) {
   if (!bytes) return fail(SVDQ_ERR_INVALID_ARGUMENT, "bytes is required");
   if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");

@@ -68,6 +68,12 @@ struct MlpReduceLaunch {
   int32_t RJ2;           // fc2's low-rank chunks per row tile
 };
 cudaError_t launch_mlp_reduce(const MlpReduceLaunch& a, cudaStream_t s);
+
+// The library's static scratch for the fused MLP pair of callers that cannot allocate
+// (mlp_static.cu): its device address on device `dev`, looked up once per device with that
+// device current.
+constexpr size_t kMlpStaticBytes = size_t(SVDQ_MLP_STATIC_SCRATCH_BYTES);
+cudaError_t mlp_static_scratch(int dev, void** ptr);
 size_t mlp_partial_bytes(int64_t NT1, int64_t MT, int32_t r2);
 
 // [M][64][2] float (cos, sin) -> the packed layout of rope_packed_bytes(M).

@@ -50,6 +50,7 @@ EXPORTED_SYMBOLS = (
     "svdq_rope_packed_bytes", "svdq_rope_pack", "svdq_w4a16_device_bytes", "svdq_w4a16_prepare_host",
     "svdq_w4a16_upload", "svdq_w4a16_linear", "svdq_w4a16_export", "svdq_w4a16_destroy",
     "svdq_layer_serialize", "svdq_layer_import", "svdq_mlp_workspace_bytes", "svdq_w4a4_linear_mlp",
+    "svdq_w4a4_linear_mlp_static",
 )
 
 
@@ -125,6 +126,7 @@ def lib():
         "svdq_layer_serialize": ([vp, vp, sz, ctypes.POINTER(sz)], st),
         "svdq_mlp_workspace_bytes": ([vp, vp, i64, ctypes.POINTER(sz)], st),
         "svdq_w4a4_linear_mlp": ([vp, vp, sz, i64, vp, vp, sz, vp, sz, ctypes.c_int, vp], st),
+        "svdq_w4a4_linear_mlp_static": ([vp, vp, sz, i64, vp, vp, sz, ctypes.c_int, vp], st),
         "svdq_layer_import": ([vp, sz, ctypes.POINTER(vp)], st),
         "svdq_w4a16_device_bytes": ([ctypes.POINTER(W4A16Desc)], sz),
         "svdq_w4a16_prepare_host": ([ctypes.POINTER(W4A16Desc), ctypes.POINTER(vp)], st),

@@ -240,6 +240,29 @@ SVDQ_API svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act
                                           const svdq_layer* fc2, void* act2, size_t act2_bytes, void* workspace,
                                           size_t workspace_bytes, int epilogue, void* stream);
 
+/*
+ * svdq_w4a4_linear_mlp without a workspace argument, for callers that cannot
+ * allocate device memory: code that runs where a cudaMalloc is not allowed or
+ * not wanted (an allocator that owns all of the GPU's memory, a plugin handed
+ * only its inputs and outputs, a framework that forbids allocation inside its
+ * callbacks).  The scratch partials live in one area of
+ * SVDQ_MLP_STATIC_SCRATCH_BYTES inside the library (a __device__ array): every
+ * GPU that loads the library holds it until the process exits.  The pages have
+ * no counterpart; it computes exactly what svdq_w4a4_linear_mlp computes.
+ * The first call on a device looks the area's address up (with that device
+ * current); make that first call before any stream capture.  Every call on a
+ * device shares the one area: calls whose kernels overlap on the GPU (other
+ * streams, other threads) race on it and give wrong results.  Nothing in the
+ * area needs to start at zero (each call overwrites every partial it reads);
+ * it keeps the last call's contents.  A pair whose partials need more than the
+ * area holds (svdq_mlp_workspace_bytes) is refused with
+ * SVDQ_ERR_UNSUPPORTED_SHAPE before anything is launched.  Allocates nothing.
+ */
+#define SVDQ_MLP_STATIC_SCRATCH_BYTES (32u << 20)
+SVDQ_API svdq_status svdq_w4a4_linear_mlp_static(const svdq_layer* fc1, const void* act1, size_t act1_bytes,
+                                                 int64_t M, const svdq_layer* fc2, void* act2, size_t act2_bytes,
+                                                 int epilogue, void* stream);
+
 /* Bytes of the packed rotary table for M rows (head_dim 128).  Host only. */
 SVDQ_API svdq_status svdq_rope_packed_bytes(int64_t M, int32_t head_dim, size_t* bytes);
 
