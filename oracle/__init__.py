@@ -21,7 +21,8 @@ NVFP4 (Blackwell), compute dtype bfloat16, QKV fusion along the output dim,
 and (fused-QKV section) one fused operator for the QKV projection, the Q/K
 normalization and the rotary embedding: ``qkv`` restates that operator.  The
 same page's second kernel family, awq_w4a16 (4-bit weights, 16-bit
-activations, for the modulation projections), is restated in ``w4a16``.
+activations, for the modulation projections), is restated in ``w4a16``; the
+INT4 variant of the 4-bit family (``--precision int4``) in ``int4``.
 
 Every reading the pages leave open (NVFP4 two-level scales, rounding, sign of
 zero, static activation scale, ...) is stated in the

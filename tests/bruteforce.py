@@ -189,3 +189,80 @@ def w4a16_forward(W, X, s, bias=None):
             row.append(y)
         Y.append(row)
     return dict(codes=codes, scales=scales, g=g, Y=Y)
+
+
+# ---------------------------------------------------------------- INT4 variant
+
+
+INT4 = [(Fraction(v), v) for v in range(-7, 8)]  # the symmetric 4-bit integer grid
+
+
+def nearest_int4(x):
+    """Nearest grid integer by exact rational distance, ties to the even integer."""
+    a = Fraction(x)
+    best = None
+    for v, q in INT4:
+        d = abs(a - v)
+        if best is None or d < best[0] or (d == best[0] and q % 2 == 0):
+            best = (d, q)
+    return best[1]
+
+
+def int4_quantize_rows(rows):
+    """Per group of 64: s = bf16(f32(amax / 7)), q = nearest grid integer to f32(t * f32(1 / s))."""
+    codes, scales = [], []
+    for row in rows:
+        rc, rs = [], []
+        for b in range(0, len(row), 64):
+            grp = row[b:b + 64]
+            s = bf16r(f32r(max(abs(t) for t in grp) / 7.0))
+            rcp = 0.0 if s == 0.0 else f32r(1.0 / s)
+            rc += [nearest_int4(f32r(t * rcp)) for t in grp]
+            rs.append(s)
+        codes.append(rc)
+        scales.append(rs)
+    return codes, scales
+
+
+def int4_layer_forward(W, X, act_amax, L1, L2, bias=None, gelu=False):
+    """The INT4 layer on nested lists: smoothing and residual as layer_forward, INT4 quantizer,
+    Y = sum over groups of s_a s_w (q_a . q_w) + (x_hat L1) L2 + b with exact rational sums."""
+    N, K = len(W), len(W[0])
+    M = len(X)
+    r = len(L2)
+    w_amax = [max(abs(W[n][j]) for n in range(N)) for j in range(K)]
+    inv = []
+    lam = []
+    for j in range(K):
+        a, w = act_amax[j], w_amax[j]
+        lj = 1.0 if (a == 0.0 or w == 0.0) else f32r(math.sqrt(f32r(a / w)))
+        lam.append(lj)
+        inv.append(f32r(1.0 / lj))
+    R = [[lam[j] * W[n][j] for n in range(N)] for j in range(K)]
+    for i in range(r):
+        for j in range(K):
+            for n in range(N):
+                R[j][n] = R[j][n] - L1[j][i] * L2[i][n]
+    R32t = [[f32r(R[j][n]) for j in range(K)] for n in range(N)]
+    wc, ws = int4_quantize_rows(R32t)
+    xh = [[bf16r(f32r(X[m][j] * inv[j])) for j in range(K)] for m in range(M)]
+    ac, as_ = int4_quantize_rows(xh)
+    lr = [[sum(Fraction(xh[m][j]) * Fraction(L1[j][i]) for j in range(K)) for i in range(r)] for m in range(M)]
+    Y = []
+    for m in range(M):
+        row = []
+        for n in range(N):
+            y = Fraction(0)
+            for gi in range(K // 64):
+                dot = sum(ac[m][k] * wc[n][k] for k in range(64 * gi, 64 * gi + 64))  # integers
+                y += Fraction(as_[m][gi]) * Fraction(ws[n][gi]) * dot
+            y += sum(lr[m][i] * Fraction(L2[i][n]) for i in range(r))
+            if bias is not None:
+                y += Fraction(bias[n])
+            yf = float(y)
+            if gelu:
+                yf = 0.5 * yf * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (yf + 0.044715 * yf ** 3)))
+            row.append(yf)
+        Y.append(row)
+    return dict(lam=lam, inv=inv, w_codes=wc, w_scales=ws, a_codes=ac, a_scales=as_, x_hat=xh,
+                lr=[[float(v) for v in row] for row in lr], Y=Y)
