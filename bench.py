@@ -562,16 +562,18 @@ def sweep_point(spec, device, steps, factors_cache):
     out = {"workload": spec.name, "M": M, "K": K, "N": N, "rank": spec.rank, "rank_total": r,
            "epilogue": "gelu_tanh" if spec.gelu else "none", "bias": bias is not None}
 
-    def layer_at(rank):
+    def layer_at(rank, fmt):
         fac = None
         if rank > 0:
             L1, L2 = factors_cache[key]
             fac = (np.ascontiguousarray(L1[:, :rank]), np.ascontiguousarray(L2[:rank]))
-        return svdq.Layer(W, amax, rank, bias=bias, factors=fac, device=device)
+        return svdq.Layer(W, amax, rank, bias=bias, factors=fac, device=device, fmt=fmt)
 
     per_set = None
-    for rank, tag in ((r, "fused"), (0, "plain")) if r > 0 else ((0, "plain"),):
-        L0 = layer_at(rank)
+    # the NVFP4 layer at its rank and at rank 0, then the INT4 variant at its rank
+    runs = ((r, "fused", svdq.FMT_NVFP4), (0, "plain", svdq.FMT_NVFP4)) if r > 0 else ((0, "plain", svdq.FMT_NVFP4),)
+    for rank, tag, fmt in runs + ((r, "int4", svdq.FMT_INT4),):
+        L0 = layer_at(rank, fmt)
         per_set = L0.device_bytes + L0.act_buffer_bytes(M) + 2 * M * K + 2 * M * N
         nsets = int(min(8, max(2, math.ceil(3 * L2_BYTES / per_set))))
         layers = [L0] + [L0.clone(device=device) for _ in range(nsets - 1)]
@@ -588,7 +590,7 @@ def sweep_point(spec, device, steps, factors_cache):
                       stream)
         t1 = _graph_seconds(k1, nsets, steps, stream, device)
         t2 = _graph_seconds(k2, nsets, steps, stream, device)
-        if tag != "plain" and spec.name.startswith("qkv") and qkv_shape(N):
+        if tag == "fused" and spec.name.startswith("qkv") and qkv_shape(N):
             # the fused QKV epilogue (per-head Q/K RMSNorm + rotary turn) on the same layers
             nq, nk = (to_dev(w) for w in WL.make_norm_weights(128, spec.seed))
             rope = torch.from_numpy(WL.make_rope(M, 128)).to(device)
@@ -629,6 +631,11 @@ def sweep_point(spec, device, steps, factors_cache):
     t_cb = _graph_seconds(gl, nsets, steps, stream, device)
     out["cublas_bf16_us"] = round(t_cb * 1e6, 3)
     out["cublas_bf16_TFLOPs"] = round(2 * M * N * K / t_cb / 1e12, 1)
+    out["int4_layer_vs_nvfp4"] = round(out["int4_layer_us"] / out["fused_layer_us" if r > 0 else "plain_layer_us"], 3)
+    # the INT4 GEMM runs on the f16 tensor path: its roofline is the measured bf16 rate (f16 runs at the same rate)
+    bf16_peak, _, peak_kind = measured_peaks()
+    out["int4_gemm_frac_of_bf16_peak"] = round(out["int4_gemm_TFLOPs"] / bf16_peak, 3)
+    out["peak_kind"] = peak_kind
     if r > 0:
         out["lowrank_overhead_layer"] = round(out["fused_layer_us"] / out["plain_layer_us"] - 1, 4)
         out["lowrank_overhead_gemm"] = round(out["fused_gemm_us"] / out["plain_gemm_us"] - 1, 4)

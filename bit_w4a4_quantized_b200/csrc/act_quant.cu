@@ -50,7 +50,7 @@ constexpr int kMaxSplits = 8;       // pulled partials: a portable cluster
 constexpr int kMaxPushSplits = 16;  // pushed partials: up to the non-portable cluster size
 constexpr uint32_t kXBytes = kBM * 128;  // 16 KB: 128 rows x 64 bf16
 constexpr uint32_t kInvSlot = 1024;      // 64 floats of 1/lambda (256 B), padded for alignment
-constexpr uint32_t kCtrlBytes = 128;
+constexpr uint32_t kCtrlBytes = 128 + 512;  // + the block-reciprocal table
 
 struct ActQuantParams {
   const float* inv_lam;  // [KC * 64]
@@ -69,7 +69,7 @@ struct ActQuantParams {
 
 // One 16-element block of one row: read x from the swizzled stage, write
 // x_hat back, return 8 bytes of E2M1 codes and the E4M3 block scale.
-__device__ __forceinline__ void quant_block(uint8_t* xrow, uint32_t t7, int g, const float* inv, float g_a,
+__device__ __forceinline__ void quant_block(uint8_t* xrow, uint32_t t7, int g, const float* inv, const float* rtab,
                                             float c_a, bool write_back, uint32_t& w0, uint32_t& w1,
                                             uint32_t& scale) {
   uint4* p0 = reinterpret_cast<uint4*>(xrow + (((2u * g) ^ t7) << 4));
@@ -97,14 +97,54 @@ __device__ __forceinline__ void quant_block(uint8_t* xrow, uint32_t t7, int g, c
     *p1 = make_uint4(h[4], h[5], h[6], h[7]);
   }
   const uint32_t sc = f32_to_e4m3(__fmul_rn(amax, c_a));
-  const float d = __fmul_rn(e4m3_value(sc), g_a);
-  const float rcp = d == 0.0f ? 0.0f : __frcp_rn(d);
+  const float rcp = rtab[sc];
   w0 = f32x8_to_e2m1(__fmul_rn(xh[0], rcp), __fmul_rn(xh[1], rcp), __fmul_rn(xh[2], rcp), __fmul_rn(xh[3], rcp),
                      __fmul_rn(xh[4], rcp), __fmul_rn(xh[5], rcp), __fmul_rn(xh[6], rcp), __fmul_rn(xh[7], rcp));
   w1 = f32x8_to_e2m1(__fmul_rn(xh[8], rcp), __fmul_rn(xh[9], rcp), __fmul_rn(xh[10], rcp),
                      __fmul_rn(xh[11], rcp), __fmul_rn(xh[12], rcp), __fmul_rn(xh[13], rcp),
                      __fmul_rn(xh[14], rcp), __fmul_rn(xh[15], rcp));
   scale = sc;
+}
+
+// INT4 instance: the smoothing half of quant_block for one 16-element block:
+// x_hat (bf16 values, as floats) into xh, written back in place when asked,
+// and the running amax of the block.
+__device__ __forceinline__ void smooth_block(uint8_t* xrow, uint32_t t7, int g, const float* inv, bool write_back,
+                                             float* xh, float& amax) {
+  uint4* p0 = reinterpret_cast<uint4*>(xrow + (((2u * g) ^ t7) << 4));
+  uint4* p1 = reinterpret_cast<uint4*>(xrow + (((2u * g + 1u) ^ t7) << 4));
+  const uint4 a = *p0, b = *p1;
+  const float4* iv = reinterpret_cast<const float4*>(inv);
+  const float4 i0 = iv[0], i1 = iv[1], i2 = iv[2], i3 = iv[3];
+  const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  const float il[16] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w,
+                        i2.x, i2.y, i2.z, i2.w, i3.x, i3.y, i3.z, i3.w};
+  uint32_t h[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float lo = __fmul_rn(bf16lo(in[j]), il[2 * j]);
+    const float hi = __fmul_rn(bf16hi(in[j]), il[2 * j + 1]);
+    h[j] = f32x2_to_bf16x2(lo, hi);
+    xh[2 * j] = bf16lo(h[j]);
+    xh[2 * j + 1] = bf16hi(h[j]);
+    amax = fmaxf(amax, fmaxf(fabsf(xh[2 * j]), fabsf(xh[2 * j + 1])));
+  }
+  if (write_back) {
+    *p0 = make_uint4(h[0], h[1], h[2], h[3]);
+    *p1 = make_uint4(h[4], h[5], h[6], h[7]);
+  }
+}
+
+// Eight INT4 codes q = clamp(rne(x * rcp), -7, 7) as two's-complement nibbles,
+// element 0 in the low nibble.
+__device__ __forceinline__ uint32_t int4x8(const float* x, float rcp) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int q = min(7, max(-7, __float2int_rn(__fmul_rn(x[j], rcp))));
+    w |= (uint32_t(q) & 0xFu) << (4 * j);
+  }
+  return w;
 }
 
 // Scale 8 fp32 ranks by 1/alpha, round to bf16, store 16 bytes of lr'.
@@ -120,7 +160,9 @@ __device__ __forceinline__ void store_lr8(const ActQuantParams& p, int mt, uint3
 
 // kLowRank = false (rank 0) leaves out every tensor-core instruction: a kernel
 // that allocates tensor memory runs one CTA per SM, the plain quantizer two.
-template <bool kLowRank>
+// kInt4 selects the INT4 quantizer (groups of 64, bf16 scales) for the NVFP4 one;
+// the smoothing, the down projection and its reduction are the same.
+template <bool kLowRank, bool kInt4 = false>
 __global__ void __launch_bounds__(kThreads1, 2)
     act_quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const ActQuantParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -163,6 +205,12 @@ __global__ void __launch_bounds__(kThreads1, 2)
     if (lowrank && p.push)  // every CTA of the cluster pushes its partial of these rows
       mbar_expect_tx(RECV, uint32_t(p.splits * (own1 - own0) * p.r_tot * 4));
     fence_mbar_init();
+  }
+  // 1 / d for every block-scale code s (d = value(s) g_a, g_a static; 0 where d is 0): one
+  // shared-memory load per block instead of decoding s and a correctly rounded reciprocal
+  if (threadIdx.x < 128) {
+    const float d = __fmul_rn(e4m3_value(threadIdx.x), p.g_a);
+    reinterpret_cast<float*>(ctrl + 128)[threadIdx.x] = (d == 0.0f || threadIdx.x == 127u) ? 0.0f : __frcp_rn(d);
   }
   if (warp == kMmaWarp1 && lowrank) {
     tmem_alloc(ctrl_s + 112u, p.tmem_cols);
@@ -211,6 +259,41 @@ __global__ void __launch_bounds__(kThreads1, 2)
         mbar_wait(FULL + 8u * (i % kStages1), uint32_t(i / kStages1) & 1u, nullptr, p.timeout_ns);
     }
     __syncwarp();
+  } else if (kInt4 && warp < 8) {
+    // ------------------------------------------------------ INT4 converters
+    // two threads per row, neighbours in a warp: thread (t, h) converts
+    // elements 32 h .. 32 h + 31 of row t; the chunk is one group of 64, whose
+    // amax the pair shares
+    const uint32_t t = uint32_t(warp) * 16u + (uint32_t(lane) >> 1), h = uint32_t(lane) & 1u;
+    const uint32_t t7 = t & 7u;
+    for (int i = 0; i < nchunks; ++i) {
+      const int s = i % kStages1;
+      const uint32_t ph = uint32_t(i / kStages1) & 1u;
+      bool ok = mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);  // the pair's shuffle below needs the whole warp
+      if (!ok) {
+        if (lane == 0) fail(0x2u);
+        break;
+      }
+      uint8_t* stage = smem + size_t(s) * p.stage_bytes;
+      uint8_t* xrow = stage + t * 128u;
+      const float* inv = reinterpret_cast<const float*>(stage + kXBytes);
+      float xh[32];
+      float amax = 0.0f;
+      smooth_block(xrow, t7, int(2 * h), inv + 32 * h, lowrank, xh, amax);
+      smooth_block(xrow, t7, int(2 * h + 1), inv + 32 * h + 16, lowrank, xh + 16, amax);
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      const uint32_t sb = f32x2_to_bf16x2(__fdiv_rn(amax, 7.0f), 0.0f) & 0xFFFFu;  // s = bf16(amax / 7)
+      const float sv = __uint_as_float(sb << 16);
+      const float rcp = sv == 0.0f ? 0.0f : __frcp_rn(sv);
+      const uint4 cw = make_uint4(int4x8(xh, rcp), int4x8(xh + 8, rcp), int4x8(xh + 16, rcp), int4x8(xh + 24, rcp));
+      const int kc = kc0 + i;
+      const size_t blk = size_t(mt) * p.KC + size_t(kc);
+      *reinterpret_cast<uint4*>(p.codes + blk * 4096u + h * 2048u + t * 16u) = cw;
+      if (h == 0) *reinterpret_cast<uint16_t*>(p.sf + (blk * 128u + t) * 2u) = uint16_t(sb);
+      if (lowrank) fence_proxy_async_smem();  // x_hat (generic writes) -> tensor-core reads
+      mbar_arrive(CONV + 8u * s);
+    }
   } else if (warp < 8) {
     // ----------------------------------------------------------- converters
     // two threads per row: thread (t, h) converts elements 32 h .. 32 h + 31
@@ -231,7 +314,8 @@ __global__ void __launch_bounds__(kThreads1, 2)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int g = int(2 * h) + j;
-        quant_block(xrow, t7, g, inv + 16 * g, p.g_a, p.c_a, lowrank, cw[2 * j], cw[2 * j + 1], sc[j]);
+        quant_block(xrow, t7, g, inv + 16 * g, reinterpret_cast<const float*>(ctrl + 128), p.c_a, lowrank, cw[2 * j],
+                    cw[2 * j + 1], sc[j]);
       }
       const int kc = kc0 + i, kt = kc >> 2, sub = kc & 3;
       uint8_t* ctile = p.codes + (size_t(mt) * p.KT + kt) * kATileBytes;
@@ -480,12 +564,13 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   p.timeout_ns = a.timeout_ns;
 
   const bool lowrank = a.r_tot > 0;
-  auto kernel = lowrank ? act_quant_kernel<true> : act_quant_kernel<false>;
+  auto kernel = a.int4 ? (lowrank ? act_quant_kernel<true, true> : act_quant_kernel<false, true>)
+                       : (lowrank ? act_quant_kernel<true> : act_quant_kernel<false>);
   int dev = 0;
   cudaGetDevice(&dev);
   auto set_smem = [&](auto k, int which, size_t bytes) -> cudaError_t {
     // the attributes are per device and kernel: remember the largest size set on each
-    static std::atomic<size_t> smem_set[2][64];
+    static std::atomic<size_t> smem_set[4][64];
     std::atomic<size_t>& done = smem_set[which][dev & 63];
     if (bytes <= done.load()) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
@@ -537,6 +622,8 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
       cudaError_t e = cudaFuncSetAttribute(act_quant_kernel<false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(act_quant_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(act_quant_kernel<true, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       nonportable[dev & 63].store(e == cudaSuccess ? 1 : -1);
     }
     const int cap = nonportable[dev & 63].load() > 0 ? kMaxPushSplits : kMaxSplits;
@@ -577,7 +664,7 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   p.rows_per = rows_per;
   p.rb_bytes = rb_bytes;
   {
-    cudaError_t e = set_smem(kernel, lowrank ? 1 : 0, smem);
+    cudaError_t e = set_smem(kernel, (lowrank ? 1 : 0) + (a.int4 ? 2 : 0), smem);
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
       return e;

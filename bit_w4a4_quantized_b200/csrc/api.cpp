@@ -14,6 +14,7 @@
 
 #include "kernels.h"
 #include "layer.h"
+#include "int4.h"
 #include "w4a16.h"
 
 namespace {
@@ -194,6 +195,7 @@ svdq_status svdq_quantize_act(const svdq_layer* L, const void* X, int64_t M, voi
   a.inv_alpha = L->inv_alpha;
   a.num_sms = L->num_sms;
   a.timeout_ns = svdq::kDefaultTimeoutNs;
+  a.int4 = L->format == SVDQ_FMT_INT4 ? 1 : 0;
   const char* why = "";
   cudaError_t e = svdq::launch_act_quant(a, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
@@ -221,6 +223,27 @@ svdq_status linear_launch(const svdq_layer* L, const void* act_buf, size_t act_b
     return fail(SVDQ_ERR_INVALID_ARGUMENT,
                 "act_buf was quantized before the layer's last LoRA swap; quantize X again (svdq_quantize_act)");
   if ((st = check_device(nullptr, nullptr)) != SVDQ_OK) return st;
+  if (L->format == SVDQ_FMT_INT4) {
+    if (qkv) return fail(SVDQ_ERR_INVALID_ARGUMENT, "the fused QKV epilogue is built for NVFP4 layers only");
+    svdq::Int4GemmLaunch a{};
+    a.act = static_cast<const uint8_t*>(act_buf);
+    a.layer = static_cast<const uint8_t*>(L->dev_buf);
+    a.Y = Y;
+    a.lg = L->g;
+    a.M = M;
+    a.r_tot = L->r_tot;
+    a.has_bias = L->has_bias ? 1 : 0;
+    a.epilogue = epilogue;
+    a.alpha = L->alpha;
+    a.pre_a = 1.0f / L->g_a;  // powers of two: exact
+    a.pre_w = 1.0f / L->g_w;
+    a.num_sms = L->num_sms;
+    a.timeout_ns = svdq::kDefaultTimeoutNs;
+    const char* why = "";
+    cudaError_t e = svdq::launch_gemm_int4(a, static_cast<cudaStream_t>(stream), &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    return SVDQ_OK;
+  }
   svdq::GemmLaunch a = qkv ? *qkv : svdq::GemmLaunch{};
   a.act = static_cast<const uint8_t*>(act_buf);
   a.layer = static_cast<const uint8_t*>(L->dev_buf);
@@ -260,6 +283,8 @@ svdq_status svdq_w4a4_linear_mlp(const svdq_layer* fc1, const void* act1, size_t
   svdq_status st = check_uploaded(fc1);
   if (st != SVDQ_OK) return st;
   if ((st = check_uploaded(fc2)) != SVDQ_OK) return st;
+  if (fc1->format != SVDQ_FMT_NVFP4 || fc2->format != SVDQ_FMT_NVFP4)
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "the fused MLP pair is built for NVFP4 layers only");
   if (!act1 || !act2) return fail(SVDQ_ERR_INVALID_ARGUMENT, "act1 and act2 are required");
   if (M < 1) return fail(SVDQ_ERR_INVALID_ARGUMENT, "M must be >= 1");
   if (M > (int64_t(1) << 31) - 1) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "M too large");
@@ -371,6 +396,8 @@ svdq_status svdq_w4a4_linear_qkv_norm_rope(const svdq_layer* L, const void* act_
                                            float eps, void* stream) {
   svdq_status st = check_uploaded(L);
   if (st != SVDQ_OK) return st;
+  if (L->format != SVDQ_FMT_NVFP4)
+    return fail(SVDQ_ERR_INVALID_ARGUMENT, "the fused QKV epilogue is built for NVFP4 layers only");
   if (head_dim != svdq::kRopeHeadDim) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "head_dim must be 128");
   if (L->g.N % 3 || (L->g.N / 3) % head_dim)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "N must be 3 x a multiple of head_dim (Q | K | V)");
@@ -591,6 +618,7 @@ svdq_status svdq_w4a16_linear(const svdq_w4a16* L, const void* X, int64_t M, voi
   a.gscale = L->gscale;
   a.has_bias = L->has_bias ? 1 : 0;
   a.num_sms = L->num_sms;
+  a.timeout_ns = svdq::kDefaultTimeoutNs;
   const char* why = "";
   cudaError_t e = svdq::launch_w4a16(a, static_cast<cudaStream_t>(stream), &why);
   if (e != cudaSuccess) return cuda_fail(e, why);
@@ -613,6 +641,23 @@ svdq_status svdq_w4a16_export(const svdq_w4a16* L, int what, void* host_dst, siz
   if (bytes < n) return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "export needs " + std::to_string(n) + " bytes");
   std::memcpy(host_dst, src, n);
   return SVDQ_OK;
+}
+
+svdq_status svdq_w4a16_poll_status(const svdq_w4a16* L, void* stream) {
+  if (!L) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is NULL");
+  if (!L->dev_buf) return fail(SVDQ_ERR_INVALID_ARGUMENT, "layer is not uploaded to a device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  uint8_t* status = static_cast<uint8_t*>(L->dev_buf);  // the image's first word
+  cudaError_t e = cudaMemcpyAsync(&word, status, 4, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(status)");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  if (word == 0) return SVDQ_OK;
+  if ((e = cudaMemsetAsync(status, 0, 4, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  char buf[96];
+  std::snprintf(buf, sizeof buf, "the W4A16 kernel gave up a bounded wait (status word 0x%x)", word);
+  return fail(SVDQ_ERR_TIMEOUT, buf);
 }
 
 void svdq_w4a16_destroy(svdq_w4a16* L) { delete L; }

@@ -106,7 +106,8 @@ svdq_status blob_read(const uint8_t* src, size_t bytes, svdq_layer** out, std::s
   if (std::memcmp(h.magic, kMagic, 8) != 0) return *err = "not a layer blob (magic)", SVDQ_ERR_INVALID_ARGUMENT;
   if (h.version != kBlobVersion || h.header_bytes != sizeof(BlobHeader))
     return *err = "unsupported blob version " + std::to_string(h.version), SVDQ_ERR_INVALID_ARGUMENT;
-  if (h.format != SVDQ_FMT_NVFP4) return *err = "unknown format in blob", SVDQ_ERR_INVALID_ARGUMENT;
+  if (h.format != SVDQ_FMT_NVFP4 && h.format != SVDQ_FMT_INT4)
+    return *err = "unknown format in blob", SVDQ_ERR_INVALID_ARGUMENT;
   if (h.K < 64 || h.N < 64 || h.K % 64 || h.N % 64 || h.K > (int64_t(1) << 24) || h.N > (int64_t(1) << 24) ||
       h.rank < 0 || h.rank % 16 || h.rank_capacity < h.rank || h.rank_capacity % 16 ||
       h.rank_capacity > kMaxRankCapacity || h.rank > h.K || h.rank > h.N)

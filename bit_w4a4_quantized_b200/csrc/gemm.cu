@@ -57,6 +57,7 @@
 
 #include <atomic>
 
+#include "int4.h"
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -813,6 +814,353 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
   }
 }
 
+// ------------------------------------------------------------------ INT4 layer
+// Kernel 2 of the INT4 layer (int4.h): the same persistent CTA pairs, tile
+// order, fold of the low-rank branch and plain epilogue as gemm_kernel; the
+// mainloop differs.  tcgen05 has no 4-bit integer MMA kind, so per group of
+// 64 inputs:
+//   * the producer copies this CTA's raw INT4 blocks of A (128 rows) and B
+//     (its 128 of the tile's 256 rows) and their bf16 scales (8.5 KB);
+//   * warps 16-19 widen them in shared memory to f16 values q s 2^e in the
+//     128-byte-swizzled K-major layout the MMA reads (q s is exact in f16 for
+//     a bf16 s, and the prescale 2^e keeps it inside f16's range);
+//   * the leader issues 4 MMAs of kind::f16 (M = 256, N = 256, K = 16) on them.
+// Inside a group of 8 inputs the widened values sit in the order 0 4 1 5 2 6 3 7
+// (two nibbles per 32-bit lane of the unpacking); A and B share that order, so
+// the sum over K is unchanged.
+constexpr int kStages4 = 4;
+constexpr int kConvWarp0 = 16;  // warps 16-19 widen the codes
+constexpr uint32_t kOffA4 = 0;                           // f16 A: 128 rows x 64 (16 KB)
+constexpr uint32_t kOffB4 = kHalf * kRowBytes;           // f16 B: this CTA's 128 rows x 64 (16 KB)
+constexpr uint32_t kOffRawA4 = 2 * kHalf * kRowBytes;    // INT4 block of A (4 KB)
+constexpr uint32_t kOffRawB4 = kOffRawA4 + kBlock4Bytes;  // INT4 block of B (4 KB)
+constexpr uint32_t kOffSA4 = kOffRawB4 + kBlock4Bytes;   // 128 bf16 scales of A
+constexpr uint32_t kOffSB4 = kOffSA4 + kScale4Bytes;     // 128 bf16 scales of B
+constexpr uint32_t kRaw4Bytes = 2 * kBlock4Bytes + 2 * kScale4Bytes;
+constexpr uint32_t kStage4 = (kOffSB4 + kScale4Bytes + 1023u) & ~1023u;  // 41 KB
+constexpr int kFullArrivals4 = 1 + 2 * 4;  // leader producer + the widening warps of both CTAs
+constexpr uint32_t kTmemCols4 = 256;
+constexpr uint32_t kY4 = (kStages4 * kStage4 + kCtrl2 + kBiasBytes + 1023u) & ~1023u;
+constexpr uint32_t kEnd4 = kY4 + kEpiWarps * 2 * kYBufBytes;
+static_assert(kStage4 % 1024 == 0, "stage must keep 1 KB alignment");
+static_assert(kEnd4 + 1024 <= 227 * 1024, "shared memory budget (INT4)");
+static_assert(kEpiWarps * 4 * kYBufBytes <= kStages4 * kStage4, "last-tile staging fits in the stage ring");
+
+struct Int4Params {
+  const uint8_t* a_codes;  // activation INT4 blocks [MT][KC][4 KB]
+  const uint8_t* a_sf;     // activation scales [MT][KC][128] bf16
+  const uint8_t* b_codes;  // weight INT4 blocks [NT][KC][2][4 KB]
+  const uint8_t* b_sf;     // weight scales [NT][KC][256] bf16
+  const uint16_t* bias;    // padded to NT * 256, or null
+  uint16_t* Y;
+  uint32_t* status;
+  int32_t M, N, MP, NT, KC, KG, RJ, r_tot, epilogue;
+  float alpha, pre_a, pre_w;
+  uint64_t timeout_ns;
+};
+
+__host__ __device__ constexpr uint32_t idesc_f16_m256(int n) {
+  return (1u << 4)                    // D format: f32; A, B: f16 (format fields 0)
+         | (uint32_t(n >> 3) << 17)   // N / 8
+         | (uint32_t(256 >> 4) << 24);
+}
+
+// Row t of a 128-row INT4 block and its bf16 scale -> 64 f16 values q s pre,
+// written as row t of a 128-byte-swizzled K-major tile.  The scale saturates
+// at 65504 / 7, so no value overflows to infinity.
+__device__ __forceinline__ void widen_int4_row(const uint8_t* raw, const uint8_t* sc, float pre, uint8_t* dst,
+                                               uint32_t t) {
+  const uint4 c0 = *reinterpret_cast<const uint4*>(raw + t * 16u);          // inputs 0..31
+  const uint4 c1 = *reinterpret_cast<const uint4*>(raw + 2048u + t * 16u);  // inputs 32..63
+  const uint32_t sb = *reinterpret_cast<const uint16_t*>(sc + t * 2u);
+  const float s = fminf(__uint_as_float(sb << 16) * pre, 9357.0f);
+  uint32_t s2;
+  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(s2) : "f"(s));
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  // nibble u (two's complement q) -> f16 1024 + (u ^ 8) = 1032 + q: one LOP3 per two values;
+  // subtracting 1032 leaves q exactly
+  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x64086408u;  // kMagic as f16x2 is (1032, 1032)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t w = words[i];
+    uint32_t v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t h = kMagic ^ ((w >> (4 * j)) & kMask);  // inputs 8 i + j (low), 8 i + j + 4 (high)
+      uint32_t q;
+      asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q) : "r"(h), "r"(kMagic));
+      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(v[j]) : "r"(q), "r"(s2));
+    }
+    *reinterpret_cast<uint4*>(dst + sw128(t, 16u * uint32_t(i))) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_constant__ GemmMaps maps,
+                                                                 const Int4Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_s + pad;
+
+  const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
+  const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int pair = int(blockIdx.x >> 1), npairs = int(gridDim.x >> 1);
+
+  uint8_t* ctrl = smem + kStages4 * kStage4;
+  const uint32_t ctrl_s = sbase + kStages4 * kStage4;
+  const uint32_t FULL = ctrl_s, EMPTY = ctrl_s + 32u, RAW = ctrl_s + 64u;
+  const uint32_t ACCF = ctrl_s + 96u, ACCE = ctrl_s + 104u, DRAIN = ctrl_s + 112u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 120);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 124);
+  uint32_t* bias_s = reinterpret_cast<uint32_t*>(ctrl + kCtrl2);  // [warp][32 bf16 pairs]
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages4; ++s) {
+      mbar_init(FULL + 8u * s, kFullArrivals4);  // leader: producer (+ fold bytes) + 8 widening warps
+      mbar_init(EMPTY + 8u * s, 1);              // both: one multicast commit per phase
+      mbar_init(RAW + 8u * s, 1);                // both: own producer (+ own raw bytes)
+    }
+    mbar_init(ACCF, 1);
+    mbar_init(ACCE, 2 * kEpiWarps);
+    mbar_init(DRAIN, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(ctrl_s + 120u, kTmemCols4);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  auto fail = [&](uint32_t code) {
+    *abort_flag = 1u;
+    atomicOr(p.status, code);
+  };
+
+  const int ntiles = p.MP * p.NT;
+  const int nlr = (p.r_tot + kRChunk - 1) / kRChunk;
+  const int tiles_mp = p.MP, tiles_nt = p.NT;
+  auto coords = [&](int tile, int& mp, int& nt) {
+    const int per_group = kGroupMP * tiles_nt;
+    const int grp = tile / per_group, in = tile % per_group;
+    const int gsize = (tiles_mp - grp * kGroupMP) < kGroupMP ? (tiles_mp - grp * kGroupMP) : kGroupMP;
+    mp = grp * kGroupMP + in % gsize;
+    nt = in / gsize;
+  };
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&maps.lr);
+      prefetch_tensormap(&maps.l2);
+      uint32_t it = 0;
+      bool stop = false;
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+        int mp, nt;
+        coords(tile, mp, nt);
+        const int mt = 2 * mp + int(rank);
+        for (int c = 0; c < p.KG; ++c) {
+          const uint32_t s = it % kStages4, ph = (it / kStages4) & 1u;
+          if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
+            fail(0x10u);
+            stop = true;
+            break;
+          }
+          const uint32_t st = sbase + s * kStage4;
+          if (leader) mbar_arrive(FULL + 8u * s);  // no bytes: the widening warps fill the operands
+          mbar_expect_tx(RAW + 8u * s, kRaw4Bytes);
+          const size_t ablk = size_t(mt) * p.KC + size_t(c);
+          const size_t bblk = size_t(nt) * p.KC + size_t(c);
+          bulk_g2s(st + kOffRawA4, p.a_codes + ablk * kBlock4Bytes, kBlock4Bytes, RAW + 8u * s);
+          bulk_g2s(st + kOffSA4, p.a_sf + ablk * kScale4Bytes, kScale4Bytes, RAW + 8u * s);
+          bulk_g2s(st + kOffRawB4, p.b_codes + (bblk * 2 + rank) * kBlock4Bytes, kBlock4Bytes, RAW + 8u * s);
+          bulk_g2s(st + kOffSB4, p.b_sf + (bblk * 2 + rank) * kScale4Bytes, kScale4Bytes, RAW + 8u * s);
+          ++it;
+        }
+        for (int j = 0; j < nlr && !stop; ++j) {
+          const uint32_t s = it % kStages4, ph = (it / kStages4) & 1u;
+          if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
+            fail(0x10u);
+            stop = true;
+            break;
+          }
+          const uint32_t st = sbase + s * kStage4;
+          const uint32_t bar = mapa(FULL + 8u * s, 0u);
+          if (leader) mbar_expect_tx(FULL + 8u * s, 2u * kFoldBytes);
+          mbar_arrive(RAW + 8u * s);  // nothing to widen: the warps only pass the stage on
+          tma_load_2d_pair(st + kOffA4, &maps.lr, 0, (mt * p.RJ + j) * kRowsA, bar);
+          tma_load_2d_pair(st + kOffB4, &maps.l2, 0, (nt * p.RJ + j) * kRowsBTile + int(rank) * kRowsA, bar);
+          ++it;
+        }
+      }
+      // every issued copy (of both CTAs) must land before the pair may exit
+      for (uint32_t i = it > kStages4 ? it - kStages4 : 0; i < it; ++i) {
+        mbar_wait(RAW + 8u * (i % kStages4), (i / kStages4) & 1u, nullptr, p.timeout_ns);
+        if (leader) mbar_wait_cluster(FULL + 8u * (i % kStages4), (i / kStages4) & 1u, nullptr, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------ MMA issue (leader)
+    if (leader && lane == 0) {
+      const uint32_t id_f16 = idesc_f16_m256(kBN), id_bf16 = idesc_bf16_m256(kBN);
+      uint32_t it = 0, tc = 0;
+      bool stop = false, any = false;
+      for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+        if (!mbar_wait(ACCE, (tc & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+          fail(0x20u);
+          break;
+        }
+        tc_fence_after();
+        for (int c = 0; c < p.KG; ++c) {
+          const uint32_t s = it % kStages4, ph = (it / kStages4) & 1u;
+          if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
+            fail(0x20u);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + s * kStage4;
+#pragma unroll
+          for (uint32_t kk = 0; kk < 4; ++kk)
+            umma_bf16_pair(tmem, sdesc_sw128(st + kOffA4 + 32u * kk), sdesc_sw128(st + kOffB4 + 32u * kk), id_f16,
+                           (c | int(kk)) ? 1u : 0u);
+          tc_commit_pair_mc(EMPTY + 8u * s, kPairMask);
+          any = true;
+          ++it;
+        }
+        for (int j = 0; j < nlr && !stop; ++j) {
+          const uint32_t s = it % kStages4, ph = (it / kStages4) & 1u;
+          if (!mbar_wait_cluster(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
+            fail(0x20u);
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = sbase + s * kStage4;
+          const int left = p.r_tot - kRChunk * j;
+          const int nks = (left < kRChunk ? left : kRChunk) / 16;
+          for (int ks = 0; ks < nks; ++ks)
+            umma_bf16_pair(tmem, sdesc_sw128(st + kOffA4 + 32u * ks), sdesc_sw128(st + kOffB4 + 32u * ks), id_bf16,
+                           1u);
+          tc_commit_pair_mc(EMPTY + 8u * s, kPairMask);
+          ++it;
+        }
+        if (stop) break;
+        tc_commit_pair_mc(ACCF, kPairMask);
+        ++tc;
+      }
+      if (any) {
+        tc_commit_pair(DRAIN);
+        mbar_wait(DRAIN, 0u, nullptr, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kConvWarp0) {  // warps 16-19
+    // ---------------------------------------------------- widening warps
+    const uint32_t t = uint32_t(warp - kConvWarp0) * 32u + uint32_t(lane);  // row of A and of B
+    uint32_t it = 0;
+    bool stop = false;
+    for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
+      for (int k = 0; k < p.KG + nlr && !stop; ++k) {
+        const uint32_t s = it % kStages4, ph = (it / kStages4) & 1u;
+        bool ok = mbar_wait(RAW + 8u * s, ph, abort_flag, p.timeout_ns);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0 && *abort_flag == 0u) fail(0x80u);
+          stop = true;
+          break;
+        }
+        if (k < p.KG) {
+          uint8_t* st = smem + s * kStage4;
+          widen_int4_row(st + kOffRawA4, st + kOffSA4, p.pre_a, st + kOffA4, t);
+          widen_int4_row(st + kOffRawB4, st + kOffSB4, p.pre_w, st + kOffB4, t);
+          fence_proxy_async_smem();  // generic writes -> tensor-core reads
+        }
+        __syncwarp();
+        // the peer's warps arrive remotely at CTA scope, as the NVFP4 scale warps do (an arrive
+        // with release at cluster scope costs about 900 clocks on the stage's critical path)
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(FULL + 8u * s);
+          else
+            mbar_arrive_cluster(FULL + 8u * s, 0u);
+        }
+        ++it;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    // as the plain instance of gemm_kernel: warp w reads TMEM lanes 32 (w % 4)
+    // .. +31 and accumulator columns 64 (w / 4) .. +63, releases the
+    // accumulator, then alpha, bias, GELU -> bf16 -> TMA tensor stores
+    uint32_t tc = 0, yslot = 0;
+    const int quarter = warp & 3, colq = warp >> 2;
+    uint8_t* ybuf = smem + kY4 + uint32_t(warp) * 2u * kYBufBytes;
+    const uint32_t ybuf_s = sbase + kY4 + uint32_t(warp) * 2u * kYBufBytes;
+    const uint32_t tl = tmem + (uint32_t(quarter * 32) << 16) + uint32_t(colq * 64);
+    for (int tile = pair; tile < ntiles; tile += npairs) {
+      int mp, nt;
+      coords(tile, mp, nt);
+      const int mt = 2 * mp + int(rank);
+      uint32_t* bias_w = bias_s + warp * 32;
+      __syncwarp();
+      if (p.bias) bias_w[lane] = *reinterpret_cast<const uint32_t*>(p.bias + size_t(nt) * kBN + colq * 64 + lane * 2);
+      __syncwarp();
+      bool ok = mbar_wait(ACCF, tc & 1u, abort_flag, p.timeout_ns);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      if (!ok) {
+        if (*abort_flag == 0u) fail(0x40u);
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld32(tl, v);
+      tmem_ld32(tl + 32u, v + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(ACCE, 0u);  // this warp's share of the accumulator is free
+      const int32_t y0 = mt * kBM + quarter * 32;
+      const bool last = tile + npairs >= ntiles;
+      if (last) yslot = 0;
+      uint8_t* const sbuf = last ? smem + uint32_t(warp) * 4u * kYBufBytes : ybuf;
+      const uint32_t sbuf_s = last ? sbase + uint32_t(warp) * 4u * kYBufBytes : ybuf_s;
+      GemmParams fp{};  // the fields finish_chunk reads
+      fp.alpha = p.alpha;
+      fp.epilogue = p.epilogue;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int n0 = nt * kBN + colq * 64 + q * 32;
+        if (n0 < p.N) {
+          uint32_t out[16];
+          finish_chunk(fp, v + 32 * q, p.bias ? bias_w + q * 16 : nullptr, out);
+          store_y16<2>(&maps.y, sbuf, sbuf_s, last, lane, out, n0, y0, p.M, yslot);
+          store_y16<2>(&maps.y, sbuf, sbuf_s, last, lane, out + 8, n0 + 16, y0, p.M, yslot);
+        }
+      }
+      ++tc;
+    }
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  cluster_sync();  // both CTAs are done with every MMA, copy and tensor-memory read
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols4);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* f = nullptr;
@@ -973,6 +1321,104 @@ cudaError_t launch_gemm(const GemmLaunch& a, cudaStream_t s, const char** why) {
   cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, maps, p);
   if (e != cudaSuccess) *why = "launch of the GEMM kernel failed";
+  return e;
+}
+
+cudaError_t launch_gemm_int4(const Int4GemmLaunch& a, cudaStream_t s, const char** why) {
+  const LayerGeom& lg = a.lg;
+  const ActGeom ag = make_act_geom(lg, a.M);
+  GemmMaps maps;
+  const uint8_t* act = a.act;
+  const uint8_t* lay = a.layer;
+  bool ok = encode_y(&maps.y, a.Y, a.M, lg.N);
+  if (ok && lg.RJ > 0) {
+    ok = encode_rows(&maps.lr, act + ag.off_lr, uint64_t(ag.MT) * ag.RJ * kATileBytes, kRowsA) &&
+         encode_rows(&maps.l2, lay + lg.off_l2t, uint64_t(lg.NT) * lg.RJ * kBTileBytes, kRowsA);
+  } else {
+    maps.lr = maps.y;  // never read without low-rank chunks
+    maps.l2 = maps.y;
+  }
+  maps.a = maps.asf = maps.b = maps.bsf = maps.y;  // the INT4 operands arrive by bulk copies
+  if (!ok) {
+    *why = "cuTensorMapEncodeTiled rejected a GEMM operand";
+    return cudaErrorInvalidValue;
+  }
+  Int4Params p{};
+  p.a_codes = act + ag.off_codes;
+  p.a_sf = act + ag.off_sf;
+  p.b_codes = lay + lg.off_bcodes;
+  p.b_sf = lay + lg.off_sfb;
+  p.bias = a.has_bias ? reinterpret_cast<const uint16_t*>(lay + lg.off_bias) : nullptr;
+  p.Y = static_cast<uint16_t*>(a.Y);
+  p.status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(lay) + lg.off_status);
+  p.M = int32_t(a.M);
+  p.N = int32_t(lg.N);
+  p.MP = int32_t(ag.MT / 2);
+  p.NT = int32_t(lg.NT);
+  p.KC = int32_t(lg.KC);
+  p.KG = int32_t(lg.K / kGroup4);
+  p.RJ = int32_t(lg.RJ);
+  p.r_tot = a.r_tot;
+  p.epilogue = a.epilogue;
+  p.alpha = a.alpha;
+  p.pre_a = a.pre_a;
+  p.pre_w = a.pre_w;
+  p.timeout_ns = a.timeout_ns;
+  const int64_t ntiles = int64_t(p.MP) * lg.NT;
+  if (ntiles > (int64_t(1) << 30)) {
+    *why = "problem too large for one launch";
+    return cudaErrorInvalidValue;
+  }
+  const size_t smem = size_t(kEnd4) + 1024;
+  static std::atomic<int> max_pairs[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (max_pairs[dev & 63].load() == 0) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               int(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) {
+      *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
+      return e;
+    }
+    cudaLaunchConfig_t q{};
+    q.gridDim = dim3(2 * unsigned(a.num_sms / 2), 1, 1);
+    q.blockDim = dim3(kThreads2, 1, 1);
+    q.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    q.attrs = at;
+    q.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, gemm_int4_kernel, &q);
+    if (e != cudaSuccess || clusters < 1) {
+      *why = "no CTA pair of the INT4 GEMM fits on this device";
+      return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+    }
+    max_pairs[dev & 63].store(clusters);
+  }
+  const int cap = max_pairs[dev & 63].load();
+  const int pairs = int(ntiles < cap ? ntiles : cap);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(kThreads2, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_int4_kernel, maps, p);
+  if (e != cudaSuccess) *why = "launch of the INT4 GEMM kernel failed";
   return e;
 }
 

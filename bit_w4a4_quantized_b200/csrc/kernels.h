@@ -20,6 +20,7 @@ struct ActQuantLaunch {
   float g_a, c_a, inv_alpha;
   int num_sms;
   uint64_t timeout_ns;
+  int32_t int4;          // INT4 layer: groups of 64 with bf16 scales (int4.h) instead of NVFP4
 };
 cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char** why);
 

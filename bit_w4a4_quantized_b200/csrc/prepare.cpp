@@ -20,6 +20,7 @@
 #include <new>
 #include <thread>
 
+#include "int4.h"
 #include "layer.h"
 #include "parallel.h"
 #include "svd.h"
@@ -121,12 +122,45 @@ void quantize_row(const float* t, int64_t k, float g, float c, PutByte&& put_byt
   }
 }
 
+// INT4: per group of 64, s = bf16(f32(amax / 7)), rcp = f32(1 / s) (0 when s is
+// 0), q = clamp(rne(f32(t * rcp)), -7, 7); codes through `put_byte(k, byte)`
+// (two's-complement nibbles, element k even in the low nibble), scales through
+// `put_scale(c, bf16 bits)`.  Returns the row's largest scale value.
+template <class PutByte, class PutScale>
+float quantize_row_int4(const float* t, int64_t k, PutByte&& put_byte, PutScale&& put_scale) {
+  float smax = 0.0f;
+  for (int64_t b = 0; b < k; b += kGroup4) {
+    float amax = 0.0f;
+    for (int i = 0; i < kGroup4; ++i) amax = std::max(amax, std::fabs(t[b + i]));
+    const uint16_t sb = f32_to_bf16_bits(amax / 7.0f);
+    const float s = bf16_bits_to_f32(sb);
+    const float rcp = s == 0.0f ? 0.0f : 1.0f / s;
+    for (int i = 0; i < kGroup4; i += 2) {
+      const float q0 = std::min(7.0f, std::max(-7.0f, std::nearbyint(t[b + i] * rcp)));
+      const float q1 = std::min(7.0f, std::max(-7.0f, std::nearbyint(t[b + i + 1] * rcp)));
+      put_byte(b + i, uint8_t((int(q0) & 0xF) | ((int(q1) & 0xF) << 4)));
+    }
+    put_scale(b / kGroup4, sb);
+    smax = std::max(smax, s);
+  }
+  return smax;
+}
+
+// The power of two 2^e with v 2^e <= 2^top (and > 2^(top - 1)); 0 for v = 0.
+int pow2_exponent(double v, int top) {
+  if (!(v > 0.0)) return 0;
+  int e;
+  std::frexp(v, &e);  // v <= 2^e
+  return std::min(100, std::max(-100, top - e));
+}
+
 }  // namespace
 
 svdq_status validate_desc(const svdq_prepare_desc* d, std::string* err) {
   if (!d) return *err = "descriptor is NULL", SVDQ_ERR_INVALID_ARGUMENT;
   if (!d->W || !d->act_amax) return *err = "W and act_amax are required", SVDQ_ERR_INVALID_ARGUMENT;
-  if (d->format != SVDQ_FMT_NVFP4) return *err = "format must be SVDQ_FMT_NVFP4", SVDQ_ERR_INVALID_ARGUMENT;
+  if (d->format != SVDQ_FMT_NVFP4 && d->format != SVDQ_FMT_INT4)
+    return *err = "format must be SVDQ_FMT_NVFP4 or SVDQ_FMT_INT4", SVDQ_ERR_INVALID_ARGUMENT;
   if ((d->L1 == nullptr) != (d->L2 == nullptr))
     return *err = "give both L1 and L2 or neither", SVDQ_ERR_INVALID_ARGUMENT;
   if (d->K < 64 || d->N < 64 || d->K % 64 || d->N % 64)
@@ -304,6 +338,7 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
       });
     }
     r_buf.reset();
+    const bool int4 = d->format == SVDQ_FMT_INT4;
     float amax_r = 0.0f;
     for (float v : tile_max) amax_r = std::max(amax_r, v);
     L->g_w = global_scale(amax_r);
@@ -329,12 +364,34 @@ svdq_status prepare_host(const svdq_prepare_desc* d, svdq_layer** out, std::stri
       inv_img[k] = k < K ? L->inv_lam[k] : 1.0f;
     }
     if (d->bias) std::memcpy(img + g.off_bias, d->bias, sizeof(uint16_t) * N);
-    parallel_for(N, threads, [&](int64_t n0, int64_t n1) {
-      for (int64_t n = n0; n < n1; ++n)
-        quantize_row(rt + size_t(n) * K, K, L->g_w, c_w,
-                     [&](int64_t k, uint8_t byte) { img[bcode_off(g, n, k)] = byte; },
-                     [&](int64_t s, uint8_t code) { img[bsf_off(g, n, s)] = code; });
-    });
+    if (!int4) {
+      parallel_for(N, threads, [&](int64_t n0, int64_t n1) {
+        for (int64_t n = n0; n < n1; ++n)
+          quantize_row(rt + size_t(n) * K, K, L->g_w, c_w,
+                       [&](int64_t k, uint8_t byte) { img[bcode_off(g, n, k)] = byte; },
+                       [&](int64_t s, uint8_t code) { img[bsf_off(g, n, s)] = code; });
+      });
+    } else {
+      // INT4 codes and bf16 group scales of R^T, then the power-of-two prescales that keep
+      // the kernel's f16 operands q s 2^e in range: the weights' largest value at most 2^15,
+      // the calibration maximum of the activations at most 2^11 (headroom for inputs above it)
+      std::vector<float> row_smax(N, 0.0f);
+      parallel_for(N, threads, [&](int64_t n0, int64_t n1) {
+        for (int64_t n = n0; n < n1; ++n)
+          row_smax[n] = quantize_row_int4(
+              rt + size_t(n) * K, K, [&](int64_t k, uint8_t byte) { img[int4_bcode_off(g, n, k)] = byte; },
+              [&](int64_t c, uint16_t sb) { std::memcpy(img + int4_bsf_off(g, n, c), &sb, 2); });
+      });
+      float smax = 0.0f;
+      for (float v : row_smax) smax = std::max(smax, v);
+      const int ew = pow2_exponent(7.0 * double(smax), 15);
+      const int ea = pow2_exponent(double(amax_xh), 11);
+      L->g_w = std::ldexp(1.0f, -ew);
+      L->g_a = std::ldexp(1.0f, -ea);
+      L->c_a = 0.0f;
+      L->alpha = std::ldexp(1.0f, -(ea + ew));
+      L->inv_alpha = std::ldexp(1.0f, ea + ew);
+    }
     for (int64_t k = 0; k < K; ++k)
       for (int i = 0; i < r; ++i) {
         const uint16_t v = L->l1[size_t(k) * r + i];
@@ -481,9 +538,17 @@ svdq_status export_array(const svdq_layer* L, int what, void* dst, size_t bytes,
     case SVDQ_EXPORT_W_CODES:
       if ((st = need(N * K / 2))) return st;
       for (int64_t n = 0; n < N; ++n)
-        for (int64_t k = 0; k < K; k += 2) out[n * (K / 2) + k / 2] = L->image[bcode_off(g, n, k)];
+        for (int64_t k = 0; k < K; k += 2)
+          out[n * (K / 2) + k / 2] =
+              L->image[L->format == SVDQ_FMT_INT4 ? int4_bcode_off(g, n, k) : bcode_off(g, n, k)];
       return SVDQ_OK;
     case SVDQ_EXPORT_W_SCALES:
+      if (L->format == SVDQ_FMT_INT4) {  // bf16 bits [N, K / 64]
+        if ((st = need(N * (K / 64) * 2))) return st;
+        for (int64_t n = 0; n < N; ++n)
+          for (int64_t c = 0; c < K / 64; ++c) std::memcpy(out + (n * (K / 64) + c) * 2, &L->image[int4_bsf_off(g, n, c)], 2);
+        return SVDQ_OK;
+      }
       if ((st = need(N * K / 16))) return st;
       for (int64_t n = 0; n < N; ++n)
         for (int64_t s = 0; s < K / 16; ++s) out[n * (K / 16) + s] = L->image[bsf_off(g, n, s)];
@@ -520,10 +585,14 @@ svdq_status act_unpack(const svdq_layer* L, int64_t M, const uint8_t* act, size_
     return SVDQ_ERR_BUFFER_TOO_SMALL;
   }
   const int64_t K = g.K;
+  const bool int4 = L->format == SVDQ_FMT_INT4;
   for (int64_t m = 0; m < M; ++m) {
     if (codes)
-      for (int64_t k = 0; k < K; k += 2) codes[m * (K / 2) + k / 2] = act[acode_off(a, m, k)];
-    if (scales)
+      for (int64_t k = 0; k < K; k += 2)
+        codes[m * (K / 2) + k / 2] = act[int4 ? int4_acode_off(a, m, k) : acode_off(a, m, k)];
+    if (scales && int4)  // bf16 bits [M, K / 64]
+      for (int64_t c = 0; c < K / 64; ++c) std::memcpy(scales + (m * (K / 64) + c) * 2, act + int4_asf_off(a, m, c), 2);
+    else if (scales)
       for (int64_t s = 0; s < K / 16; ++s) scales[m * (K / 16) + s] = act[asf_off(a, m, s)];
     if (lr)
       for (int64_t rho = 0; rho < L->r_tot; ++rho) std::memcpy(&lr[m * L->r_tot + rho], act + lr_off(a, m, rho), 2);

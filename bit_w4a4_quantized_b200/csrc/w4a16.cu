@@ -9,20 +9,28 @@
 // hardware E2M1 -> f16x2 conversion, times the E4M3 block scale: exact in f16),
 // B = 16 inputs x 8 rows of X (x~ in shared memory; rows past M are zero
 // operands in registers).  The prepared image stores each 16 x 64 weight tile
-// in fragment order, so one 16-byte load per lane brings the A operands of
-// four MMAs.  A CTA of 8 warps takes a 16-row tile of the output; its warps
-// split K (tile kt goes to warp kt % 8), issue all their weight loads before
-// any arithmetic, and add their partial sums through shared memory in a fixed
-// order.  With one row of X the MMA would be 7/8 padding, so that launch does
+// in fragment order, so one 16-byte read per lane brings the A operands of
+// four MMAs.
+//
+// A CTA takes 16-row tiles of the output in turn.  One producer thread keeps a
+// ring of up to four stages full with bulk copies (cp.async.bulk) of the next
+// tiles' codes and scales, up to 48 weight tiles of 16 x 64 (27 KB) per stage,
+// so the weight stream never waits for the arithmetic; eight compute warps
+// split each row tile's K (tile kt goes to warp kt % 8), read their operands
+// from the stage, and add their partial sums through shared memory in a fixed
+// order, summed by a warp that rotates with the row tile (the partial-sum
+// buffer alternates with the tile, so one barrier per tile suffices).  With one row of X the MMA would be 7/8 padding, so that launch does
 // the same tiles on the CUDA cores instead: mixed-precision fused multiply-adds
 // (f16 operands, float32 accumulator) straight from the f16 weights, no
-// conversion to float32.
+// conversion to float32.  Every wait is bounded: a timeout sets the layer's
+// status word and the CTA drains its copies and exits.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <atomic>
 
 #include "layout.h"
+#include "ptx.cuh"
 #include "w4a16.h"
 
 namespace svdq {
@@ -48,10 +56,12 @@ W4A16Geom make_w4a16_geom(int64_t K, int64_t N) {
 
 namespace {
 
-constexpr int kThreadsW = 256;  // 8 warps
-constexpr int kWarpsW = kThreadsW / 32;
+constexpr int kWarpsW = 8;                   // compute warps
+constexpr int kThreadsW = 32 * kWarpsW + 32;  // + one producer warp
+constexpr int kProducerWarpW = kWarpsW;
 constexpr int kMaxMW = 8;  // rows of X per launch: the MMA's N
-constexpr int kTilesPerWarp = 6;  // weight tiles whose loads a warp issues together (K = 3072: all of them)
+constexpr int kStagesW = 4;
+constexpr uint32_t kTileCodeBytes = 512, kTileScaleBytes = 64;
 
 struct W4A16Params {
   const uint4* codes;   // [N16 / 16][KT][32 lanes] x 16 bytes
@@ -60,8 +70,13 @@ struct W4A16Params {
   const uint16_t* bias;  // or null
   const uint16_t* X;
   uint16_t* Y;
+  uint32_t* status;
   int64_t K, N, M, NT, KT;
   float g;
+  int32_t chunk;   // weight tiles (16 x 64) per stage, a multiple of kWarpsW
+  int32_t stages;  // ring depth, 2 .. kStagesW
+  uint32_t off_red, off_ring, off_ctrl;  // shared-memory sections (bytes)
+  uint64_t timeout_ns;
 };
 
 // Four code bytes (8 E2M1 codes, each byte's first in its low nibble) -> four
@@ -161,41 +176,72 @@ __device__ __forceinline__ void tile_dot(float (*acc)[kM], uint4 cw, uint2 sw, c
 }
 
 // kDot = 0: the MMA path (2 to 8 rows of X); kDot = 1: the CUDA-core path for one row.
-// The one-row instance fits 64 registers, so 4 CTAs share an SM (measured 15.2 -> 14.6 us at K = 3072,
-// N = 18432).  The MMA instance is faster with room for 106 registers and 2 CTAs per SM (M = 4:
-// 18.7 -> 17.3 us) than held to 80 registers and 3.
+// Warps 0-7 compute, warp 8 lane 0 fills the ring.  Stage s holds `chunk` weight tiles of
+// one row tile: their codes (chunk x 512 bytes), then their scales (chunk x 64 bytes).
 template <int kDot>
-__global__ void __launch_bounds__(kThreadsW, kDot ? 4 : 1) w4a16_kernel(const W4A16Params p) {
-  extern __shared__ uint32_t smem_w[];
+__global__ void __launch_bounds__(kThreadsW, 2) w4a16_kernel(const W4A16Params p) {
+  extern __shared__ __align__(128) uint8_t smem_w[];
   const int64_t K = p.K;
   const uint32_t RW = uint32_t(K / 2) + 4;  // x~ row stride in f16 pairs (+4: rows start on different banks)
   const uint32_t MR = uint32_t(p.M);        // rows of x~ kept (B columns past M are zero in registers)
-  uint32_t* xs = smem_w;                    // [M][RW] f16 pairs
-  float* red = reinterpret_cast<float*>(smem_w + MR * RW);  // [8 warps][32 lanes][4]
+  uint32_t* xs = reinterpret_cast<uint32_t*>(smem_w);             // [M][RW] f16 pairs
+  float* red = reinterpret_cast<float*>(smem_w + p.off_red);      // [8 warps][32 lanes][4]
+  const uint32_t ring_s = ptx::smem_u32(smem_w + p.off_ring);
+  const uint32_t stage_bytes = uint32_t(p.chunk) * (kTileCodeBytes + kTileScaleBytes);
+  const uint32_t ctrl_s = ptx::smem_u32(smem_w + p.off_ctrl);
+  const uint32_t FULL = ctrl_s, EMPTY = ctrl_s + 8u * kStagesW;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem_w + p.off_ctrl + 16u * kStagesW);
   const int warp = int(threadIdx.x >> 5), lane = int(threadIdx.x & 31);
   const int g = lane >> 2, c = lane & 3;
+  const int64_t nchunks = (p.KT + p.chunk - 1) / p.chunk;
 
-  // the first tile's weight loads go out before x~ is staged
-  int64_t nt = blockIdx.x;
-  uint4 cw[kTilesPerWarp];
-  uint2 sw[kTilesPerWarp];
-  auto load = [&](int64_t tile, int64_t kt0) {
-#pragma unroll
-    for (int i = 0; i < kTilesPerWarp; ++i) {
-      const int64_t kt = kt0 + int64_t(i) * kWarpsW;
-      if (tile < p.NT && kt < p.KT) {
-        cw[i] = __ldg(p.codes + (tile * p.KT + kt) * 32 + lane);
-        sw[i] = __ldg(p.scales + (tile * p.KT + kt) * 8 + g);
-      } else {
-        cw[i] = make_uint4(0u, 0u, 0u, 0u);
-        sw[i] = make_uint2(0u, 0u);
-      }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      ptx::mbar_init(FULL + 8u * s, 1);
+      ptx::mbar_init(EMPTY + 8u * s, kWarpsW);
     }
+    *abort_flag = 0u;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  auto fail = [&](uint32_t code) {
+    *abort_flag = 1u;
+    atomicOr(p.status, code);
   };
-  load(nt, warp);
 
-  // x~ = f16(x / s), saturating
-  for (uint32_t i = threadIdx.x; i < MR * uint32_t(K / 2); i += kThreadsW) {
+  if (warp == kProducerWarpW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t u = 0;
+      bool stop = false;
+      for (int64_t nt = blockIdx.x; nt < p.NT && !stop; nt += gridDim.x) {
+        for (int64_t ch = 0; ch < nchunks; ++ch, ++u) {
+          const uint32_t s = u % uint32_t(p.stages), ph = (u / uint32_t(p.stages)) & 1u;
+          if (!ptx::mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
+            fail(0x100u);
+            stop = true;
+            break;
+          }
+          const int64_t kt0 = ch * p.chunk;
+          const uint32_t n = uint32_t(p.KT - kt0 < p.chunk ? p.KT - kt0 : p.chunk);
+          const uint32_t st = ring_s + s * stage_bytes;
+          ptx::mbar_expect_tx(FULL + 8u * s, n * (kTileCodeBytes + kTileScaleBytes));
+          ptx::bulk_g2s(st, p.codes + (nt * p.KT + kt0) * 32, n * kTileCodeBytes, FULL + 8u * s);
+          ptx::bulk_g2s(st + uint32_t(p.chunk) * kTileCodeBytes, p.scales + (nt * p.KT + kt0) * 8,
+                        n * kTileScaleBytes, FULL + 8u * s);
+        }
+      }
+      // every issued copy must land before the CTA may exit
+      const uint32_t S = uint32_t(p.stages);
+      for (uint32_t i = u > S ? u - S : 0; i < u; ++i)
+        ptx::mbar_wait(FULL + 8u * (i % S), (i / S) & 1u, nullptr, p.timeout_ns);
+    }
+    return;  // the compute warps' barriers below count 256 threads
+  }
+
+  // ------------------------------------------------------------- compute
+  // x~ = f16(x / s), saturating (the producer's first copies are already in flight)
+  for (uint32_t i = threadIdx.x; i < MR * uint32_t(K / 2); i += 32 * kWarpsW) {
     const uint32_t m = i / uint32_t(K / 2), w = i % uint32_t(K / 2);
     const uint32_t xb = *reinterpret_cast<const uint32_t*>(p.X + int64_t(m) * K + 2 * int64_t(w));
     const float2 is = *reinterpret_cast<const float2*>(p.inv_s + 2 * int64_t(w));
@@ -204,29 +250,43 @@ __global__ void __launch_bounds__(kThreadsW, kDot ? 4 : 1) w4a16_kernel(const W4
     const __half2 h = __floats2half2_rn(lo, hi);
     xs[m * RW + w] = *reinterpret_cast<const uint32_t*>(&h);
   }
-  __syncthreads();
+  ptx::named_sync(1, 32 * kWarpsW);
 
-  for (; nt < p.NT; nt += gridDim.x) {
+  // Every compute warp runs the same loop and meets every barrier, also after a
+  // timeout (it then skips the work); only the producer leaves early.
+  uint32_t u = 0, tcount = 0;
+  bool bad = false;
+  for (int64_t nt = blockIdx.x; nt < p.NT; nt += gridDim.x) {
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     float dacc[2][kDot > 0 ? kDot : 1] = {};
     const uint32_t* xrow = uint32_t(g) < MR ? xs + uint32_t(g) * RW : nullptr;
-    for (int64_t kt0 = warp;; kt0 += int64_t(kTilesPerWarp) * kWarpsW) {
-#pragma unroll
-      for (int i = 0; i < kTilesPerWarp; ++i) {
-        const int64_t kt = kt0 + int64_t(i) * kWarpsW;
-        if (kt < p.KT) {
-          if constexpr (kDot > 0)
-            tile_dot<kDot>(dacc, cw[i], sw[i], xs + uint32_t(kt) * 32u, RW, c);
-          else
-            tile_mma(acc, cw[i], sw[i], xrow ? xrow + uint32_t(kt) * 32u : nullptr, c);
+    for (int64_t ch = 0; ch < nchunks; ++ch, ++u) {
+      const uint32_t s = u % uint32_t(p.stages), ph = (u / uint32_t(p.stages)) & 1u;
+      if (!bad) {
+        bool ok = ptx::mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (!ok) {
+          if (lane == 0 && *abort_flag == 0u) fail(0x200u);
+          bad = true;
         }
       }
-      const int64_t next = kt0 + int64_t(kTilesPerWarp) * kWarpsW;
-      if (next < p.KT) {
-        load(nt, next);  // more of this row tile (K > 3072)
-      } else {
-        load(nt + gridDim.x, warp);  // the next row tile's first loads overlap the reduction
-        break;
+      if (!bad) {
+        const int64_t kt0 = ch * p.chunk;
+        const int n = int(p.KT - kt0 < p.chunk ? p.KT - kt0 : p.chunk);
+        const uint8_t* st = smem_w + p.off_ring + s * stage_bytes;
+        const uint4* cws = reinterpret_cast<const uint4*>(st);
+        const uint2* sws = reinterpret_cast<const uint2*>(st + uint32_t(p.chunk) * kTileCodeBytes);
+        for (int i = warp; i < n; i += kWarpsW) {
+          const uint32_t kt = uint32_t(kt0) + uint32_t(i);
+          const uint4 cw = cws[i * 32 + lane];
+          const uint2 sw = sws[i * 8 + g];
+          if constexpr (kDot > 0)
+            tile_dot<kDot>(dacc, cw, sw, xs + kt * 32u, RW, c);
+          else
+            tile_mma(acc, cw, sw, xrow ? xrow + kt * 32u : nullptr, c);
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(EMPTY + 8u * s);  // this warp is done with the stage
       }
     }
     if constexpr (kDot > 0) {
@@ -245,18 +305,20 @@ __global__ void __launch_bounds__(kThreadsW, kDot ? 4 : 1) w4a16_kernel(const W4
       acc[1] = (c == 0 && kDot > 1) ? dacc[0][kDot > 1 ? 1 : 0] : 0.0f;
       acc[3] = (c == 0 && kDot > 1) ? dacc[1][kDot > 1 ? 1 : 0] : 0.0f;
     }
-    // the 8 warps' partial tiles, added in warp order
-    *reinterpret_cast<float4*>(red + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    __syncthreads();
-    if (warp == 0) {
-      float4 t = *reinterpret_cast<const float4*>(red + lane * 4);
+    // the 8 warps' partial tiles, added in warp order by one warp (rotating); the buffer
+    // alternates with the row tile, so one barrier per tile suffices
+    float* rb = red + (tcount & 1u) * (kWarpsW * 32 * 4);
+    *reinterpret_cast<float4*>(rb + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    ptx::named_sync(1, 32 * kWarpsW);
+    if (warp == int(tcount % kWarpsW) && !bad) {
+      float4 t = *reinterpret_cast<const float4*>(rb + lane * 4);
 #pragma unroll
       for (int w = 1; w < kWarpsW; ++w) {
-        const float4 u = *reinterpret_cast<const float4*>(red + (w * 32 + lane) * 4);
-        t.x += u.x;
-        t.y += u.y;
-        t.z += u.z;
-        t.w += u.w;
+        const float4 v = *reinterpret_cast<const float4*>(rb + (w * 32 + lane) * 4);
+        t.x += v.x;
+        t.y += v.y;
+        t.z += v.z;
+        t.w += v.w;
       }
       // lane (g, c): rows n = 16 nt + g (x, y) and + 8 (z, w); X rows m = 2 c (x, z) and 2 c + 1 (y, w)
       const float v[4] = {t.x, t.y, t.z, t.w};
@@ -271,7 +333,7 @@ __global__ void __launch_bounds__(kThreadsW, kDot ? 4 : 1) w4a16_kernel(const W4
         }
       }
     }
-    __syncthreads();  // red is rewritten by the next row tile
+    ++tcount;
   }
 }
 
@@ -307,17 +369,48 @@ cudaError_t launch_w4a16(const W4A16Launch& a, cudaStream_t s, const char** why)
   p.scales = reinterpret_cast<const uint2*>(a.layer + a.g.off_scales);
   p.inv_s = reinterpret_cast<const float*>(a.layer + a.g.off_inv_s);
   p.bias = a.has_bias ? reinterpret_cast<const uint16_t*>(a.layer + a.g.off_bias) : nullptr;
+  p.status = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(a.layer));  // the image's first word
   p.K = a.g.K;
   p.N = a.g.N;
   p.NT = a.g.N16 / 16;
   p.KT = a.g.KT;
   p.g = a.gscale;
+  p.timeout_ns = a.timeout_ns;
   // rows of X in launches of at most 8 (the MMA's N), stream ordered
   for (int64_t m0 = 0; m0 < a.M; m0 += kMaxMW) {
     p.X = a.X + m0 * a.g.K;
     p.Y = a.Y + m0 * a.g.N;
     p.M = a.M - m0 < kMaxMW ? a.M - m0 : kMaxMW;
-    const size_t smem = (size_t(p.M) * size_t(a.g.K / 2 + 4) + size_t(kThreadsW) * 4) * 4;
+    // shared memory: x~ | partial sums | ring | barriers.  Two CTAs per SM if a ring of two
+    // or more stages (40 KB or more, or all of K) fits in half the SM, else one CTA; the
+    // largest stage first.
+    const size_t xs_bytes = size_t(round_up(int64_t(p.M) * (a.g.K / 2 + 4) * 4, 128));
+    const size_t red_bytes = 2 * size_t(kWarpsW) * 32 * 16, ctrl_bytes = 128;
+    const size_t fixed = xs_bytes + red_bytes + ctrl_bytes;
+    const int64_t max_chunk = round_up(p.KT, kWarpsW);
+    size_t smem = 0;
+    for (size_t budget : {size_t(113) * 1024, size_t(227) * 1024}) {
+      for (int64_t chunk = 48; chunk >= kWarpsW && smem == 0; chunk -= kWarpsW) {
+        const int64_t ck = chunk < max_chunk ? chunk : max_chunk;
+        const size_t stage = size_t(ck) * (kTileCodeBytes + kTileScaleBytes);
+        if (fixed + 2 * stage > budget) continue;
+        int64_t st = int64_t((budget - fixed) / stage);
+        if (st > kStagesW) st = kStagesW;
+        // two CTAs per SM only with at least 40 KB of weights in flight per CTA
+        if (budget < size_t(227) * 1024 && size_t(st) * stage < size_t(40) * 1024 && ck < max_chunk) continue;
+        p.chunk = int32_t(ck);
+        p.stages = int32_t(st);
+        smem = fixed + size_t(st) * stage;
+      }
+      if (smem) break;
+    }
+    if (smem == 0) {
+      *why = "K is too large for the W4A16 kernel (x~ leaves no room for its weight ring)";
+      return cudaErrorInvalidConfiguration;
+    }
+    p.off_red = uint32_t(xs_bytes);
+    p.off_ring = uint32_t(xs_bytes + red_bytes);
+    p.off_ctrl = uint32_t(xs_bytes + red_bytes + size_t(p.stages) * size_t(p.chunk) * (kTileCodeBytes + kTileScaleBytes));
     const int per_sm = p.M == 1 ? blocks_per_sm<1>(smem) : blocks_per_sm<0>(smem);
     if (per_sm < 1) {
       *why = "the W4A16 kernel does not fit on this device";
@@ -325,7 +418,7 @@ cudaError_t launch_w4a16(const W4A16Launch& a, cudaStream_t s, const char** why)
     }
     int64_t blocks = int64_t(per_sm) * a.num_sms;
     if (blocks > p.NT) blocks = p.NT;
-    if (p.M == 1)  // one row of X: the CUDA cores (measured 15 us against 18 us for the MMA at M = 1..4)
+    if (p.M == 1)  // one row of X: the CUDA cores (the MMA's 8 columns would be 7/8 padding)
       w4a16_kernel<1><<<unsigned(blocks), kThreadsW, smem, s>>>(p);
     else
       w4a16_kernel<0><<<unsigned(blocks), kThreadsW, smem, s>>>(p);

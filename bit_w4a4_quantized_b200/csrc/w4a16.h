@@ -40,6 +40,7 @@ struct W4A16Launch {
   float gscale;
   int32_t has_bias;
   int num_sms;
+  uint64_t timeout_ns;  // per bounded wait; a timeout sets the image's status word
 };
 cudaError_t launch_w4a16(const W4A16Launch& a, cudaStream_t s, const char** why);
 

@@ -25,6 +25,7 @@ ERR_INTERNAL = 7
 ERR_HOST_ALLOC = 8
 
 FMT_NVFP4 = 1
+FMT_INT4 = 2
 PREPARE_KEEP_R = 1
 EPI_NONE = 0
 EPI_GELU_TANH = 1
@@ -48,7 +49,8 @@ EXPORTED_SYMBOLS = (
     "svdq_get_layer_info", "svdq_poll_status", "svdq_layer_destroy", "svdq_test_override_device_arch",
     "svdq_test_bounded_wait", "svdq_layer_clone", "svdq_w4a4_linear_qkv_norm_rope",
     "svdq_rope_packed_bytes", "svdq_rope_pack", "svdq_w4a16_device_bytes", "svdq_w4a16_prepare_host",
-    "svdq_w4a16_upload", "svdq_w4a16_linear", "svdq_w4a16_export", "svdq_w4a16_destroy",
+    "svdq_w4a16_upload", "svdq_w4a16_linear", "svdq_w4a16_export", "svdq_w4a16_poll_status",
+    "svdq_w4a16_destroy",
     "svdq_layer_serialize", "svdq_layer_import", "svdq_mlp_workspace_bytes", "svdq_w4a4_linear_mlp",
     "svdq_w4a4_linear_mlp_static",
 )
@@ -133,6 +135,7 @@ def lib():
         "svdq_w4a16_upload": ([vp, vp, sz, vp], st),
         "svdq_w4a16_linear": ([vp, vp, i64, vp, vp], st),
         "svdq_w4a16_export": ([vp, ctypes.c_int, vp, sz], st),
+        "svdq_w4a16_poll_status": ([vp, vp], st),
         "svdq_w4a16_destroy": ([vp], None),
         "svdq_test_override_device_arch": ([ctypes.c_int], None),
         "svdq_test_bounded_wait": ([ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32), vp], st),
@@ -254,7 +257,8 @@ class Layer:
     """One prepared SVDQuant W4A4 + low-rank layer (host handle + device image)."""
 
     def __init__(self, W, act_amax, rank, *, rank_capacity=None, bias=None, factors=None, seed=0, threads=0,
-                 keep_r=False, power_iters=0, oversample=0, device=None, stream=None):
+                 keep_r=False, power_iters=0, oversample=0, device=None, stream=None, fmt=FMT_NVFP4):
+        """fmt: FMT_NVFP4 (E2M1 codes, E4M3 scales per 16) or FMT_INT4 (codes -7..7, bf16 scales per 64)."""
         self._h = None
         w = _bf16_bits(W)
         self.N, self.K = w.shape
@@ -267,7 +271,7 @@ class Layer:
         d = PrepareDesc()
         d.K, d.N, d.rank = self.K, self.N, rank
         d.rank_capacity = rank if rank_capacity is None else rank_capacity
-        d.format = FMT_NVFP4
+        d.format = fmt
         d.num_threads = threads
         d.flags = PREPARE_KEEP_R if keep_r else 0
         d.W, d.bias, d.act_amax = _ptr(w), _ptr(b), _ptr(amax)
@@ -282,6 +286,7 @@ class Layer:
         self._h = h
         self._keep = None
         self.rank = rank
+        self.fmt = fmt
         self.dev_buf = None
         if device is not None:
             self.upload(device, stream)
@@ -293,6 +298,7 @@ class Layer:
         c = Layer.__new__(Layer)
         c._h, c._keep, c.desc = h, None, self.desc
         c.N, c.K, c.rank, c.device_bytes, c.dev_buf = self.N, self.K, self.rank, self.device_bytes, None
+        c.fmt = self.fmt
         if device is not None:
             c.upload(device, stream)
         return c
@@ -316,6 +322,7 @@ class Layer:
         i = LayerInfo()
         check(lib().svdq_get_layer_info(h, ctypes.byref(i)))
         c.N, c.K, c.rank, c.device_bytes = i.N, i.K, i.rank, i.device_bytes
+        c.fmt = i.format
         if device is not None:
             c.upload(device, stream)
         return c
@@ -457,17 +464,21 @@ class Layer:
             EXPORT_W_SCALES: ((N, K // 16), np.uint8), EXPORT_SIGMA: ((r,), np.float64),
             EXPORT_SCALARS: ((4,), np.float32), EXPORT_RESID_NORM: ((2,), np.float64),
         }
+        if self.fmt == FMT_INT4:  # bf16 bits of one scale per 64 inputs
+            shapes[EXPORT_W_SCALES] = ((N, K // 64), np.uint16)
         shape, dt = shapes[what]
         out = np.empty(shape, dtype=dt)
         check(lib().svdq_layer_export(self._h, what, out.ctypes.data, out.nbytes))
         return out
 
     def act_unpack(self, act_host, M):
-        """Logical codes [M, K/2], scales [M, K/16], lr bf16 bits [M, r_tot] of a host copy."""
+        """Logical codes [M, K/2], scales [M, K/16] (INT4: bf16 bits [M, K/64]), lr bf16 bits [M, r_tot]
+        of a host copy."""
         a = np.ascontiguousarray(np.asarray(act_host, dtype=np.uint8))
         rt = self.info().rank_total
         codes = np.empty((M, self.K // 2), np.uint8)
-        scales = np.empty((M, self.K // 16), np.uint8)
+        scales = np.empty((M, self.K // 64), np.uint16) if self.fmt == FMT_INT4 else np.empty((M, self.K // 16),
+                                                                                               np.uint8)
         lr = np.empty((M, rt), np.uint16)
         check(lib().svdq_act_unpack(self._h, M, a.ctypes.data, a.nbytes, codes.ctypes.data, scales.ctypes.data,
                                     lr.ctypes.data if rt else None))
@@ -539,6 +550,10 @@ class W4A16Layer:
         out = np.empty(shape, dtype=dt)
         check(lib().svdq_w4a16_export(self._h, what, out.ctypes.data, out.nbytes))
         return out
+
+    def poll_status(self, stream=None):
+        """Raise SvdqError if the kernel gave up a bounded wait since the last poll."""
+        check(lib().svdq_w4a16_poll_status(self._h, _stream(stream)))
 
     def close(self):
         if self._h is not None and _lib is not None:

@@ -73,7 +73,23 @@ typedef enum svdq_status {
 
 typedef struct svdq_layer svdq_layer; /* opaque host handle of one prepared layer */
 
-enum { SVDQ_FMT_NVFP4 = 1 };
+/*
+ * 4-bit formats (the Diffusers/Nunchaku page: the svdq_w4a4 kernel family has
+ * NVFP4 and INT4 variants, chosen by --precision nvfp4|int4 at quantization):
+ *   SVDQ_FMT_NVFP4: E2M1 codes with an E4M3 scale per 16 elements along K and a
+ *     float32 tensor scale (g_a for X_hat, g_w for R);
+ *   SVDQ_FMT_INT4: codes -7..7 with a bf16 scale per 64 elements along K,
+ *     s = bf16(amax / 7) (the summary page's quantizer round(X / s),
+ *     s = max|X| / q_max, with q_max = 7); no tensor scale.  tcgen05 has no
+ *     4-bit integer MMA, so kernel 2 widens the codes to f16 values q s 2^e in
+ *     shared memory and runs the f16 MMA; e is a per-layer power of two (e_a
+ *     for X_hat from the calibration maximum, e_w for R), reported as
+ *     g_a = 2^-e_a and g_w = 2^-e_w.  Inputs whose |X_hat| exceeds 32 times the
+ *     calibration maximum saturate in that operand (a scale above 65504 / 7
+ *     after the prescale is clamped there).  The fused QKV and MLP entry points
+ *     take NVFP4 layers only.
+ */
+enum { SVDQ_FMT_NVFP4 = 1, SVDQ_FMT_INT4 = 2 };
 enum { SVDQ_PREPARE_KEEP_R = 1 /* keep float32 R in the handle for SVDQ_EXPORT_R */ };
 enum { SVDQ_EPI_NONE = 0, SVDQ_EPI_GELU_TANH = 1 };
 
@@ -88,7 +104,7 @@ typedef struct svdq_prepare_desc {
                               W_q, W_k, W_v concatenated along N in that order)    */
   int32_t rank;            /* r of the low-rank branch, multiple of 16, may be 0   */
   int32_t rank_capacity;   /* >= rank, multiple of 16, <= 256: room for LoRA ranks */
-  int32_t format;          /* SVDQ_FMT_NVFP4                                       */
+  int32_t format;          /* SVDQ_FMT_NVFP4 or SVDQ_FMT_INT4                      */
   int32_t num_threads;     /* host threads for preparation; 0 = all cores          */
   int32_t flags;           /* SVDQ_PREPARE_* bits                                  */
   const uint16_t* W;       /* host bf16 [N, K] row-major (nn.Linear weight)        */
@@ -162,7 +178,8 @@ SVDQ_API svdq_status svdq_act_buffer_bytes(const svdq_layer* layer, int64_t M, s
  * Kernel 1 (Nunchaku fusion of the down projection into the quantizer,
  * SVDQuant summary page section 4.3 / Figure 6(b)).  One pass over X:
  *   x_hat = bf16(x / lambda); per 16 elements along K: E4M3 block scale,
- *   E2M1 codes; lr' = bf16((x_hat L1) / (g_a g_w)) on the tensor cores.
+ *   E2M1 codes (INT4 layer: per 64 elements a bf16 scale and codes -7..7);
+ *   lr' = bf16((x_hat L1) / (g_a g_w)) on the tensor cores.
  * X: device bf16 [M, K] row-major, 16-byte aligned, row stride K.
  * act_buf: device, >= svdq_act_buffer_bytes(M) bytes, 256-byte aligned.
  */
@@ -173,7 +190,8 @@ SVDQ_API svdq_status svdq_quantize_act(const svdq_layer* layer, const void* X, i
  * Kernel 2 (Nunchaku fusion of the up projection into the 4-bit GEMM, same
  * section): Y = act(g_a g_w (Q(X_hat) Q(R) + lr' L2) + b) with the FP4
  * block-scaled MMA and the bf16 up projection accumulating into the same
- * tensor-memory tile.
+ * tensor-memory tile (INT4 layer: the f16 MMA on the widened codes, see
+ * SVDQ_FMT_INT4).
  * act_buf: the buffer svdq_quantize_act filled for the same M, through this
  *   handle, after its last svdq_lora_swap.  The handle notes the last 64 act_bufs
  *   it filled; one of those filled before a later swap holds lr' columns of the
@@ -299,8 +317,9 @@ enum {
   SVDQ_EXPORT_L2 = 4,         /* bf16 [rank, N]                                   */
   SVDQ_EXPORT_R = 5,          /* float [K, N] = float32(R)                        */
   SVDQ_EXPORT_W_CODES = 6,    /* uint8 [N, K/2] E2M1 codes of R^T, element 2i in
-                                 the low nibble                                   */
-  SVDQ_EXPORT_W_SCALES = 7,   /* uint8 [N, K/16] E4M3 block scales                */
+                                 the low nibble (INT4: two's-complement codes)    */
+  SVDQ_EXPORT_W_SCALES = 7,   /* uint8 [N, K/16] E4M3 block scales (INT4: bf16
+                                 bits [N, K/64], N K / 32 bytes)                  */
   SVDQ_EXPORT_SIGMA = 8,      /* double [rank] singular values (library SVD only) */
   SVDQ_EXPORT_SCALARS = 9,    /* float [4]: g_a, g_w, alpha = g_a g_w, 1/alpha    */
   SVDQ_EXPORT_RESID_NORM = 10 /* double [2]: ||W_hat^T - L1 L2||_F with float64
@@ -313,7 +332,9 @@ SVDQ_API svdq_status svdq_layer_export(const svdq_layer* layer, int what, void* 
 /*
  * Unpack a host copy of an activation buffer (M rows) into logical layouts:
  * codes uint8 [M, K/2], scales uint8 [M, K/16], lr bf16 [M, rank_total]
- * (rank_total = rank + attached LoRA rank).  Any output may be NULL.
+ * (rank_total = rank + attached LoRA rank).  Any output may be NULL.  For an
+ * INT4 layer the codes are two's-complement nibbles and `scales` receives bf16
+ * bits [M, K/64] (M K / 32 bytes).
  */
 SVDQ_API svdq_status svdq_act_unpack(const svdq_layer* layer, int64_t M, const void* act_host, size_t bytes,
                             uint8_t* codes, uint8_t* scales, uint16_t* lr);
@@ -408,8 +429,10 @@ SVDQ_API svdq_status svdq_w4a16_upload(svdq_w4a16* layer, void* dev_buf, size_t 
 /*
  * Y = g f16(X diag(s)^-1) deq^T + b.  X: device bf16 [M, K] row-major,
  * 16-byte aligned; Y: device bf16 [M, N] row-major, 2-byte aligned; any M >= 1
- * (rows go 8 at a time, one launch each, stream ordered).  No bounded waits:
- * the kernel's CTAs never wait on one another.
+ * (rows go 8 at a time, one launch each, stream ordered).  Inside a CTA the
+ * weight ring's waits are bounded: a wait that gives up sets the status word
+ * of the layer's image and the CTA drains its copies and exits (its output
+ * rows are then unwritten); svdq_w4a16_poll_status reports it.
  * Range: the divided activation x / s is rounded to f16, not kept as bf16.
  * Magnitudes above 65504 saturate to +-65504 and magnitudes below 2^-14 lose
  * bits (f16 subnormals, zero below 2^-25); between them f16 keeps 3 more bits
@@ -424,6 +447,13 @@ SVDQ_API svdq_status svdq_w4a16_linear(const svdq_w4a16* layer, const void* X, i
  * SVDQ_EXPORT_INV_LAMBDA float [K] (1/s), SVDQ_EXPORT_SCALARS float [1] (g).
  */
 SVDQ_API svdq_status svdq_w4a16_export(const svdq_w4a16* layer, int what, void* host_dst, size_t bytes);
+
+/*
+ * Reads (and clears) the status word of an uploaded W4A16 layer on `stream`
+ * (synchronizing it): SVDQ_OK, or SVDQ_ERR_TIMEOUT if a kernel gave up a
+ * bounded wait since the last poll.
+ */
+SVDQ_API svdq_status svdq_w4a16_poll_status(const svdq_w4a16* layer, void* stream);
 
 /* Free the handle's host memory (the caller frees dev_buf). NULL is a no-op. */
 SVDQ_API void svdq_w4a16_destroy(svdq_w4a16* layer);
