@@ -819,18 +819,23 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_kernel(const __grid_constan
 // order, fold of the low-rank branch and plain epilogue as gemm_kernel; the
 // mainloop differs.  tcgen05 has no 4-bit integer MMA kind, so per group of
 // 64 inputs:
-//   * the producer copies this CTA's raw INT4 blocks of A (128 rows) and B
-//     (its 128 of the tile's 256 rows) and their bf16 scales (8.5 KB);
-//   * warps 16-19 widen them in shared memory to f16 values q s 2^e in the
-//     128-byte-swizzled K-major layout the MMA reads (q s is exact in f16 for
-//     a bf16 s, and the prescale 2^e keeps it inside f16's range);
-//   * the leader issues 4 MMAs of kind::f16 (M = 256, N = 256, K = 16) on them.
-// Inside a group of 8 inputs the widened values sit in the order 0 4 1 5 2 6 3 7
-// (two nibbles per 32-bit lane of the unpacking); A and B share that order, so
-// the sum over K is unchanged.
+//   * the producer (warp 24) copies this CTA's raw INT4 blocks of A (128 rows)
+//     and B (its 128 of the tile's 256 rows) and their bf16 scales (8.5 KB);
+//   * two groups of widening warps (16-19 and 20-23) take alternate groups of
+//     64, so two are widened at once.  Thread t widens row t of A and of B to
+//     f16 values q s 2^e (q s is exact in f16 for a bf16 s, and the prescale
+//     2^e keeps it inside f16's range): the row of A into tensor memory
+//     (tcgen05.st, the warp's own lane quarter), the row of B into the
+//     128-byte-swizzled K-major tile in shared memory;
+//   * the leader (warp 25) issues 4 MMAs of kind::f16 (M = 256, N = 256,
+//     K = 16), A from tensor memory and B from shared memory.
+// A in tensor memory keeps 32 KB per stage (the widened A written and read
+// back) off shared memory.  Inside a group of 8 inputs the widened values sit
+// in the order 0 4 1 5 2 6 3 7 (two nibbles per 32-bit lane of the
+// unpacking); A and B share that order, so the sum over K is unchanged.
 constexpr int kStages4 = 4;
-constexpr int kConvWarp0 = 16;  // warps 16-19 widen the codes
-constexpr uint32_t kOffA4 = 0;                           // f16 A: 128 rows x 64 (16 KB)
+constexpr int kConvWarp0 = 16;  // warps 16-23 widen the codes, in two groups of 4
+constexpr uint32_t kOffA4 = 0;                           // the fold's lr' chunk (16 KB)
 constexpr uint32_t kOffB4 = kHalf * kRowBytes;           // f16 B: this CTA's 128 rows x 64 (16 KB)
 constexpr uint32_t kOffRawA4 = 2 * kHalf * kRowBytes;    // INT4 block of A (4 KB)
 constexpr uint32_t kOffRawB4 = kOffRawA4 + kBlock4Bytes;  // INT4 block of B (4 KB)
@@ -838,8 +843,10 @@ constexpr uint32_t kOffSA4 = kOffRawB4 + kBlock4Bytes;   // 128 bf16 scales of A
 constexpr uint32_t kOffSB4 = kOffSA4 + kScale4Bytes;     // 128 bf16 scales of B
 constexpr uint32_t kRaw4Bytes = 2 * kBlock4Bytes + 2 * kScale4Bytes;
 constexpr uint32_t kStage4 = (kOffSB4 + kScale4Bytes + 1023u) & ~1023u;  // 41 KB
-constexpr int kFullArrivals4 = 1 + 2 * 4;  // leader producer + the widening warps of both CTAs
-constexpr uint32_t kTmemCols4 = 256;
+constexpr int kFullArrivals4 = 1 + 2 * 4;  // leader producer + one widening group of both CTAs
+constexpr int kThreads4 = 832, kProducerWarp4 = 24, kMmaWarp4 = 25;  // 16 epilogue + 8 widening + 2
+constexpr uint32_t kTmemCols4 = 512;  // accumulator 256 + A of 4 stages x 32
+constexpr uint32_t kColA4 = 256;
 constexpr uint32_t kY4 = (kStages4 * kStage4 + kCtrl2 + kBiasBytes + 1023u) & ~1023u;
 constexpr uint32_t kEnd4 = kY4 + kEpiWarps * 2 * kYBufBytes;
 static_assert(kStage4 % 1024 == 0, "stage must keep 1 KB alignment");
@@ -895,7 +902,43 @@ __device__ __forceinline__ void widen_int4_row(const uint8_t* raw, const uint8_t
   }
 }
 
-__global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_constant__ GemmMaps maps,
+// The same widening into 32 registers (64 f16 values of row t, pairs in the smem order) for a
+// tensor-memory store: register 4 i + j holds inputs 8 i + j (low) and 8 i + j + 4 (high).
+__device__ __forceinline__ void widen_int4_row_regs(const uint8_t* raw, const uint8_t* sc, float pre, uint32_t t,
+                                                    uint32_t* out) {
+  const uint4 c0 = *reinterpret_cast<const uint4*>(raw + t * 16u);
+  const uint4 c1 = *reinterpret_cast<const uint4*>(raw + 2048u + t * 16u);
+  const uint32_t sb = *reinterpret_cast<const uint16_t*>(sc + t * 2u);
+  const float s = fminf(__uint_as_float(sb << 16) * pre, 9357.0f);
+  uint32_t s2;
+  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(s2) : "f"(s));
+  const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  constexpr uint32_t kMask = 0x000F000Fu, kMagic = 0x64086408u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t w = words[i];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t h = kMagic ^ ((w >> (4 * j)) & kMask);
+      uint32_t q;
+      asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(q) : "r"(h), "r"(kMagic));
+      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(out[4 * i + j]) : "r"(q), "r"(s2));
+    }
+  }
+}
+
+// D (+)= A(tensor memory) B(shared memory)^T, both CTAs of the pair, kind::f16.
+__device__ __forceinline__ void umma_f16_tmem_a_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads4, 1) gemm_int4_kernel(const __grid_constant__ GemmMaps maps,
                                                                  const Int4Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
@@ -928,7 +971,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_co
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp4) {
     tmem_alloc_pair(ctrl_s + 120u, kTmemCols4);
     tmem_relinquish_pair();
   }
@@ -955,7 +998,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_co
     nt = in / gsize;
   };
 
-  if (warp == kProducerWarp) {
+  if (warp == kProducerWarp4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&maps.lr);
@@ -1007,7 +1050,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_co
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kMmaWarp4) {
     // ------------------------------------------------------ MMA issue (leader)
     if (leader && lane == 0) {
       const uint32_t id_f16 = idesc_f16_m256(kBN), id_bf16 = idesc_bf16_m256(kBN);
@@ -1030,8 +1073,8 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_co
           const uint32_t st = sbase + s * kStage4;
 #pragma unroll
           for (uint32_t kk = 0; kk < 4; ++kk)
-            umma_bf16_pair(tmem, sdesc_sw128(st + kOffA4 + 32u * kk), sdesc_sw128(st + kOffB4 + 32u * kk), id_f16,
-                           (c | int(kk)) ? 1u : 0u);
+            umma_f16_tmem_a_pair(tmem, tmem + kColA4 + 32u * s + 8u * kk, sdesc_sw128(st + kOffB4 + 32u * kk), id_f16,
+                                 (c | int(kk)) ? 1u : 0u);
           tc_commit_pair_mc(EMPTY + 8u * s, kPairMask);
           any = true;
           ++it;
@@ -1063,14 +1106,20 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_co
       }
     }
     __syncwarp();
-  } else if (warp >= kConvWarp0) {  // warps 16-19
+  } else if (warp >= kConvWarp0) {  // warps 16-23
     // ---------------------------------------------------- widening warps
-    const uint32_t t = uint32_t(warp - kConvWarp0) * 32u + uint32_t(lane);  // row of A and of B
+    const uint32_t t = uint32_t((warp - kConvWarp0) & 3) * 32u + uint32_t(lane);  // row of A and of B
+    const uint32_t lanes = (uint32_t((warp - kConvWarp0) & 3) * 32u) << 16;  // this warp's lane quarter
+    const uint32_t grp = uint32_t(warp - kConvWarp0) >> 2;  // group 0 takes the even stages, group 1 the odd
     uint32_t it = 0;
     bool stop = false;
     for (int tile = pair; tile < ntiles && !stop; tile += npairs) {
       for (int k = 0; k < p.KG + nlr && !stop; ++k) {
         const uint32_t s = it % kStages4, ph = (it / kStages4) & 1u;
+        if ((it & 1u) != grp) {
+          ++it;
+          continue;
+        }
         bool ok = mbar_wait(RAW + 8u * s, ph, abort_flag, p.timeout_ns);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (!ok) {
@@ -1080,9 +1129,15 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_co
         }
         if (k < p.KG) {
           uint8_t* st = smem + s * kStage4;
-          widen_int4_row(st + kOffRawA4, st + kOffSA4, p.pre_a, st + kOffA4, t);
+          {
+            uint32_t a[32];
+            widen_int4_row_regs(st + kOffRawA4, st + kOffSA4, p.pre_a, t, a);
+            tmem_st32(tmem + lanes + kColA4 + 32u * s, a);
+          }
           widen_int4_row(st + kOffRawB4, st + kOffSB4, p.pre_w, st + kOffB4, t);
+          tmem_wait_st();
           fence_proxy_async_smem();  // generic writes -> tensor-core reads
+          tc_fence_before();
         }
         __syncwarp();
         // the peer's warps arrive remotely at CTA scope, as the NVFP4 scale warps do (an arrive
@@ -1155,7 +1210,7 @@ __global__ void __launch_bounds__(kThreads2, 1) gemm_int4_kernel(const __grid_co
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   cluster_sync();  // both CTAs are done with every MMA, copy and tensor-memory read
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp4) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, kTmemCols4);
   }
@@ -1384,7 +1439,7 @@ cudaError_t launch_gemm_int4(const Int4GemmLaunch& a, cudaStream_t s, const char
     }
     cudaLaunchConfig_t q{};
     q.gridDim = dim3(2 * unsigned(a.num_sms / 2), 1, 1);
-    q.blockDim = dim3(kThreads2, 1, 1);
+    q.blockDim = dim3(kThreads4, 1, 1);
     q.dynamicSmemBytes = smem;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -1405,7 +1460,7 @@ cudaError_t launch_gemm_int4(const Int4GemmLaunch& a, cudaStream_t s, const char
   const int pairs = int(ntiles < cap ? ntiles : cap);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(unsigned(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(kThreads2, 1, 1);
+  cfg.blockDim = dim3(kThreads4, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
