@@ -284,6 +284,52 @@ def oracle_throughput(spec, budget_s, min_steps=1, max_rows=None, steps=None, wa
 
 
 # --------------------------------------------------------------- our arm
+def flux_layer_point(spec, device, steps):
+    """Kernel 1 and kernel 2 times of one FLUX-sized layer (its rank plus any LoRA rank), graph-timed over
+    rotating buffer sets larger than L2, with kernel 2's fraction of the FP4 roofline: the extra keys of
+    the bench line that carry the larger layers next to the headline one."""
+    import torch
+
+    from bit_w4a4_quantized_b200 import svdq
+    from bit_w4a4_quantized_b200 import workloads as WL
+
+    M, K, N = spec.M, spec.K, spec.N
+    X = WL.make_x(M, K, spec.seed, spec.x_dist, spec.x_outliers, spec.x_outlier_scale)
+    amax = svdq.calibrate_amax(X)
+    r = spec.rank + (spec.lora_rank or 0)  # an adapter only adds ranks to the branch
+    L0 = svdq.Layer(spec.w(), amax, r, bias=spec.b(), device=device)
+    epi = svdq.EPI_GELU_TANH if spec.gelu else svdq.EPI_NONE
+    Xd = torch.from_numpy(X.view(np.uint16).astype(np.int16)).view(torch.bfloat16).to(device)
+    per_set = L0.device_bytes + L0.act_buffer_bytes(M) + 2 * M * K + 2 * M * N
+    nsets = int(min(8, max(2, math.ceil(3 * L2_BYTES / per_set))))
+    layers = [L0] + [L0.clone(device=device) for _ in range(nsets - 1)]
+    Xs = [Xd] + [Xd.clone() for _ in range(nsets - 1)]
+    acts = [L.new_act_buffer(M) for L in layers]
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(nsets):
+            layers[i].quantize_act(Xs[i], acts[i])
+            layers[i].linear(acts[i], M, out=Ys[i], epilogue=epi)
+        stream.synchronize()
+    k1 = _capture([lambda i=i: layers[i].quantize_act(Xs[i], acts[i]) for i in range(nsets)], stream)
+    k2 = _capture([lambda i=i: layers[i].linear(acts[i], M, out=Ys[i], epilogue=epi) for i in range(nsets)], stream)
+    t1 = _graph_seconds(k1, nsets, steps, stream, device)
+    t2 = _graph_seconds(k2, nsets, steps, stream, device)
+    for L in layers:
+        L.poll_status()
+    bf16_peak, _, peak_src = measured_peaks()
+    fp4 = 2 * M * N * K
+    roof_s = fp4 / (4.0 * bf16_peak * 1e12) + 2 * M * N * r / (bf16_peak * 1e12)
+    out = {"M": M, "K": K, "N": N, "rank_total": r, "act_quant_us": round(t1 * 1e6, 3),
+           "gemm_us": round(t2 * 1e6, 3), "gemm_TFLOPs": round(fp4 / t2 / 1e12, 1),
+           "gemm_frac_of_roofline": round(roof_s / t2, 4), "peak_basis": f"{peak_src} bf16 x 4 (FP4)"}
+    del k1, k2
+    for L in layers:
+        L.close()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -407,7 +453,7 @@ def run_ours(args):
     # end to end through the public API with host buffers (pinned): every step copies its X in
     # and its Y out inside the timed region, double-buffered so both directions of the link and
     # the kernels overlap (svdq.HostPipeline)
-    e2e_steps = max(3, min(args.steps, 30))
+    e2e_steps = max(3, min(args.steps, 100))  # the first copy in and the last copy out are not overlapped
     pipe = svdq.HostPipeline(layers[0], M, epilogue=epi)
     Xh = [Xd.cpu().pin_memory() for _ in range(2)]
     Yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -476,6 +522,13 @@ def run_ours(args):
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_flux_layers:
+        # kernel 2 on the larger FLUX layers too (outside the timed region)
+        del step_graphs, k1_graphs, k2_graphs
+        step_graphs = k1_graphs = k2_graphs = None
+        torch.cuda.empty_cache()
+        out["flux_layers"] = {s.name: flux_layer_point(s, device, 30)
+                              for s in (WL.CFG3_FC1, WL.CFG3_FC2, WL.CFG4)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, el, done, rows, threads = oracle_throughput(spec, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -868,6 +921,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-flux-layers", action="store_true",
+                    help="skip the extra per-layer kernel times of the larger FLUX layers")
     ap.add_argument("--sweep", default=None,
                     help="per-shape report instead of the bench line: 'all', 'sweep', 'w4a16', 'mlp' or workload names, "
                          "comma separated")
