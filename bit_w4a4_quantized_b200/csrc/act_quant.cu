@@ -600,13 +600,14 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   // the split count is planned once per device and shape (it queries the runtime's cluster occupancy)
   using PlanKey = std::tuple<int, int64_t, int32_t, int32_t, int>;
   static std::mutex plan_mu;
-  static std::map<PlanKey, int> planned;
+  static std::map<PlanKey, std::pair<int, size_t>> planned;  // split count, least shared memory
   const PlanKey key{dev, ag.MT, p.KC, a.r_tot, a.num_sms};
   int cached = 0;
+  size_t min_smem = 0;
   {
     std::lock_guard<std::mutex> lk(plan_mu);
     auto it = planned.find(key);
-    if (it != planned.end()) cached = it->second;
+    if (it != planned.end()) cached = it->second.first, min_smem = it->second.second;
   }
   plan(1, &smem, &push, &rows_per, &rb_bytes);
   const int per_sm = smem <= 113 * 1024 ? 2 : 1;
@@ -628,6 +629,39 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
     }
     const int cap = nonportable[dev & 63].load() > 0 ? kMaxPushSplits : kMaxSplits;
     if (splits > cap) splits = cap;
+    // Short K (at most 64 chunks): the largest cluster whose clusters of all row tiles are
+    // resident with one CTA per SM, launched with shared memory enough to keep two CTAs off an
+    // SM.  Fewer, longer splits on SMs of their own beat two CTAs per SM here (the cluster's
+    // slowest CTA sets the reduction's end); long K keeps the two-per-SM plan below.
+    int one_sm = 0;
+    if (p.KC <= 64) {
+      constexpr size_t kOneSm = 116 * 1024;
+      for (int s = cap; s >= 2 && one_sm == 0; --s) {
+        plan(s, &smem, &push, &rows_per, &rb_bytes);
+        if (!push && s > kMaxSplits) continue;
+        const size_t sm = smem < kOneSm ? kOneSm : smem;
+        if (sm > size_t(227) * 1024) continue;
+        if (set_smem(act_quant_kernel<false>, 0, sm) != cudaSuccess) break;
+        cudaLaunchConfig_t q{};
+        q.gridDim = dim3(unsigned(s), unsigned(ag.MT), 1);
+        q.blockDim = dim3(kThreads1, 1, 1);
+        q.dynamicSmemBytes = sm;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = unsigned(s);
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        q.attrs = at;
+        q.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, act_quant_kernel<false>, &q) == cudaSuccess &&
+            int64_t(clusters) >= ag.MT) {
+          one_sm = s;
+          min_smem = sm;
+        }
+      }
+    }
+    if (one_sm > 0) splits = 1;  // skip the two-per-SM search
     for (; splits > 1; --splits) {
       plan(splits, &smem, &push, &rows_per, &rb_bytes);
       if (!push && splits > kMaxSplits) continue;  // pulled partials: at most a portable cluster
@@ -652,13 +686,15 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
           int64_t(clusters) >= ag.MT)
         break;
     }
+    if (one_sm > 0) splits = one_sm;
   }
   if (cached == 0) {
     std::lock_guard<std::mutex> lk(plan_mu);
     if (planned.size() > 4096) planned.clear();
-    planned[key] = splits;
+    planned[key] = {splits, min_smem};
   }
   plan(splits, &smem, &push, &rows_per, &rb_bytes);
+  if (smem < min_smem) smem = min_smem;
   p.splits = splits;
   p.push = push;
   p.rows_per = rows_per;

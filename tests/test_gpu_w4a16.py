@@ -44,22 +44,25 @@ def test_parity(M, K, N, with_s, with_bias):
     ref = W4.prepare(W.astype(np.float32), s=s, bias=None if b is None else b.astype(np.float32))
     want = W4.linear(ref, X.astype(np.float32))
     err = assert_y_close(y_to_f64(Y), want)
+    L.poll_status()
     print(f"W4A16 M{M} K{K} N{N}: max rel err {err:.2e}")
 
 
 @pytest.mark.parametrize("M,K,N", [(3, 4096, 200), (1, 12288, 40), (8, 12288, 40), (9, 12288, 17)])
 def test_largest_k_and_several_passes_over_k(M, K, N):
-    """K above 3072 takes each warp through K in several passes of 6 tiles
-    (K = 4096: a partial second pass); K = 12288 is the largest K the layer
-    takes, and 8 rows of it the largest shared-memory request (196 KB).  Nine
-    rows run as one 8-row launch on the tensor cores and one 1-row launch on the
-    CUDA cores."""
+    """K above 3072 takes each row tile through several stages of the weight ring
+    (48 tiles of 16 x 64 per stage; K = 4096: a partial second stage); K = 12288
+    is the largest K the layer takes, and 8 rows of it the largest shared-memory
+    request (x~ 196 KB, one CTA per SM with a ring of smaller stages).  Nine rows
+    run as one 8-row launch on the tensor cores and one 1-row launch on the CUDA
+    cores.  No bounded wait may have given up."""
     X, W, s, b = _case(M, K, N, 51 + M, True, True)
     L = svdq.W4A16Layer(W, s=s, bias=b, device="cuda")
     Y = L.linear(_dev(X))
     torch.cuda.synchronize()
     ref = W4.prepare(W.astype(np.float32), s=s, bias=b.astype(np.float32))
     assert_y_close(y_to_f64(Y), W4.linear(ref, X.astype(np.float32)))
+    L.poll_status()
 
 
 @pytest.mark.parametrize("M", [1, 2, 4])
