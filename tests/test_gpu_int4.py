@@ -171,3 +171,36 @@ def test_int4_fused_epilogues_are_refused():
     with pytest.raises(svdq.SvdqError) as e:
         case.layer.linear_qkv_norm_rope(act, M, nq, nq, rope)
     assert e.value.status == svdq.ERR_INVALID_ARGUMENT and "NVFP4" in str(e.value)
+
+
+def test_int4_zero_rows_give_the_bias():
+    """All-zero rows: every group's scale is 0 and every code 0 (oracle and kernel alike), so Y is the bias."""
+    spec = WL.CFG1
+    X = spec.x()
+    X[5:70] = 0
+    case = Int4Case(X, spec.w(), spec.rank, bias=WL.make_bias(spec.N, 3))
+    act, Y = case.run()
+    ref = case.check_act(act)
+    assert np.all(ref.codes[5:70] == 0) and np.all(ref.scales[5:70] == 0)
+    case.check_y(Y, ref)
+
+
+def test_int4_inputs_far_above_calibration_stay_finite():
+    """The kernel's f16 operand holds q s 2^e_a with e_a set from the calibration maximum; a row 1000 times
+    above it saturates there (a documented limit of the INT4 path) and must not turn into inf or NaN.
+    Rows inside the range still match the oracle."""
+    spec = WL.CFG1
+    X = spec.x()
+    case = Int4Case(X, spec.w(), spec.rank)
+    Xbig = X.astype(np.float32)
+    Xbig[3] *= 1000.0
+    Xd = torch.from_numpy(WL.to_bf16(Xbig).view(np.uint16).astype(np.int16)).view(torch.bfloat16).cuda()
+    act = case.layer.quantize_act(Xd)
+    Y = case.layer.linear(act, Xd.shape[0])
+    torch.cuda.synchronize()
+    y = y_to_f64(Y)
+    assert np.all(np.isfinite(y))
+    rows = np.array([r for r in range(X.shape[0]) if r != 3])
+    ref = I4.quantize_act(case.ref, WL.to_bf16(Xbig).astype(np.float32)[rows])
+    assert_y_close(y[rows], I4.linear(case.ref, ref))
+    case.layer.poll_status()
