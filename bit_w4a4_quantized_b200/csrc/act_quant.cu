@@ -636,7 +636,8 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
     int one_sm = 0;
     if (p.KC <= 64) {
       constexpr size_t kOneSm = 116 * 1024;
-      for (int s = cap; s >= 2 && one_sm == 0; --s) {
+      // every CTA needs a chunk of its own: at most KC splits
+      for (int s = cap < p.KC ? cap : int(p.KC); s >= 2 && one_sm == 0; --s) {
         plan(s, &smem, &push, &rows_per, &rb_bytes);
         if (!push && s > kMaxSplits) continue;
         const size_t sm = smem < kOneSm ? kOneSm : smem;
