@@ -874,13 +874,16 @@ __host__ __device__ constexpr uint32_t idesc_f16_m256(int n) {
 
 // Row t of a 128-row INT4 block and its bf16 scale -> 64 f16 values q s pre,
 // written as row t of a 128-byte-swizzled K-major tile.  The scale saturates
-// at 65504 / 7, so no value overflows to infinity.
+// at 9352, the largest f16 value whose sevenfold stays finite in f16 (7 x 9352
+// rounds to 65472): a clamp at 65504 / 7 itself would round up to 9360 in f16,
+// and 7 x 9360 = 65520 rounds to infinity.  So no value overflows.
+constexpr float kMaxWideScale4 = 9352.0f;  // largest f16 s with 7 s finite in f16
 __device__ __forceinline__ void widen_int4_row(const uint8_t* raw, const uint8_t* sc, float pre, uint8_t* dst,
                                                uint32_t t) {
   const uint4 c0 = *reinterpret_cast<const uint4*>(raw + t * 16u);          // inputs 0..31
   const uint4 c1 = *reinterpret_cast<const uint4*>(raw + 2048u + t * 16u);  // inputs 32..63
   const uint32_t sb = *reinterpret_cast<const uint16_t*>(sc + t * 2u);
-  const float s = fminf(__uint_as_float(sb << 16) * pre, 9357.0f);
+  const float s = fminf(__uint_as_float(sb << 16) * pre, kMaxWideScale4);
   uint32_t s2;
   asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(s2) : "f"(s));
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -909,7 +912,7 @@ __device__ __forceinline__ void widen_int4_row_regs(const uint8_t* raw, const ui
   const uint4 c0 = *reinterpret_cast<const uint4*>(raw + t * 16u);
   const uint4 c1 = *reinterpret_cast<const uint4*>(raw + 2048u + t * 16u);
   const uint32_t sb = *reinterpret_cast<const uint16_t*>(sc + t * 2u);
-  const float s = fminf(__uint_as_float(sb << 16) * pre, 9357.0f);
+  const float s = fminf(__uint_as_float(sb << 16) * pre, kMaxWideScale4);
   uint32_t s2;
   asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(s2) : "f"(s));
   const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};

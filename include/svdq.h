@@ -85,8 +85,9 @@ typedef struct svdq_layer svdq_layer; /* opaque host handle of one prepared laye
  *     shared memory and runs the f16 MMA; e is a per-layer power of two (e_a
  *     for X_hat from the calibration maximum, e_w for R), reported as
  *     g_a = 2^-e_a and g_w = 2^-e_w.  Inputs whose |X_hat| exceeds 32 times the
- *     calibration maximum saturate in that operand (a scale above 65504 / 7
- *     after the prescale is clamped there).  The fused QKV and MLP entry points
+ *     calibration maximum saturate in that operand (a scale above 9352, the
+ *     largest f16 value whose sevenfold stays finite, after the prescale is
+ *     clamped there).  The fused QKV and MLP entry points
  *     take NVFP4 layers only.
  */
 enum { SVDQ_FMT_NVFP4 = 1, SVDQ_FMT_INT4 = 2 };
