@@ -10,15 +10,17 @@
 // and lr' = bf16((x_hat L1) / (g_a g_w)) on the tensor cores.
 //
 // Design (sm_100a):
-//   * CTA = 128 rows of X x a slice of K.  Warp 8 streams X chunks of 128 rows
-//     x 64 columns with a 2D TMA load (128-byte swizzle), the matching
-//     1/lambda slice and L1^T chunk with bulk copies, through a 4-stage
-//     mbarrier ring.
-//   * Warps 0-7: two threads per row convert 32 elements each in shared
-//     memory, write x_hat back in place (it is the A operand of the MMA),
-//     and store codes and block scales straight into the GEMM's tiled layout.
-//   * Warp 9: one thread issues tcgen05.mma kind::f16 (M = 128, N = rank)
-//     accumulating X_hat L1 in tensor memory.
+//   * CTA = 128 rows of X x a slice of K.  The producer warp streams X chunks
+//     of 128 rows x 64 columns with a 2D TMA load (128-byte swizzle), the
+//     matching 1/lambda slice and L1^T chunk with bulk copies, through an
+//     mbarrier ring (4 stages with two CTAs per SM, 6 or 8 with one).
+//   * Converter warps (one group of 8 with two CTAs per SM, two groups taking
+//     alternate chunks with one): two threads per row convert 32 elements
+//     each in shared memory, write x_hat back in place (it is the A operand
+//     of the MMA), and store codes and block scales straight into the GEMM's
+//     tiled layout.
+//   * The MMA warp: one thread issues tcgen05.mma kind::f16 (M = 128,
+//     N = rank) accumulating X_hat L1 in tensor memory.
 //   * K is split across the CTAs of a cluster so that enough CTAs stream HBM;
 //     their partial X_hat L1 tiles are summed in a fixed order through
 //     distributed shared memory (no global scratch, deterministic).
@@ -42,15 +44,18 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kStages1 = 4;
-constexpr int kThreads1 = 320;  // warps 0-7 convert, 8 produce, 9 issue MMAs
-constexpr int kConvThreads = 256;
-constexpr int kProducerWarp1 = 8, kMmaWarp1 = 9;
+// S stages and G groups of eight converter warps (group g takes the chunks i with i % G == g),
+// then the producer warp and the MMA warp.  S = 4 has one group and runs two CTAs per SM; the
+// one-CTA-per-SM instances (S = 6 or 8) have two groups, and S is even, so that a stage's chunks
+// always belong to one group.
+constexpr int kConvThreads = 256;  // one group
+__host__ __device__ constexpr int groups1(int stages) { return stages == 4 ? 1 : 2; }
+__host__ __device__ constexpr int threads1(int stages) { return 32 * (8 * groups1(stages) + 2); }
+constexpr uint32_t ctrl_bytes1(int stages) { return 32u * uint32_t(stages) + 512u; }  // barriers + reciprocal table
 constexpr int kMaxSplits = 8;       // pulled partials: a portable cluster
 constexpr int kMaxPushSplits = 16;  // pushed partials: up to the non-portable cluster size
 constexpr uint32_t kXBytes = kBM * 128;  // 16 KB: 128 rows x 64 bf16
 constexpr uint32_t kInvSlot = 1024;      // 64 floats of 1/lambda (256 B), padded for alignment
-constexpr uint32_t kCtrlBytes = 128 + 512;  // + the block-reciprocal table
 
 struct ActQuantParams {
   const float* inv_lam;  // [KC * 64]
@@ -162,9 +167,12 @@ __device__ __forceinline__ void store_lr8(const ActQuantParams& p, int mt, uint3
 // that allocates tensor memory runs one CTA per SM, the plain quantizer two.
 // kInt4 selects the INT4 quantizer (groups of 64, bf16 scales) for the NVFP4 one;
 // the smoothing, the down projection and its reduction are the same.
-template <bool kLowRank, bool kInt4 = false>
-__global__ void __launch_bounds__(kThreads1, 2)
+template <bool kLowRank, bool kInt4 = false, int kS = 4>
+__global__ void __launch_bounds__(threads1(kS), kS == 4 ? 2 : 1)
     act_quant_kernel(const __grid_constant__ CUtensorMap tmap_x, const ActQuantParams p) {
+  constexpr int kG = groups1(kS);
+  static_assert(kS % kG == 0, "a stage's chunks must belong to one converter group");
+  constexpr int kProducerWarp1 = 8 * kG, kMmaWarp1 = 8 * kG + 1;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_s & 1023u)) & 1023u;
@@ -179,21 +187,25 @@ __global__ void __launch_bounds__(kThreads1, 2)
   constexpr bool lowrank = kLowRank;
 
   // [stages][receive buffer of pushed partials: splits x rows_per x r_tot floats][control]
-  const uint32_t rb_s = sbase + kStages1 * p.stage_bytes;
-  const float* rb = reinterpret_cast<const float*>(smem + kStages1 * p.stage_bytes);
-  uint8_t* ctrl = smem + kStages1 * p.stage_bytes + p.rb_bytes;
-  const uint32_t ctrl_s = sbase + kStages1 * p.stage_bytes + p.rb_bytes;
-  const uint32_t FULL = ctrl_s, CONV = ctrl_s + 32u, EMPTY = ctrl_s + 64u;
-  const uint32_t ACCF = ctrl_s + 96u, DRAIN = ctrl_s + 104u;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 112);
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 116);
-  const uint32_t RECV = ctrl_s + 120u;  // the pushed partials of this CTA's rows have landed
+  const uint32_t rb_s = sbase + kS * p.stage_bytes;
+  const float* rb = reinterpret_cast<const float*>(smem + kS * p.stage_bytes);
+  uint8_t* ctrl = smem + kS * p.stage_bytes + p.rb_bytes;
+  const uint32_t ctrl_s = sbase + kS * p.stage_bytes + p.rb_bytes;
+  // control block: FULL, CONV, EMPTY [kS] each, ACCF, DRAIN, the tensor-memory slot, the abort
+  // flag, RECV; the block-reciprocal table at 32 kS
+  constexpr uint32_t kB = 8u * kS;
+  const uint32_t FULL = ctrl_s, CONV = ctrl_s + kB, EMPTY = ctrl_s + 2u * kB;
+  const uint32_t ACCF = ctrl_s + 3u * kB, DRAIN = ACCF + 8u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 3u * kB + 16u);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(ctrl + 3u * kB + 20u);
+  const uint32_t RECV = ctrl_s + 3u * kB + 24u;  // the pushed partials of this CTA's rows have landed
+  float* rtab = reinterpret_cast<float*>(ctrl + 4u * kB);
   const int crank = kLowRank && p.splits > 1 ? int(cluster_ctarank()) : 0;
   const int own0 = crank * p.rows_per;
   const int own1 = own0 + p.rows_per < kBM ? own0 + p.rows_per : kBM;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages1; ++s) {
+    for (int s = 0; s < kS; ++s) {
       mbar_init(FULL + 8u * s, 1);
       mbar_init(CONV + 8u * s, kConvThreads);
       mbar_init(EMPTY + 8u * s, 1);
@@ -210,10 +222,10 @@ __global__ void __launch_bounds__(kThreads1, 2)
   // shared-memory load per block instead of decoding s and a correctly rounded reciprocal
   if (threadIdx.x < 128) {
     const float d = __fmul_rn(e4m3_value(threadIdx.x), p.g_a);
-    reinterpret_cast<float*>(ctrl + 128)[threadIdx.x] = (d == 0.0f || threadIdx.x == 127u) ? 0.0f : __frcp_rn(d);
+    rtab[threadIdx.x] = (d == 0.0f || threadIdx.x == 127u) ? 0.0f : __frcp_rn(d);
   }
   if (warp == kMmaWarp1 && lowrank) {
-    tmem_alloc(ctrl_s + 112u, p.tmem_cols);
+    tmem_alloc(ctrl_s + 3u * kB + 16u, p.tmem_cols);
     tmem_relinquish();
   }
   if (lowrank) tc_fence_before();
@@ -238,8 +250,8 @@ __global__ void __launch_bounds__(kThreads1, 2)
       const uint32_t tx = kXBytes + 256u + (lowrank ? uint32_t(p.r_tot) * 128u : 0u);
       int issued = 0;
       for (int i = 0; i < nchunks; ++i) {
-        const int s = i % kStages1;
-        const uint32_t ph = uint32_t(i / kStages1) & 1u;
+        const int s = i % kS;
+        const uint32_t ph = uint32_t(i / kS) & 1u;
         if (!mbar_wait(EMPTY + 8u * s, ph ^ 1u, abort_flag, p.timeout_ns)) {
           fail(0x1u);
           break;
@@ -255,20 +267,20 @@ __global__ void __launch_bounds__(kThreads1, 2)
         issued = i + 1;
       }
       // every issued copy must land before this CTA may exit
-      for (int i = issued > kStages1 ? issued - kStages1 : 0; i < issued; ++i)
-        mbar_wait(FULL + 8u * (i % kStages1), uint32_t(i / kStages1) & 1u, nullptr, p.timeout_ns);
+      for (int i = issued > kS ? issued - kS : 0; i < issued; ++i)
+        mbar_wait(FULL + 8u * (i % kS), uint32_t(i / kS) & 1u, nullptr, p.timeout_ns);
     }
     __syncwarp();
-  } else if (kInt4 && warp < 8) {
+  } else if (kInt4 && warp < 8 * kG) {
     // ------------------------------------------------------ INT4 converters
     // two threads per row, neighbours in a warp: thread (t, h) converts
     // elements 32 h .. 32 h + 31 of row t; the chunk is one group of 64, whose
     // amax the pair shares
-    const uint32_t t = uint32_t(warp) * 16u + (uint32_t(lane) >> 1), h = uint32_t(lane) & 1u;
+    const uint32_t t = uint32_t(warp & 7) * 16u + (uint32_t(lane) >> 1), h = uint32_t(lane) & 1u;
     const uint32_t t7 = t & 7u;
-    for (int i = 0; i < nchunks; ++i) {
-      const int s = i % kStages1;
-      const uint32_t ph = uint32_t(i / kStages1) & 1u;
+    for (int i = warp >> 3; i < nchunks; i += kG) {
+      const int s = i % kS;
+      const uint32_t ph = uint32_t(i / kS) & 1u;
       bool ok = mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns);
       ok = __all_sync(0xFFFFFFFFu, ok);  // the pair's shuffle below needs the whole warp
       if (!ok) {
@@ -294,15 +306,15 @@ __global__ void __launch_bounds__(kThreads1, 2)
       if (lowrank) fence_proxy_async_smem();  // x_hat (generic writes) -> tensor-core reads
       mbar_arrive(CONV + 8u * s);
     }
-  } else if (warp < 8) {
+  } else if (warp < 8 * kG) {
     // ----------------------------------------------------------- converters
     // two threads per row: thread (t, h) converts elements 32 h .. 32 h + 31
     // of row t of each 64-column chunk (two 16-element blocks)
-    const uint32_t t = threadIdx.x & 127u, h = threadIdx.x >> 7;
+    const uint32_t t = threadIdx.x & 127u, h = (threadIdx.x >> 7) & 1u;
     const uint32_t t7 = t & 7u;
-    for (int i = 0; i < nchunks; ++i) {
-      const int s = i % kStages1;
-      const uint32_t ph = uint32_t(i / kStages1) & 1u;
+    for (int i = warp >> 3; i < nchunks; i += kG) {
+      const int s = i % kS;
+      const uint32_t ph = uint32_t(i / kS) & 1u;
       if (!mbar_wait(FULL + 8u * s, ph, abort_flag, p.timeout_ns)) {
         fail(0x2u);
         break;
@@ -314,7 +326,7 @@ __global__ void __launch_bounds__(kThreads1, 2)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int g = int(2 * h) + j;
-        quant_block(xrow, t7, g, inv + 16 * g, reinterpret_cast<const float*>(ctrl + 128), p.c_a, lowrank, cw[2 * j],
+        quant_block(xrow, t7, g, inv + 16 * g, rtab, p.c_a, lowrank, cw[2 * j],
                     cw[2 * j + 1], sc[j]);
       }
       const int kc = kc0 + i, kt = kc >> 2, sub = kc & 3;
@@ -331,8 +343,8 @@ __global__ void __launch_bounds__(kThreads1, 2)
       bool any = false;
       const uint32_t idesc = idesc_bf16(p.r_tot);
       for (int i = 0; i < nchunks; ++i) {
-        const int s = i % kStages1;
-        const uint32_t ph = uint32_t(i / kStages1) & 1u;
+        const int s = i % kS;
+        const uint32_t ph = uint32_t(i / kS) & 1u;
         if (!mbar_wait(CONV + 8u * s, ph, abort_flag, p.timeout_ns)) {
           fail(0x4u);
           break;
@@ -564,13 +576,11 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   p.timeout_ns = a.timeout_ns;
 
   const bool lowrank = a.r_tot > 0;
-  auto kernel = a.int4 ? (lowrank ? act_quant_kernel<true, true> : act_quant_kernel<false, true>)
-                       : (lowrank ? act_quant_kernel<true> : act_quant_kernel<false>);
   int dev = 0;
   cudaGetDevice(&dev);
   auto set_smem = [&](auto k, int which, size_t bytes) -> cudaError_t {
     // the attributes are per device and kernel: remember the largest size set on each
-    static std::atomic<size_t> smem_set[4][64];
+    static std::atomic<size_t> smem_set[8][64];
     std::atomic<size_t>& done = smem_set[which][dev & 63];
     if (bytes <= done.load()) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
@@ -584,9 +594,9 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   // is asked of the rank-0 instance, which has the same resources but no
   // tensor-memory allocation (for which the calculator assumes one CTA per SM,
   // while clusters of this kernel run two per SM).
-  auto plan = [&](int sp, size_t* smem_out, int* push_out, int* rows_out, uint32_t* rb_out) {
+  auto plan = [&](int sp, int stages, size_t* smem_out, int* push_out, int* rows_out, uint32_t* rb_out) {
     const int rows = (kBM + sp - 1) / sp;
-    const size_t base = size_t(kStages1) * p.stage_bytes + kCtrlBytes + 1024;
+    const size_t base = size_t(stages) * p.stage_bytes + ctrl_bytes1(stages) + 1024;
     const size_t rb = lowrank && sp > 1 ? size_t(round_up(int64_t(sp) * rows * a.r_tot * 4, 1024)) : 0;
     const bool push = rb > 0 && (base + rb <= 113 * 1024 || (base > 113 * 1024 && base + rb <= 227 * 1024));
     *push_out = push ? 1 : 0;
@@ -600,16 +610,17 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   // the split count is planned once per device and shape (it queries the runtime's cluster occupancy)
   using PlanKey = std::tuple<int, int64_t, int32_t, int32_t, int>;
   static std::mutex plan_mu;
-  static std::map<PlanKey, std::pair<int, size_t>> planned;  // split count, least shared memory
+  // split count, stages, least shared memory
+  static std::map<PlanKey, std::tuple<int, int, size_t>> planned;
   const PlanKey key{dev, ag.MT, p.KC, a.r_tot, a.num_sms};
-  int cached = 0;
+  int cached = 0, stages = 4;
   size_t min_smem = 0;
   {
     std::lock_guard<std::mutex> lk(plan_mu);
     auto it = planned.find(key);
-    if (it != planned.end()) cached = it->second.first, min_smem = it->second.second;
+    if (it != planned.end()) std::tie(cached, stages, min_smem) = it->second;
   }
-  plan(1, &smem, &push, &rows_per, &rb_bytes);
+  plan(1, 4, &smem, &push, &rows_per, &rb_bytes);
   const int per_sm = smem <= 113 * 1024 ? 2 : 1;
   int splits = cached > 0 ? cached : int((int64_t(per_sm) * a.num_sms) / ag.MT);
   const int max_splits = lowrank ? kMaxPushSplits : 64;
@@ -625,27 +636,40 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
         e = cudaFuncSetAttribute(act_quant_kernel<true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(act_quant_kernel<true, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(act_quant_kernel<true, false, 8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(act_quant_kernel<true, true, 8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(act_quant_kernel<true, false, 6>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(act_quant_kernel<true, true, 6>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       nonportable[dev & 63].store(e == cudaSuccess ? 1 : -1);
     }
     const int cap = nonportable[dev & 63].load() > 0 ? kMaxPushSplits : kMaxSplits;
     if (splits > cap) splits = cap;
     // Short K (at most 64 chunks): the largest cluster whose clusters of all row tiles are
     // resident with one CTA per SM, launched with shared memory enough to keep two CTAs off an
-    // SM.  Fewer, longer splits on SMs of their own beat two CTAs per SM here (the cluster's
-    // slowest CTA sets the reduction's end); long K keeps the two-per-SM plan below.
+    // SM, and with two converter groups and eight stages (six where eight do not fit) so that
+    // the SM keeps as many converter warps and loads in flight as two CTAs would.  Fewer, longer splits on SMs of their own beat
+    // two CTAs per SM here (the cluster's slowest CTA sets the reduction's end); long K keeps
+    // the two-per-SM plan below.
     int one_sm = 0;
     if (p.KC <= 64) {
       constexpr size_t kOneSm = 116 * 1024;
       // every CTA needs a chunk of its own: at most KC splits
       for (int s = cap < p.KC ? cap : int(p.KC); s >= 2 && one_sm == 0; --s) {
-        plan(s, &smem, &push, &rows_per, &rb_bytes);
+        int st = 8;
+        plan(s, st, &smem, &push, &rows_per, &rb_bytes);
+        if (smem > size_t(227) * 1024) plan(s, st = 6, &smem, &push, &rows_per, &rb_bytes);
         if (!push && s > kMaxSplits) continue;
         const size_t sm = smem < kOneSm ? kOneSm : smem;
         if (sm > size_t(227) * 1024) continue;
-        if (set_smem(act_quant_kernel<false>, 0, sm) != cudaSuccess) break;
+        auto qk = st == 8 ? act_quant_kernel<true, false, 8> : act_quant_kernel<true, false, 6>;
+        if (set_smem(qk, st == 8 ? 4 : 6, sm) != cudaSuccess) break;
         cudaLaunchConfig_t q{};
         q.gridDim = dim3(unsigned(s), unsigned(ag.MT), 1);
-        q.blockDim = dim3(kThreads1, 1, 1);
+        q.blockDim = dim3(threads1(st), 1, 1);
         q.dynamicSmemBytes = sm;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeClusterDimension;
@@ -655,16 +679,16 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
         q.attrs = at;
         q.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, act_quant_kernel<false>, &q) == cudaSuccess &&
-            int64_t(clusters) >= ag.MT) {
+        if (cudaOccupancyMaxActiveClusters(&clusters, qk, &q) == cudaSuccess && int64_t(clusters) >= ag.MT) {
           one_sm = s;
           min_smem = sm;
+          stages = st;
         }
       }
     }
     if (one_sm > 0) splits = 1;  // skip the two-per-SM search
     for (; splits > 1; --splits) {
-      plan(splits, &smem, &push, &rows_per, &rb_bytes);
+      plan(splits, 4, &smem, &push, &rows_per, &rb_bytes);
       if (!push && splits > kMaxSplits) continue;  // pulled partials: at most a portable cluster
       cudaError_t e = set_smem(act_quant_kernel<false>, 0, smem);
       if (e != cudaSuccess) {
@@ -673,7 +697,7 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
       }
       cudaLaunchConfig_t q{};
       q.gridDim = dim3(unsigned(splits), unsigned(ag.MT), 1);
-      q.blockDim = dim3(kThreads1, 1, 1);
+      q.blockDim = dim3(threads1(4), 1, 1);
       q.dynamicSmemBytes = smem;
       cudaLaunchAttribute at[1];
       at[0].id = cudaLaunchAttributeClusterDimension;
@@ -692,16 +716,21 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   if (cached == 0) {
     std::lock_guard<std::mutex> lk(plan_mu);
     if (planned.size() > 4096) planned.clear();
-    planned[key] = {splits, min_smem};
+    planned[key] = {splits, stages, min_smem};
   }
-  plan(splits, &smem, &push, &rows_per, &rb_bytes);
+  plan(splits, stages, &smem, &push, &rows_per, &rb_bytes);
   if (smem < min_smem) smem = min_smem;
   p.splits = splits;
   p.push = push;
   p.rows_per = rows_per;
   p.rb_bytes = rb_bytes;
+  auto kernel = stages == 8 ? (a.int4 ? act_quant_kernel<true, true, 8> : act_quant_kernel<true, false, 8>)
+                : stages == 6 ? (a.int4 ? act_quant_kernel<true, true, 6> : act_quant_kernel<true, false, 6>)
+                : a.int4      ? (lowrank ? act_quant_kernel<true, true> : act_quant_kernel<false, true>)
+                              : (lowrank ? act_quant_kernel<true> : act_quant_kernel<false>);
+  const int slot = stages == 4 ? (lowrank ? 1 : 0) + (a.int4 ? 2 : 0) : (stages == 8 ? 4 : 6) + (a.int4 ? 1 : 0);
   {
-    cudaError_t e = set_smem(kernel, (lowrank ? 1 : 0) + (a.int4 ? 2 : 0), smem);
+    cudaError_t e = set_smem(kernel, slot, smem);
     if (e != cudaSuccess) {
       *why = "cudaFuncSetAttribute(shared memory size / carveout) failed";
       return e;
@@ -709,7 +738,7 @@ cudaError_t launch_act_quant(const ActQuantLaunch& a, cudaStream_t s, const char
   }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(unsigned(splits), unsigned(ag.MT), 1);
-  cfg.blockDim = dim3(kThreads1, 1, 1);
+  cfg.blockDim = dim3(threads1(stages), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
