@@ -19,11 +19,12 @@
 // split each row tile's K (tile kt goes to warp kt % 8), read their operands
 // from the stage, and add their partial sums through shared memory in a fixed
 // order, summed by a warp that rotates with the row tile (the partial-sum
-// buffer alternates with the tile, so one barrier per tile suffices).  With one row of X the MMA would be 7/8 padding, so that launch does
-// the same tiles on the CUDA cores instead: mixed-precision fused multiply-adds
-// (f16 operands, float32 accumulator) straight from the f16 weights, no
-// conversion to float32.  Every wait is bounded: a timeout sets the layer's
-// status word and the CTA drains its copies and exits.
+// buffer alternates with the tile, so one barrier per tile suffices).  One row
+// of X runs the same MMA path: the MMA is then 7/8 padding, but it does the
+// mixed-precision multiply-adds in one instruction per 256 weights, which the
+// CUDA cores would spend one instruction per weight on.  Every wait is
+// bounded: a timeout sets the layer's status word and the CTA drains its
+// copies and exits.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -135,50 +136,17 @@ __device__ __forceinline__ void tile_mma(float* acc, uint4 cw, uint2 sw, const u
   }
 }
 
-// acc + x.lo w.lo + x.hi w.hi with f16 operands and a float32 accumulator
-// (exact products, float32 sums).
-__device__ __forceinline__ float fma2_f16_f32(uint32_t x2, uint32_t w2, float acc) {
-  asm("{\n .reg .f16 xl, xh, wl, wh;\n mov.b32 {xl, xh}, %1;\n mov.b32 {wl, wh}, %2;\n"
-      " fma.rn.f32.f16 %0, xl, wl, %0;\n fma.rn.f32.f16 %0, xh, wh, %0;\n}"
-      : "+f"(acc)
-      : "r"(x2), "r"(w2));
-  return acc;
+// Two bf16 inputs (one word) divided by their s (times 1/s), saturated to f16's range and
+// rounded to f16: one word of x~.
+__device__ __forceinline__ uint32_t x_tilde2(uint32_t xb, float is_lo, float is_hi) {
+  const float lo = fminf(fmaxf(__uint_as_float(xb << 16) * is_lo, -65504.0f), 65504.0f);
+  const float hi = fminf(fmaxf(__uint_as_float(xb & 0xFFFF0000u) * is_hi, -65504.0f), 65504.0f);
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// The same 16 x 64 tile on the CUDA cores, for kM <= 2 rows of X (the MMA's 8
-// columns would be mostly padding): lane (g, c) adds its 16 weights of rows g
-// (acc[0][m]) and g + 8 (acc[1][m]) times x~; xs: x~ rows as f16 pairs, at the
-// tile's first input.
-template <int kM>
-__device__ __forceinline__ void tile_dot(float (*acc)[kM], uint4 cw, uint2 sw, const uint32_t* xs, uint32_t RW,
-                                         int c) {
-  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-  uint32_t sg[2], sg8[2];  // scales of rows g and g + 8: steps {0, 1}, {2, 3}
-  e4m3x4_to_f16x2(sw.x, sg[0], sg[1]);
-  e4m3x4_to_f16x2(sw.y, sg8[0], sg8[1]);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    uint32_t h[4];
-    e2m1x8_to_f16x2(words[j], h);
-    const uint32_t s0 = dup_half(sg[j >> 1], j & 1);   // row g
-    const uint32_t s1 = dup_half(sg8[j >> 1], j & 1);  // row g + 8
-    const uint32_t a0 = hmul2(h[0], s0);  // row g, inputs 16 j + 2 c, + 1
-    const uint32_t a1 = hmul2(h[1], s1);  // row g + 8, the same inputs
-    const uint32_t a2 = hmul2(h[2], s0);  // row g, inputs 16 j + 2 c + 8, + 9
-    const uint32_t a3 = hmul2(h[3], s1);  // row g + 8, the same inputs
-#pragma unroll
-    for (int m = 0; m < kM; ++m) {
-      const uint32_t x0 = xs[m * RW + 8 * j + c], x1 = xs[m * RW + 8 * j + c + 4];
-      acc[0][m] = fma2_f16_f32(x1, a2, fma2_f16_f32(x0, a0, acc[0][m]));
-      acc[1][m] = fma2_f16_f32(x1, a3, fma2_f16_f32(x0, a1, acc[1][m]));
-    }
-  }
-}
-
-// kDot = 0: the MMA path (2 to 8 rows of X); kDot = 1: the CUDA-core path for one row.
 // Warps 0-7 compute, warp 8 lane 0 fills the ring.  Stage s holds `chunk` weight tiles of
 // one row tile: their codes (chunk x 512 bytes), then their scales (chunk x 64 bytes).
-template <int kDot>
 __global__ void __launch_bounds__(kThreadsW, 2) w4a16_kernel(const W4A16Params p) {
   extern __shared__ __align__(128) uint8_t smem_w[];
   const int64_t K = p.K;
@@ -240,15 +208,20 @@ __global__ void __launch_bounds__(kThreadsW, 2) w4a16_kernel(const W4A16Params p
   }
 
   // ------------------------------------------------------------- compute
-  // x~ = f16(x / s), saturating (the producer's first copies are already in flight)
-  for (uint32_t i = threadIdx.x; i < MR * uint32_t(K / 2); i += 32 * kWarpsW) {
-    const uint32_t m = i / uint32_t(K / 2), w = i % uint32_t(K / 2);
-    const uint32_t xb = *reinterpret_cast<const uint32_t*>(p.X + int64_t(m) * K + 2 * int64_t(w));
-    const float2 is = *reinterpret_cast<const float2*>(p.inv_s + 2 * int64_t(w));
-    const float lo = fminf(fmaxf(__uint_as_float(xb << 16) * is.x, -65504.0f), 65504.0f);
-    const float hi = fminf(fmaxf(__uint_as_float(xb & 0xFFFF0000u) * is.y, -65504.0f), 65504.0f);
-    const __half2 h = __floats2half2_rn(lo, hi);
-    xs[m * RW + w] = *reinterpret_cast<const uint32_t*>(&h);
+  // x~ = f16(x / s), saturating (the producer's first copies are already in flight); eight
+  // inputs per thread and step: 16-byte loads (X is 16-byte aligned, K a multiple of 64)
+  const uint32_t KV = uint32_t(K / 8);  // 16-byte vectors per row of X
+  for (uint32_t i = threadIdx.x; i < MR * KV; i += 32 * kWarpsW) {
+    const uint32_t m = i / KV, v = i % KV;
+    const uint4 xb = *reinterpret_cast<const uint4*>(p.X + int64_t(m) * K + 8 * int64_t(v));
+    const float4 s0 = *reinterpret_cast<const float4*>(p.inv_s + 8 * int64_t(v));
+    const float4 s1 = *reinterpret_cast<const float4*>(p.inv_s + 8 * int64_t(v) + 4);
+    uint4 o;
+    o.x = x_tilde2(xb.x, s0.x, s0.y);
+    o.y = x_tilde2(xb.y, s0.z, s0.w);
+    o.z = x_tilde2(xb.z, s1.x, s1.y);
+    o.w = x_tilde2(xb.w, s1.z, s1.w);
+    *reinterpret_cast<uint4*>(xs + m * RW + 4 * v) = o;
   }
   ptx::named_sync(1, 32 * kWarpsW);
 
@@ -258,7 +231,6 @@ __global__ void __launch_bounds__(kThreadsW, 2) w4a16_kernel(const W4A16Params p
   bool bad = false;
   for (int64_t nt = blockIdx.x; nt < p.NT; nt += gridDim.x) {
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    float dacc[2][kDot > 0 ? kDot : 1] = {};
     const uint32_t* xrow = uint32_t(g) < MR ? xs + uint32_t(g) * RW : nullptr;
     for (int64_t ch = 0; ch < nchunks; ++ch, ++u) {
       const uint32_t s = u % uint32_t(p.stages), ph = (u / uint32_t(p.stages)) & 1u;
@@ -280,30 +252,11 @@ __global__ void __launch_bounds__(kThreadsW, 2) w4a16_kernel(const W4A16Params p
           const uint32_t kt = uint32_t(kt0) + uint32_t(i);
           const uint4 cw = cws[i * 32 + lane];
           const uint2 sw = sws[i * 8 + g];
-          if constexpr (kDot > 0)
-            tile_dot<kDot>(dacc, cw, sw, xs + kt * 32u, RW, c);
-          else
-            tile_mma(acc, cw, sw, xrow ? xrow + kt * 32u : nullptr, c);
+          tile_mma(acc, cw, sw, xrow ? xrow + kt * 32u : nullptr, c);
         }
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(EMPTY + 8u * s);  // this warp is done with the stage
       }
-    }
-    if constexpr (kDot > 0) {
-      // the 4 lanes of a row group hold disjoint inputs: add them (lane c = 0 keeps the sums), then lay
-      // the result out as the MMA accumulator would hold it: lane (g, c) row g (x, y), row g + 8 (z, w),
-      // X rows 2 c, 2 c + 1
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int m = 0; m < kDot; ++m) {
-          dacc[h][m] += __shfl_xor_sync(0xFFFFFFFFu, dacc[h][m], 1);
-          dacc[h][m] += __shfl_xor_sync(0xFFFFFFFFu, dacc[h][m], 2);
-        }
-      acc[0] = c == 0 ? dacc[0][0] : 0.0f;
-      acc[2] = c == 0 ? dacc[1][0] : 0.0f;
-      acc[1] = (c == 0 && kDot > 1) ? dacc[0][kDot > 1 ? 1 : 0] : 0.0f;
-      acc[3] = (c == 0 && kDot > 1) ? dacc[1][kDot > 1 ? 1 : 0] : 0.0f;
     }
     // the 8 warps' partial tiles, added in warp order by one warp (rotating); the buffer
     // alternates with the row tile, so one barrier per tile suffices
@@ -341,7 +294,6 @@ __global__ void __launch_bounds__(kThreadsW, 2) w4a16_kernel(const W4A16Params p
 // attribute and occupancy calls cost microseconds of host time; a launch
 // should not).  The carveout asks for all of the unified L1 as shared memory,
 // or the driver may size it for one CTA.
-template <int kDot>
 int blocks_per_sm(size_t smem) {
   static std::atomic<int64_t> cached_key[64];
   static std::atomic<int> cached_val[64];
@@ -349,12 +301,12 @@ int blocks_per_sm(size_t smem) {
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   const int64_t key = int64_t(smem) + 1;
   if (cached_key[dev & 63].load() == key) return cached_val[dev & 63].load();
-  if (cudaFuncSetAttribute(w4a16_kernel<kDot>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
-      cudaFuncSetAttribute(w4a16_kernel<kDot>, cudaFuncAttributePreferredSharedMemoryCarveout,
+  if (cudaFuncSetAttribute(w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(w4a16_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                            int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
     return 0;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, w4a16_kernel<kDot>, kThreadsW, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, w4a16_kernel, kThreadsW, smem) != cudaSuccess)
     return 0;
   cached_val[dev & 63].store(per_sm);
   cached_key[dev & 63].store(key);
@@ -411,17 +363,14 @@ cudaError_t launch_w4a16(const W4A16Launch& a, cudaStream_t s, const char** why)
     p.off_red = uint32_t(xs_bytes);
     p.off_ring = uint32_t(xs_bytes + red_bytes);
     p.off_ctrl = uint32_t(xs_bytes + red_bytes + size_t(p.stages) * size_t(p.chunk) * (kTileCodeBytes + kTileScaleBytes));
-    const int per_sm = p.M == 1 ? blocks_per_sm<1>(smem) : blocks_per_sm<0>(smem);
+    const int per_sm = blocks_per_sm(smem);
     if (per_sm < 1) {
       *why = "the W4A16 kernel does not fit on this device";
       return cudaErrorInvalidConfiguration;
     }
     int64_t blocks = int64_t(per_sm) * a.num_sms;
     if (blocks > p.NT) blocks = p.NT;
-    if (p.M == 1)  // one row of X: the CUDA cores (the MMA's 8 columns would be 7/8 padding)
-      w4a16_kernel<1><<<unsigned(blocks), kThreadsW, smem, s>>>(p);
-    else
-      w4a16_kernel<0><<<unsigned(blocks), kThreadsW, smem, s>>>(p);
+    w4a16_kernel<<<unsigned(blocks), kThreadsW, smem, s>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       *why = "launch of the W4A16 kernel failed";
