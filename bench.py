@@ -169,6 +169,7 @@ class ClockSampler:
 
 
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}  # an earlier measurement on the same B200 pool
+FALLBACK_BF16_SUSTAINED = 1400.0  # the same GEMM back to back under the 1000 W cap (about 1.3 GHz)
 
 
 def measured_peaks():
@@ -197,6 +198,28 @@ def measured_peaks():
     else:
         origin = "measured, fallback for " + ", ".join(fell_back)
     return out[0], out[1], origin
+
+
+def sustained_bf16_peak():
+    """(bf16 TFLOP/s, origin) of a GEMM kept busy for seconds under the power cap, from
+    MEASURED_PEAKS.json (`bf16_tflops_sustained`), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            v = json.load(fh).get("bf16_tflops_sustained")
+    except (OSError, ValueError, AttributeError):
+        v = None
+    if isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0:
+        return float(v), "measured"
+    return FALLBACK_BF16_SUSTAINED, "fallback"
+
+
+def power_capped(clocks):
+    """True when the clock samples of the timed region show the power cap holding the SM clock
+    below its maximum: the kernels then run at the sustained rate, not the burst one."""
+    if not clocks or "sw_power_cap" not in clocks.get("reasons", []):
+        return False
+    mhz, top = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    return mhz is not None and top is not None and mhz < top - 15
 
 
 KERNEL_SOURCES = {
@@ -475,8 +498,14 @@ def run_ours(args):
     value = aggregate(2 * M * N * K * args.steps, world, t_step_max) / 1e12
     e2e_value = aggregate(2 * M * N * K * e2e_steps, world, t_e2e) / 1e12
 
-    # roofline of the dominant kernel
+    # roofline of the dominant kernel: the burst bf16 peak, or the sustained one when the power
+    # cap held the clock down during the timed region
     bf16_peak, hbm_peak, peak_src = measured_peaks()
+    bf16_src = f"{peak_src} burst"
+    clocks = clk.summary()
+    if power_capped(clocks):
+        bf16_peak, src = sustained_bf16_peak()
+        bf16_src = f"{src} sustained"
     fp4_peak = bf16_peak * 4.0  # dense FP4 / BF16 nominal ratio (9 / 2.25 PFLOP/s)
     per_k2 = t_k2 / args.steps
     per_k1 = t_k1 / args.steps
@@ -490,7 +519,7 @@ def run_ours(args):
                 "traffic_source": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture "
                                   "(profiles/gemm_kernel_attention_projection.md); Y stays in L2 during the kernel"}
         roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["peak_basis"] = (f"{peak_src} bf16 {bf16_peak} TF/s x 4 (nominal FP4:BF16) for the FP4 flops, "
+        roof["peak_basis"] = (f"{bf16_src} bf16 {bf16_peak} TF/s x 4 (nominal FP4:BF16) for the FP4 flops, "
                               f"bf16 {bf16_peak} TF/s for the fold")
     else:
         roof = {"kernel": "act_quant (kernel 1)", "bound": "hbm", "achieved": k1_bytes / per_k1 / 1e9,
@@ -498,7 +527,6 @@ def run_ours(args):
                 "peak_basis": f"{peak_src} HBM copy"}
         roof["frac"] = roof["achieved"] / roof["peak"]
 
-    clocks = clk.summary()
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step_max / args.steps * 1e3, 5), "higher_is_better": True,
@@ -915,8 +943,8 @@ def relaunch(args, argv):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")

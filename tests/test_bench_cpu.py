@@ -81,6 +81,20 @@ def test_measured_peaks_fall_back_per_value(tmp_path, monkeypatch):
     assert bench.measured_peaks() == (1590.0, 6650.0, "fallback")
 
 
+def test_sustained_peak_and_power_cap_rule(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.sustained_bf16_peak() == (1400.0, "fallback")  # no file
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"bf16_tflops": 1666.4, "bf16_tflops_sustained": 1363.8}')
+    assert bench.sustained_bf16_peak() == (1363.8, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").write_text("[]")
+    assert bench.sustained_bf16_peak() == (1400.0, "fallback")
+    # the sustained peak applies only when the power cap held the median clock below its maximum
+    assert bench.power_capped({"sm_mhz": 1893.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]})
+    assert not bench.power_capped({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]})
+    assert not bench.power_capped({"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": []})
+    assert not bench.power_capped({})
+
+
 def test_clock_summary_keeps_the_benchmarked_gpu_under_load():
     c = bench.ClockSampler(uuid="GPU-bbbb")
     c.lines = [
