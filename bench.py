@@ -891,7 +891,9 @@ def run_reference(args):
     if rank != 0:
         return 0  # the oracle runs on the host of rank 0 only
     spec = workload_spec(args.workload)
-    budget = args.cpu_budget
+    # every step is a sample of the workload's rows; the budget spreads over all steps, so it is
+    # larger than the cpu_baseline's, or a 2000-step run would time one-row calls (call overhead)
+    budget = args.ref_budget
     v, el, done, rows, threads = oracle_throughput(spec, budget, steps=args.steps, warmup=args.warmup)
     out = {
         "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": world,
@@ -948,6 +950,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of CPU oracle work")
+    ap.add_argument("--ref-budget", type=float, default=60.0,
+                    help="seconds of CPU oracle work for --impl reference (spread over --steps + --warmup)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flux-layers", action="store_true",
                     help="skip the extra per-layer kernel times of the larger FLUX layers")
