@@ -90,8 +90,11 @@ def run_ring(S, G, nchunks, seed, max_steps=200000):
     raise AssertionError("the model did not settle")
 
 
-@pytest.mark.parametrize("S,G", [(4, 1), (8, 2), (6, 2)])
+@pytest.mark.parametrize("S,G", [(4, 1), (8, 2), (6, 2), (4, 2)])
 def test_kernel_layouts_never_read_a_stale_stage(S, G):
+    """(4, 1), (8, 2), (6, 2): the activation kernel's instances.  (4, 2): the INT4 GEMM's ring,
+    whose two widening groups take alternate stages the same way (they wait for the landed codes,
+    widen them and arrive on the stage's barrier for the MMA thread)."""
     for nchunks in list(range(1, 20)) + [24, 48, 64]:
         for seed in range(40):
             done, bad = run_ring(S, G, nchunks, seed=1000 * nchunks + seed)
